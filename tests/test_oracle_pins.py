@@ -1,0 +1,453 @@
+"""Pins for the fp64 oracle against facts it does not compute itself.
+
+Each test fixes the oracle to something independent of its own code: a textbook or library
+routine (torch CPU scaled_dot_product_attention and autograd in fp64), a pure-Python brute
+force on tiny grids, closed forms of the rotary embedding, invariants of softmax and RoPE,
+or numerical derivatives.  None of these needs a GPU.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import Grid
+from synth import WORKLOADS, bf16_bits_to_f64, make_raster_inputs
+
+pytestmark = pytest.mark.filterwarnings("ignore::UserWarning")
+
+
+def _grid(w):
+    return Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t)
+
+
+def _inputs(name):
+    w = WORKLOADS[name]
+    x = make_raster_inputs(w, with_grad=True)
+    return w, {k: (bf16_bits_to_f64(v) if v is not None and v.dtype == np.uint16 else v)
+               for k, v in x.items()}
+
+
+def _sdpa(q, k, v, scale, mask=None, need_grad=False):
+    """torch CPU fp64 SDPA on raster [B, N, H, D] arrays; mask [B, H, N, Nk] bool (True = keep)."""
+    tq, tk, tv = (torch.tensor(a.transpose(0, 2, 1, 3).copy(), dtype=torch.float64,
+                               requires_grad=need_grad) for a in (q, k, v))
+    m = None if mask is None else torch.tensor(mask)
+    o = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=m, scale=scale)
+    return o, (tq, tk, tv)
+
+
+# ------------------------------------------------------------------ layout / geometry
+def test_slot_map_matches_block_members():
+    for name in ("tiny", "tiny_ragged", "small", "small_b2"):
+        g = _grid(WORKLOADS[name])
+        sm = g.slot_map(g.t_frames)
+        mem = g.block_members(g.t_frames)
+        for b in range(g.nbq):
+            valid = [int(x) for x in sm[b] if x >= 0]
+            assert valid == mem[b]
+        # every token appears exactly once
+        allv = np.sort(sm[sm >= 0])
+        assert np.array_equal(allv, np.arange(g.t_frames * g.grid_h * g.grid_w))
+
+
+def test_workload_geometry_matches_pages():
+    """Golden geometry: latent grid and block counts of the measured workloads."""
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(__file__), "golden", "geometry.json")) as f:
+        gold = json.load(f)
+    for name, rec in gold["workloads"].items():
+        w = WORKLOADS[name]
+        assert [w.t_frames + w.cached_t, w.grid_h, w.grid_w] == rec["latent_grid"]
+        nbq, nbc = w.n_blocks()
+        assert nbq + nbc == rec["key_blocks"]
+        assert nbq == rec["query_blocks"]
+        assert w.top_r == rec["top_r"]
+        assert abs(w.top_r / (nbq + nbc) - rec["density"]) < 5e-3
+
+
+# ------------------------------------------------------------------ prologue pins
+def test_rope_closed_form_small_head():
+    """D = 12: split (4, 4, 4), theta = 10000.  Hand-worked angles at position (1, 2, 3):
+    t pairs turn by 1 and 0.01 rad, h pairs by 2 and 0.02, w pairs by 3 and 0.03."""
+    assert oracle.rope_split(12) == (4, 4, 4)
+    x = np.zeros((1, 1, 1, 12))
+    x[..., 0::2] = 1.0  # every pair = (1, 0)
+    y = oracle.rope3d(x, np.array([1.0]), np.array([2.0]), np.array([3.0]), 10000.0)
+    angles = [1.0, 0.01, 2.0, 0.02, 3.0, 0.03]
+    for p, a in enumerate(angles):
+        assert y[0, 0, 0, 2 * p] == pytest.approx(math.cos(a), abs=1e-15)
+        assert y[0, 0, 0, 2 * p + 1] == pytest.approx(math.sin(a), abs=1e-15)
+
+
+def test_rope_split_head128():
+    assert oracle.rope_split(128) == (44, 42, 42)
+    assert oracle.rope_split(64) == (24, 20, 20)
+
+
+def test_rope_position_zero_is_identity_and_norm_preserving():
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((1, 6, 3, 128))
+    z = np.zeros(6)
+    assert np.array_equal(oracle.rope3d(x, z, z, z, 10000.0), x)
+    pos = rng.integers(0, 90, size=(3, 6)).astype(np.float64)
+    y = oracle.rope3d(x, pos[0], pos[1], pos[2], 10000.0)
+    pn_x = x[..., 0::2] ** 2 + x[..., 1::2] ** 2
+    pn_y = y[..., 0::2] ** 2 + y[..., 1::2] ** 2
+    np.testing.assert_allclose(pn_y, pn_x, rtol=1e-12, atol=1e-12)
+
+
+def test_rope_relative_position_per_axis():
+    """q(m) . k(n) depends only on m - n along each axis."""
+    rng = np.random.default_rng(7)
+    q = rng.standard_normal((1, 1, 1, 128))
+    k = rng.standard_normal((1, 1, 1, 128))
+
+    def dot(m, n):
+        a = oracle.rope3d(q, *[np.array([float(c)]) for c in m], 10000.0)
+        b = oracle.rope3d(k, *[np.array([float(c)]) for c in n], 10000.0)
+        return float(np.sum(a * b))
+    base = dot((5, 7, 11), (2, 3, 4))
+    assert dot((3, 4, 7), (0, 0, 0)) == pytest.approx(base, rel=1e-11, abs=1e-11)
+    assert dot((20, 30, 40), (17, 26, 33)) == pytest.approx(base, rel=1e-11, abs=1e-11)
+    assert dot((5, 7, 11), (2, 3, 5)) != pytest.approx(base, rel=1e-6)
+
+
+def test_rmsnorm_unit_rms_and_commutes_with_rope():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((1, 10, 2, 128)) * 3.0
+    g1 = np.ones(128)
+    y = oracle.rms_norm(x, g1, 1e-6)
+    np.testing.assert_allclose(np.sqrt(np.mean(y * y, axis=-1)), 1.0, rtol=1e-6)
+    t, h, w = oracle.grid_positions(1, 2, 5, t_offset=3)
+    a = oracle.rope3d(oracle.rms_norm(x, g1, 1e-6), t, h, w, 10000.0)
+    b = oracle.rms_norm(oracle.rope3d(x, t, h, w, 10000.0), g1, 1e-6)
+    np.testing.assert_allclose(a, b, rtol=1e-12, atol=1e-12)
+    # a gain scales channels after normalisation
+    gam = rng.standard_normal(128)
+    np.testing.assert_allclose(oracle.rms_norm(x, gam, 1e-6), y * gam, rtol=1e-12)
+
+
+def test_prologue_positions_follow_raster_order():
+    """Token n of a (T, Hg, Wg) raster sits at (n // (Hg Wg), (n // Wg) % Hg, n % Wg)."""
+    t, h, w = oracle.grid_positions(3, 4, 5, t_offset=2)
+    n = np.arange(60)
+    assert np.array_equal(t, n // 20 + 2)
+    assert np.array_equal(h, (n // 5) % 4)
+    assert np.array_equal(w, n % 5)
+
+
+# ------------------------------------------------------------------ routing pins
+def _brute_route(q, k, grid, r):
+    """Pure-Python scalar routing on tiny grids (loops only)."""
+    B, N, H, D = q.shape
+    mem = grid.block_members(grid.t_frames)
+    idx_all, cnt_all = {}, {}
+    for b in range(B):
+        for h in range(H):
+            means = []
+            for arr in (q, k):
+                ms = []
+                for toks in mem:
+                    ms.append([sum(float(arr[b, t, h, d]) for t in toks) / len(toks)
+                               for d in range(D)])
+                means.append(ms)
+            for i in range(grid.nbq):
+                sc = []
+                for j in range(grid.nbk):
+                    s = sum(means[0][i][d] * means[1][j][d] for d in range(D))
+                    if grid.chunk_t and grid.key_block_chunk(j) > grid.query_block_chunk(i):
+                        s = -math.inf
+                    sc.append(s)
+                chosen = []
+                left = list(range(grid.nbk))
+                while len(chosen) < r:
+                    best = None
+                    for j in left:
+                        if sc[j] == -math.inf:
+                            continue
+                        if best is None or sc[j] > sc[best]:
+                            best = j  # strict '>' keeps the lower index on ties
+                    if best is None:
+                        break
+                    chosen.append(best)
+                    left.remove(best)
+                idx_all[(b, h, i)] = sorted(chosen)
+                cnt_all[(b, h, i)] = len(chosen)
+    return idx_all, cnt_all
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_ragged"])
+def test_route_brute_force(name):
+    w, x = _inputs(name)
+    g = _grid(w)
+    idx, cnt, _ = oracle.route(x["q"], x["k"], g, w.top_r)
+    bi, bc = _brute_route(x["q"], x["k"], g, w.top_r)
+    for key, sel in bi.items():
+        b, h, i = key
+        assert cnt[b, h, i] == bc[key]
+        assert list(idx[b, h, i, :cnt[b, h, i]]) == sel
+        assert all(v == -1 for v in idx[b, h, i, cnt[b, h, i]:])
+
+
+def test_route_brute_force_causal():
+    g = Grid(8, 4, 4, (2, 4, 4), chunk_t=4)
+    rng = np.random.default_rng(3)
+    q = rng.standard_normal((1, 128, 1, 8))
+    k = rng.standard_normal((1, 128, 1, 8))
+    idx, cnt, _ = oracle.route(q, k, g, 3)
+    bi, bc = _brute_route(q, k, g, 3)
+    for (b, h, i), sel in bi.items():
+        assert list(idx[b, h, i, :cnt[b, h, i]]) == sel and cnt[b, h, i] == bc[(b, h, i)]
+    # query blocks 0,1 (chunk 0) may only see key blocks 0,1: cnt = 2 < r
+    assert list(cnt[0, 0]) == [2, 2, 3, 3]
+    assert list(idx[0, 0, 0]) == [0, 1, -1]
+
+
+def test_route_exact_ties_lower_index_wins():
+    g = Grid(2, 4, 16, (2, 4, 4))  # 4 blocks along w
+    rng = np.random.default_rng(11)
+    q = rng.standard_normal((1, 128, 1, 16))
+    k = rng.standard_normal((1, 128, 1, 16))
+    mem = g.block_members(2)
+    k[0, mem[3]] = k[0, mem[1]]  # blocks 1 and 3 identical -> equal scores for every query
+    _, _, s = oracle.route(q, k, g, 1)
+    for i in range(4):
+        assert s[0, 0, i, 1] == s[0, 0, i, 3]
+    # force blocks 1 and 3 to be the two largest, so r = 1 must pick block 1
+    q[0, :] = 0.0
+    q[0, mem[0]] = k[0, mem[1]].mean(axis=0)
+    idx, cnt, s = oracle.route(q, k, g, 1)
+    assert s[0, 0, 0, 1] == s[0, 0, 0, 3]
+    assert idx[0, 0, 0, 0] == 1
+
+
+def test_route_proportional_block_ranks_first():
+    g = Grid(4, 8, 8, (2, 4, 4))
+    rng = np.random.default_rng(13)
+    k = rng.standard_normal((1, 256, 1, 64))
+    mem = g.block_members(4)
+    kbar5 = k[0, mem[5], 0].mean(axis=0)
+    q = rng.standard_normal((1, 256, 1, 64)) * 1e-3
+    q[0, mem[2], 0] += 10.0 * kbar5  # query block 2 is aligned with key block 5
+    _, _, s = oracle.route(q, k, g, 8)
+    assert int(np.argmax(s[0, 0, 2])) == 5
+
+
+def test_route_all_blocks_when_r_equals_nb():
+    w, x = _inputs("tiny")
+    g = _grid(w)
+    idx, cnt, _ = oracle.route(x["q"], x["k"], g, g.nbk)
+    assert np.all(cnt == g.nbk)
+    assert np.array_equal(idx[0, 0, 3], np.arange(g.nbk))
+
+
+def test_route_causal_never_selects_later_chunk():
+    w, x = _inputs("small_cont")
+    g = _grid(w)
+    idx, cnt, s = oracle.route(x["q"], x["k"], g, w.top_r, k_cache=x["kc"])
+    for i in range(g.nbq):
+        for j in idx[0, 0, i]:
+            if j >= 0:
+                assert g.key_block_chunk(int(j)) <= g.query_block_chunk(i)
+    # continuation: key blocks 0..nbc-1 are cached, all cached chunks precede the queries
+    assert g.nbc == g.nbq
+
+
+def test_near_tie_rule():
+    row = np.array([0.5, 0.30000, 0.300001, 0.1, -np.inf])
+    assert oracle.near_tie_ok([0, 1], [0, 1], row)
+    assert oracle.near_tie_ok([0, 1], [0, 2], row)          # 0.3 vs 0.300001: within 1e-4
+    assert not oracle.near_tie_ok([0, 3], [0, 2], row)      # 0.1 is far from tau
+    assert not oracle.near_tie_ok([0], [0, 2], row)         # counts differ
+
+
+# ------------------------------------------------------------------ attention pins
+def _token_mask(grid, idx, B, H):
+    """Dense token-level keep mask [B, H, N, N] from block selections (current keys only)."""
+    mem = grid.block_members(grid.t_frames)
+    n = grid.t_frames * grid.grid_h * grid.grid_w
+    m = np.zeros((B, H, n, n), dtype=bool)
+    for b in range(B):
+        for h in range(H):
+            for i, qi in enumerate(mem):
+                for j in idx[b, h, i]:
+                    if j >= 0:
+                        m[b, h, np.ix_(qi, mem[j])[0], np.ix_(qi, mem[j])[1]] = True
+    return m
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_ragged", "tiny_d128"])
+def test_all_blocks_equals_dense_sdpa(name):
+    w, x = _inputs(name)
+    g = _grid(w)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    idx, _, _ = oracle.route(x["q"], x["k"], g, g.nbk)
+    o, lse = oracle.attend(x["q"], x["k"], x["v"], idx, g, scale)
+    ref, _ = _sdpa(x["q"], x["k"], x["v"], scale)
+    np.testing.assert_allclose(o, ref.detach().numpy().transpose(0, 2, 1, 3), atol=1e-12)
+    od, lsed = oracle.dense_attention(x["q"], x["k"], x["v"], scale)
+    np.testing.assert_allclose(lse, lsed, atol=1e-12)
+    # LSE against a direct log-sum-exp of the logits of one token
+    qv, kv = x["q"][0, 17, 1], x["k"][0, :, 1]
+    logits = kv @ qv * scale
+    assert lse[0, 17, 1] == pytest.approx(math.log(np.sum(np.exp(logits))), rel=1e-12)
+
+
+@pytest.mark.parametrize("name", ["tiny", "tiny_ragged"])
+def test_sparse_equals_masked_sdpa(name):
+    """Attention over the selected blocks equals dense attention with every other key masked
+    (torch's boolean mask gives masked keys exactly zero weight)."""
+    w, x = _inputs(name)
+    g = _grid(w)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    idx, _, _ = oracle.route(x["q"], x["k"], g, w.top_r)
+    o, _ = oracle.attend(x["q"], x["k"], x["v"], idx, g, scale)
+    mask = _token_mask(g, idx, w.batch, w.heads)
+    ref, _ = _sdpa(x["q"], x["k"], x["v"], scale, mask=mask)
+    np.testing.assert_allclose(o, ref.detach().numpy().transpose(0, 2, 1, 3), atol=1e-12)
+
+
+def _brute_attend_token(q, k, v, idx_row, grid, b, h, n, scale):
+    mem = grid.block_members(grid.t_frames)
+    keys = [t for j in idx_row if j >= 0 for t in mem[j]]
+    logits = [scale * sum(q[b, n, h, d] * k[b, t, h, d] for d in range(q.shape[-1])) for t in keys]
+    m = max(logits)
+    e = [math.exp(z - m) for z in logits]
+    s = sum(e)
+    out = [sum(e[a] / s * v[b, t, h, d] for a, t in enumerate(keys)) for d in range(q.shape[-1])]
+    return out, m + math.log(s), [z / s for z in e]
+
+
+def test_attend_brute_force_tokens():
+    w, x = _inputs("tiny_ragged")
+    g = _grid(w)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    idx, _, _ = oracle.route(x["q"], x["k"], g, w.top_r)
+    o, lse, probs = oracle.attend(x["q"], x["k"], x["v"], idx, g, scale, return_probs=True)
+    mem = g.block_members(g.t_frames)
+    for (b, h, i) in [(0, 0, 0), (0, 1, 3), (0, 1, g.nbq - 1)]:
+        for pos, n in enumerate(mem[i][:5]):
+            ref, ref_lse, ref_p = _brute_attend_token(x["q"], x["k"], x["v"], idx[b, h, i], g,
+                                                      b, h, n, scale)
+            np.testing.assert_allclose(o[b, n, h], ref, atol=1e-12)
+            assert lse[b, n, h] == pytest.approx(ref_lse, rel=1e-12)
+            np.testing.assert_allclose(probs[(b, h, i)][pos], ref_p, atol=1e-14)
+
+
+def test_softmax_rows_sum_to_one_and_special_values():
+    w, x = _inputs("tiny_ragged")
+    g = _grid(w)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    idx, _, _ = oracle.route(x["q"], x["k"], g, w.top_r)
+    _, _, probs = oracle.attend(x["q"], x["k"], x["v"], idx, g, scale, return_probs=True)
+    for p in probs.values():
+        assert np.max(np.abs(p.sum(axis=1) - 1.0)) < 1e-12
+        assert np.all(p >= 0)
+    # V == c gives O == c
+    vc = np.full_like(x["v"], 0.75)
+    o, _ = oracle.attend(x["q"], x["k"], vc, idx, g, scale)
+    np.testing.assert_allclose(o, 0.75, atol=1e-14)
+    # Q == 0 gives the mean of the selected valid V rows
+    o0, _ = oracle.attend(np.zeros_like(x["q"]), x["k"], x["v"], idx, g, scale)
+    mem = g.block_members(g.t_frames)
+    sel = [t for j in idx[0, 1, 2] if j >= 0 for t in mem[j]]
+    np.testing.assert_allclose(o0[0, mem[2][0], 1], x["v"][0, sel, 1].mean(axis=0), atol=1e-13)
+
+
+def test_continuation_cache_equals_full_grid():
+    """Without the causal mask, a cached run equals a plain run on the whole key grid whose
+    query rows are the last frames."""
+    w, x = _inputs("small_cont")
+    g = _grid(w)
+    gf = Grid(w.t_frames + w.cached_t, w.grid_h, w.grid_w, w.blk)  # full grid, no cache
+    g0 = Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, 0)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    kf = np.concatenate([x["kc"], x["k"]], axis=1)
+    vf = np.concatenate([x["vc"], x["v"]], axis=1)
+    nc = w.n_cached_tokens
+    qf = np.concatenate([np.zeros_like(x["kc"]), x["q"]], axis=1)
+    idx, cnt, s = oracle.route(x["q"], x["k"], g0, w.top_r, k_cache=x["kc"])
+    # same selections on the full grid: query block i of the cached run is block i + nbc
+    idx_f = -np.ones((w.batch, w.heads, gf.nbq, w.top_r), dtype=np.int32)
+    idx_f[:, :, g0.nbc:] = idx
+    o, lse = oracle.attend(x["q"], x["k"], x["v"], idx, g0, scale, k_cache=x["kc"], v_cache=x["vc"])
+    qb = [(b, h, i) for b in range(w.batch) for h in range(w.heads) for i in range(g0.nbc, gf.nbq)]
+    of, lsef = oracle.attend(qf, kf, vf, idx_f, gf, scale, query_blocks=qb)
+    np.testing.assert_allclose(o, of[:, nc:], atol=1e-12)
+    np.testing.assert_allclose(lse, lsef[:, nc:], atol=1e-12)
+    # and the routing scores on the full grid agree for the query rows
+    qbar_full = oracle.block_means(qf, gf.block_members(gf.t_frames))
+    kbar_full = oracle.block_means(kf, gf.block_members(gf.t_frames))
+    s_full = np.einsum("bhid,bhjd->bhij", qbar_full, kbar_full)
+    np.testing.assert_allclose(s, s_full[:, :, g0.nbc:], rtol=1e-12, atol=1e-14)
+    assert g.nbc == g0.nbc
+
+
+# ------------------------------------------------------------------ backward pins
+@pytest.mark.parametrize("name", ["tiny", "tiny_ragged"])
+def test_bwd_matches_torch_autograd_masked(name):
+    w, x = _inputs(name)
+    g = _grid(w)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    for r in (w.top_r, g.nbk):
+        idx, _, _ = oracle.route(x["q"], x["k"], g, r)
+        dq, dk, dv = oracle.attend_bwd(x["q"], x["k"], x["v"], x["do"], idx, g, scale)
+        mask = _token_mask(g, idx, w.batch, w.heads)
+        o, (tq, tk, tv) = _sdpa(x["q"], x["k"], x["v"], scale, mask=mask, need_grad=True)
+        tdo = torch.tensor(x["do"].transpose(0, 2, 1, 3).copy(), dtype=torch.float64)
+        (o * tdo).sum().backward()
+        for mine, t in ((dq, tq), (dk, tk), (dv, tv)):
+            np.testing.assert_allclose(mine, t.grad.numpy().transpose(0, 2, 1, 3), atol=1e-11)
+
+
+def test_bwd_finite_differences():
+    w, x = _inputs("tiny_ragged")
+    g = _grid(w)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    idx, _, _ = oracle.route(x["q"], x["k"], g, w.top_r)
+    dq, dk, dv = oracle.attend_bwd(x["q"], x["k"], x["v"], x["do"], idx, g, scale)
+    rng = np.random.default_rng(17)
+    eps = 1e-5
+
+    def loss(q, k, v):
+        o, _ = oracle.attend(q, k, v, idx, g, scale)
+        return float(np.sum(o * x["do"]))
+    for name, grad in (("q", dq), ("k", dk), ("v", dv)):
+        for _ in range(12):
+            pos = tuple(int(rng.integers(0, s)) for s in x[name].shape)
+            args = {"q": x["q"].copy(), "k": x["k"].copy(), "v": x["v"].copy()}
+            args[name][pos] += eps
+            lp = loss(args["q"], args["k"], args["v"])
+            args[name][pos] -= 2 * eps
+            lm = loss(args["q"], args["k"], args["v"])
+            num = (lp - lm) / (2 * eps)
+            assert grad[pos] == pytest.approx(num, rel=1e-6, abs=1e-8)
+
+
+def test_bwd_continuation_grads_only_reach_current_keys():
+    w, x = _inputs("small_cont")
+    g = _grid(w)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    idx, _, _ = oracle.route(x["q"], x["k"], g, w.top_r, k_cache=x["kc"])
+    dq, dk, dv = oracle.attend_bwd(x["q"], x["k"], x["v"], x["do"], idx, g, scale,
+                                   k_cache=x["kc"], v_cache=x["vc"])
+    # full-grid autograd with the cache as part of the keys; compare current-key gradients
+    nc = w.n_cached_tokens
+    gf = Grid(w.t_frames + w.cached_t, w.grid_h, w.grid_w, w.blk)
+    kf = np.concatenate([x["kc"], x["k"]], axis=1)
+    vf = np.concatenate([x["vc"], x["v"]], axis=1)
+    qf = np.concatenate([np.zeros_like(x["kc"]), x["q"]], axis=1)
+    dof = np.concatenate([np.zeros_like(x["kc"]), x["do"]], axis=1)
+    idx_f = -np.ones((w.batch, w.heads, gf.nbq, w.top_r), dtype=np.int32)
+    idx_f[:, :, g.nbc:] = idx
+    mask = _token_mask(gf, idx_f, w.batch, w.heads)
+    mask[:, :, :nc, :nc] = True  # cached query rows are discarded; keep their softmax finite
+    o, (tq, tk, tv) = _sdpa(qf, kf, vf, scale, mask=mask, need_grad=True)
+    tdo = torch.tensor(dof.transpose(0, 2, 1, 3).copy(), dtype=torch.float64)
+    (o * tdo).sum().backward()
+    np.testing.assert_allclose(dq, tq.grad.numpy().transpose(0, 2, 1, 3)[:, nc:], atol=1e-11)
+    np.testing.assert_allclose(dk, tk.grad.numpy().transpose(0, 2, 1, 3)[:, nc:], atol=1e-11)
+    np.testing.assert_allclose(dv, tv.grad.numpy().transpose(0, 2, 1, 3)[:, nc:], atol=1e-11)
