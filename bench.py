@@ -1,0 +1,347 @@
+#!/usr/bin/env python
+"""Benchmark of the BSA hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input resident in HBM:
+fused QK-RMSNorm + 3D-RoPE prologue (with block means) -> block-pooled top-r routing ->
+sparse attention forward -> sparse attention backward (with the forward's routing; dO is
+a fixed synthetic upstream gradient).  Default workload: the 720p refine stage (24x45x80
+latent tokens padded to 24x48x80, 4x4x8 blocks, top-r 72, 32 heads x 128, bf16).
+
+value    = effective TFLOP/s of the step on selected-block tile FLOPs (4*BS^2*D per
+           selected (query block, key block) pair forward, 2.5x that backward) summed over
+           all ranks / max-over-ranks step time.
+e2e      = the same metric through the public pipeline API with host (pinned) raster
+           inputs copied in and the output O copied back inside the timed region.
+roofline = the forward attention kernel against the measured dense bf16 tensor peak.
+
+Multi-GPU (torchrun): every rank runs an independent replica of the workload (the path
+has no exchange step: routing and attention are independent per (batch, head)), so
+scaling is weak; ranks meet only at the timing barriers.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import WORKLOADS, make_raster_inputs  # noqa: E402
+
+
+def tile_flops(bs: int, d: int, n_pairs: int) -> float:
+    return 4.0 * bs * bs * d * n_pairs
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) >= 9:
+                rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_oracle_sample(w, budget_s: float = 12.0):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload: routing of
+    one head plus forward attention of as many query blocks of that head as fit the budget,
+    and backward of a few; reported in TFLOP/s of the same tile-FLOP convention."""
+    import oracle
+    grid = oracle.Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t)
+    x = make_raster_inputs(w, with_grad=True)
+    from synth import bf16_bits_to_f64
+    h = 0
+    q = bf16_bits_to_f64(x["q"][:, :, h:h + 1])
+    k = bf16_bits_to_f64(x["k"][:, :, h:h + 1])
+    v = bf16_bits_to_f64(x["v"][:, :, h:h + 1])
+    do = bf16_bits_to_f64(x["do"][:, :, h:h + 1])
+    kc = bf16_bits_to_f64(x["kc"][:, :, h:h + 1]) if w.cached_t else None
+    vc = bf16_bits_to_f64(x["vc"][:, :, h:h + 1]) if w.cached_t else None
+    gq = x["gamma_q"] if w.qknorm else None
+    gk = x["gamma_k"] if w.qknorm else None
+    theta = w.theta if w.rope else 0.0
+    scale = 1.0 / np.sqrt(w.head_dim)
+    t0 = time.perf_counter()
+    qp = oracle.prologue(q, w.t_frames, w.grid_h, w.grid_w, gamma=gq, eps=w.eps, theta=theta,
+                         t_offset=w.cached_t)
+    kp = oracle.prologue(k, w.t_frames, w.grid_h, w.grid_w, gamma=gk, eps=w.eps, theta=theta,
+                         t_offset=w.cached_t)
+    idx, cnt, _ = oracle.route(qp, kp, grid, w.top_r, k_cache=kc)
+    t_route = time.perf_counter() - t0
+    n_blocks, t_attn = 0, 0.0
+    rng = np.random.default_rng(0)
+    order = rng.permutation(grid.nbq)
+    while t_attn < budget_s and n_blocks < grid.nbq:
+        i = int(order[n_blocks])
+        t1 = time.perf_counter()
+        oracle.attend(qp, kp, v, idx, grid, scale, k_cache=kc, v_cache=vc, query_blocks=[(0, 0, i)])
+        t_attn += time.perf_counter() - t1
+        n_blocks += 1
+    pairs = float(np.mean(cnt[0, 0])) * n_blocks
+    fl = tile_flops(grid.bs, w.head_dim, 1) * pairs
+    cores = len(os.sched_getaffinity(0))
+    return {
+        "value": fl / (t_attn + t_route * n_blocks / grid.nbq) / 1e12,
+        "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        "sample": f"fp64 oracle: prologue+route of 1/{w.heads} heads, forward attention of "
+                  f"{n_blocks} query blocks of that head ({pairs:.0f} block pairs); route time "
+                  f"prorated to the sampled blocks; {t_attn + t_route:.1f} s of CPU work",
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="720p", choices=["720p", "480p", "480p_cont"])
+    ap.add_argument("--no-bwd", action="store_true", help="forward path only")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = WORKLOADS[args.workload]
+    with_bwd = not args.no_bwd
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        t0 = time.perf_counter()
+        vals = [cpu_oracle_sample(w, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+                for _ in range(args.warmup + args.steps)][args.warmup:]
+        v = float(np.median([x["value"] for x in vals]))
+        cb = dict(vals[-1])
+        cb["value"] = v
+        line = {"impl": "reference", "metric": "BSA fwd(+bwd) effective TFLOP/s at 720p tokens",
+                "value": v, "unit": "TFLOP/s", "n_gpus": args.gpus, "steps": args.steps,
+                "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                "config": {"workload": args.workload, "tokens": w.n_tokens, "heads": w.heads,
+                           "head_dim": w.head_dim, "block": list(w.blk), "top_r": w.top_r},
+                "cpu_baseline": cb,
+                "e2e": {"value": v, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0},
+                "wall_s": time.perf_counter() - t0}
+        print(json.dumps(line))
+        return 0
+
+    import torch
+    import torch.distributed as dist
+    import block_sparse_attention_route_b200 as bsa
+    from block_sparse_attention_route_b200.pipeline import BsaPipeline
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    g = bsa.Geometry.from_workload(w)
+    x = make_raster_inputs(w, with_grad=with_bwd, seed_offset=0)
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+
+    pipe = BsaPipeline(g, w.top_r, rope_theta=w.theta if w.rope else 0.0, qknorm=w.qknorm,
+                       eps=w.eps, with_bwd=with_bwd, device=str(dev))
+    if w.qknorm:
+        pipe.set_gamma(torch.from_numpy(x["gamma_q"]).to(dev), torch.from_numpy(x["gamma_k"]).to(dev))
+    if w.cached_t:
+        pipe.load_cache(dev_bf16(x["kc"]), dev_bf16(x["vc"]))
+    q_d, k_d, v_d = dev_bf16(x["q"]), dev_bf16(x["k"]), dev_bf16(x["v"])
+    if with_bwd:
+        do_d = dev_bf16(x["do"])
+        pipe.load_grad(do_d)
+    stream = torch.cuda.current_stream(dev)
+
+    ev = {}
+
+    def step(record: bool):
+        marks = []
+        if record:
+            marks.append(torch.cuda.Event(enable_timing=True)); marks[-1].record(stream)
+        pipe.prologue(q_d, k_d, v_d, stream)
+        if record:
+            marks.append(torch.cuda.Event(enable_timing=True)); marks[-1].record(stream)
+        pipe.route(stream)
+        if record:
+            marks.append(torch.cuda.Event(enable_timing=True)); marks[-1].record(stream)
+        pipe.attn_fwd(stream)
+        if record:
+            marks.append(torch.cuda.Event(enable_timing=True)); marks[-1].record(stream)
+        if with_bwd:
+            pipe.backward(stream)
+            if record:
+                marks.append(torch.cuda.Event(enable_timing=True)); marks[-1].record(stream)
+        return marks
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    st = bsa.bsa_device_status()
+    if st != 0:
+        raise SystemExit(f"device status {st} after warm-up")
+
+    n_pairs = int(pipe.cnt.sum().item())
+    fl_fwd = tile_flops(g.bs, g.head_dim, n_pairs)
+    fl_step = fl_fwd * (3.5 if with_bwd else 1.0)
+
+    barrier()
+    torch.cuda.synchronize()
+    all_marks = []
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    with ClockSampler(dev.index or 0) as clk:
+        t0.record(stream)
+        for _ in range(args.steps):
+            all_marks.append(step(True))
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier()
+    ms = t0.elapsed_time(t1) / args.steps
+    names = ["prologue", "route", "fwd"] + (["bwd"] if with_bwd else [])
+    parts = {n: float(np.mean([m[i].elapsed_time(m[i + 1]) for m in all_marks]))
+             for i, n in enumerate(names)}
+    st = bsa.bsa_device_status()
+    if st != 0:
+        raise SystemExit(f"device status {st} after timing")
+
+    ms_max = ms
+    if world > 1:
+        tt = torch.tensor([ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms_max = float(tt.item())
+
+    # ---------------- end to end through the public pipeline, host buffers in and out
+    pin = {k_: torch.from_numpy(x[k_].view(np.int16)).pin_memory() for k_ in ("q", "k", "v")}
+    o_host = torch.empty(pipe.o.shape, dtype=torch.bfloat16).pin_memory()
+    e_steps = max(2, min(args.steps, 5))
+    qh = torch.empty_like(q_d)
+    kh = torch.empty_like(k_d)
+    vh = torch.empty_like(v_d)
+    for _ in range(2):
+        for dst, key in ((qh, "q"), (kh, "k"), (vh, "v")):
+            dst.view(torch.int16).copy_(pin[key], non_blocking=True)
+        pipe.forward(qh, kh, vh, stream)
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        qh.view(torch.int16).copy_(pin["q"], non_blocking=True)
+        kh.view(torch.int16).copy_(pin["k"], non_blocking=True)
+        vh.view(torch.int16).copy_(pin["v"], non_blocking=True)
+        pipe.forward(qh, kh, vh, stream)
+        if with_bwd:
+            pipe.backward(stream)
+        o_host.copy_(pipe.o, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e_ms = e0.elapsed_time(e1) / e_steps
+    if world > 1:
+        tt = torch.tensor([e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e_ms = float(tt.item())
+    h2d = sum(pin[k_].numel() * 2 for k_ in pin)
+    d2h = o_host.numel() * 2
+
+    peaks = load_peaks()
+    fwd_ms = parts["fwd"]
+    achieved = fl_fwd / (fwd_ms * 1e-3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    value = world * fl_step / (ms_max * 1e-3) / 1e12
+    line = {
+        "metric": "BSA fwd(+bwd) effective TFLOP/s at 720p tokens",
+        "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": args.workload, "tokens": w.n_tokens, "padded_tokens": g.nbq * g.bs,
+                   "heads": w.heads, "head_dim": w.head_dim, "block": list(w.blk),
+                   "top_r": w.top_r, "selected_pairs": n_pairs, "with_bwd": with_bwd,
+                   "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (126 MB)"},
+        "ms_per_call": parts,
+        "tflops_fwd": achieved,
+        "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel", "achieved": achieved,
+                     "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "peak_source": f"{peaks['source']} bf16 dense, sustained",
+                     "traffic": None},
+        "e2e": {"value": world * fl_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": args.steps * (3 + (4 if with_bwd else 0)),
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_oracle_sample(w)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

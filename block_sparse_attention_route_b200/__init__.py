@@ -1,0 +1,201 @@
+"""Block sparse attention over 3D latent video tokens on B200 (sm_100a).
+
+Thin ctypes binding over ``libbsa.so`` (the C ABI in ``include/bsa.h``).  Functions keep
+the C names and only marshal arguments: every step of the path runs in the library's CUDA
+kernels.  PyTorch supplies device memory and streams.  There is no CPU fallback: importing
+works without a GPU, but every compute call needs the built library and an sm_100 device.
+
+Build the library with ``python -m block_sparse_attention_route_b200.build``.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+from typing import Optional
+
+__all__ = [
+    "Geometry", "BsaError", "lib", "bsa_workspace_size", "rope3d_qknorm_prologue", "bsa_route",
+    "bsa_attn_fwd", "bsa_attn_bwd", "bsa_device_status", "bsa_error_string", "blocked_shape",
+    "WS_ROUTE", "WS_FWD", "WS_BWD",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbsa.so")
+WS_ROUTE, WS_FWD, WS_BWD = 1, 2, 3
+STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_CUDA",
+          4: "BSA_ERR_TIMEOUT", 5: "BSA_ERR_BAD_INDEX", 6: "BSA_ERR_WORKSPACE"}
+
+
+class BsaError(RuntimeError):
+    def __init__(self, code: int, where: str, detail: str):
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({detail})")
+        self.code = code
+
+
+class _Geom(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("t_frames", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
+                ("cached_t", ctypes.c_int32), ("blk_t", ctypes.c_int32), ("blk_h", ctypes.c_int32),
+                ("blk_w", ctypes.c_int32), ("causal_chunk_t", ctypes.c_int32),
+                ("softmax_scale", ctypes.c_float)]
+
+
+@dataclasses.dataclass(frozen=True)
+class Geometry:
+    """Mirror of ``bsa_geom_t`` (see include/bsa.h for the meaning of every field)."""
+    batch: int
+    heads: int
+    head_dim: int
+    t_frames: int
+    grid_h: int
+    grid_w: int
+    blk: tuple = (4, 4, 8)
+    cached_t: int = 0
+    causal_chunk_t: int = 0
+    softmax_scale: float = 0.0
+
+    def c(self) -> _Geom:
+        return _Geom(self.batch, self.heads, self.head_dim, self.t_frames, self.grid_h,
+                     self.grid_w, self.cached_t, self.blk[0], self.blk[1], self.blk[2],
+                     self.causal_chunk_t, float(self.softmax_scale))
+
+    @property
+    def bs(self) -> int:
+        return self.blk[0] * self.blk[1] * self.blk[2]
+
+    def n_blocks(self, frames: int) -> int:
+        up = lambda x, b: -(-x // b)  # noqa: E731
+        return up(frames, self.blk[0]) * up(self.grid_h, self.blk[1]) * up(self.grid_w, self.blk[2])
+
+    @property
+    def nbq(self) -> int:
+        return self.n_blocks(self.t_frames)
+
+    @property
+    def nbc(self) -> int:
+        return self.n_blocks(self.cached_t) if self.cached_t else 0
+
+    @property
+    def scale(self) -> float:
+        return self.softmax_scale or 1.0 / math.sqrt(self.head_dim)
+
+    @classmethod
+    def from_workload(cls, w) -> "Geometry":
+        return cls(w.batch, w.heads, w.head_dim, w.t_frames, w.grid_h, w.grid_w, tuple(w.blk),
+                   w.cached_t, w.chunk_t)
+
+
+def blocked_shape(g: Geometry, frames: Optional[int] = None):
+    """Shape [B, H, NB, BS, D] of the blocked layout over ``frames`` (default t_frames)."""
+    return (g.batch, g.heads, g.n_blocks(frames or g.t_frames), g.bs, g.head_dim)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbsa.so; raises if it has not been built (there is no fallback path)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with "
+                              "`python -m block_sparse_attention_route_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I32, F, S = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
+        G = ctypes.POINTER(_Geom)
+        sig = {
+            "bsa_abi_version": (I32, []),
+            "bsa_workspace_size": (S, [G, I32, I32]),
+            "rope3d_qknorm_prologue": (I32, [G, I32, I32, P, P, P, P, P, F, F, P, P, P, P, P, P]),
+            "bsa_route": (I32, [G, I32, P, P, P, P, P, P, P, P, S, P]),
+            "bsa_attn_fwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P]),
+            "bsa_attn_bwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
+            "bsa_device_status": (I32, [P]),
+            "bsa_error_string": (ctypes.c_char_p, [I32]),
+            "bsa_last_error_detail": (ctypes.c_char_p, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = L
+    return _lib
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must live on the GPU")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return t.data_ptr()
+
+
+def _nbytes(t) -> int:
+    if t is None or isinstance(t, int):
+        return 0
+    return t.numel() * t.element_size()
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise BsaError(code, where, lib().bsa_last_error_detail().decode())
+
+
+def bsa_error_string(code: int) -> str:
+    return lib().bsa_error_string(code).decode()
+
+
+def bsa_workspace_size(g: Geometry, top_r: int, which: int) -> int:
+    return int(lib().bsa_workspace_size(ctypes.byref(g.c()), top_r, which))
+
+
+def rope3d_qknorm_prologue(g: Geometry, frames: int, t_offset: int, q, k, v, gamma_q, gamma_k,
+                           eps: float, rope_theta: float, q_blk, k_blk, v_blk, q_pool=None,
+                           k_pool=None, stream=None):
+    _check(lib().rope3d_qknorm_prologue(
+        ctypes.byref(g.c()), frames, t_offset, _ptr(q), _ptr(k), _ptr(v), _ptr(gamma_q),
+        _ptr(gamma_k), eps, rope_theta, _ptr(q_blk), _ptr(k_blk), _ptr(v_blk), _ptr(q_pool),
+        _ptr(k_pool), _stream(stream)), "rope3d_qknorm_prologue")
+
+
+def bsa_route(g: Geometry, top_r: int, q_blk, k_blk, q_pool, k_pool, kpool_cache, idx, cnt,
+              ws=None, stream=None):
+    nbytes = _nbytes(ws)
+    _check(lib().bsa_route(
+        ctypes.byref(g.c()), top_r, _ptr(q_blk), _ptr(k_blk), _ptr(q_pool), _ptr(k_pool),
+        _ptr(kpool_cache), _ptr(idx), _ptr(cnt), _ptr(ws), nbytes, _stream(stream)), "bsa_route")
+
+
+def bsa_attn_fwd(g: Geometry, top_r: int, q_blk, k_blk, v_blk, k_cache_blk, v_cache_blk, idx,
+                 cnt, o_blk, lse, stream=None):
+    _check(lib().bsa_attn_fwd(
+        ctypes.byref(g.c()), top_r, _ptr(q_blk), _ptr(k_blk), _ptr(v_blk), _ptr(k_cache_blk),
+        _ptr(v_cache_blk), _ptr(idx), _ptr(cnt), _ptr(o_blk), _ptr(lse), _stream(stream)),
+        "bsa_attn_fwd")
+
+
+def bsa_attn_bwd(g: Geometry, top_r: int, q_blk, k_blk, v_blk, k_cache_blk, v_cache_blk, o_blk,
+                 lse, do_blk, idx, cnt, dq_blk, dk_blk, dv_blk, ws, stream=None):
+    nbytes = _nbytes(ws)
+    _check(lib().bsa_attn_bwd(
+        ctypes.byref(g.c()), top_r, _ptr(q_blk), _ptr(k_blk), _ptr(v_blk), _ptr(k_cache_blk),
+        _ptr(v_cache_blk), _ptr(o_blk), _ptr(lse), _ptr(do_blk), _ptr(idx), _ptr(cnt),
+        _ptr(dq_blk), _ptr(dk_blk), _ptr(dv_blk), _ptr(ws), nbytes, _stream(stream)),
+        "bsa_attn_bwd")
+
+
+def bsa_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status code (0 = OK)."""
+    return int(lib().bsa_device_status(_stream(stream)))

@@ -1,0 +1,443 @@
+// attn_fwd.cu -- sparse flash-attention forward over the selected key blocks (sm_100a).
+//
+// Source: "LongCat-Video视频生成模型发布 迈出世界模型探索第一步", section 块稀疏注意力（BSA）
+// (attention is computed only over the top-r key blocks of each query block) and
+// "LongCat-Video : Generate 1 minute long AI videos with this model", section "Sparse
+// attention".  The pages' kernel rides on FlashAttention for older GPUs; this one is a
+// Blackwell design: TMA tiles -> tcgen05.mma with accumulators in TMEM.
+//
+// Work item = (b, h, query block i): a 128-row Q tile (the block's BS slots first) against
+// the K/V tiles of idx[b,h,i,0:cnt].  Persistent CTAs (one per SM), items in head-major
+// order so the CTAs running at once share one head's K/V in L2.  Each CTA keeps two items
+// in flight ("lanes" A and B) so one lane's softmax overlaps the other lane's MMAs.
+//
+// Warp roles (320 threads):
+//   warps 0-3  softmax + epilogue of lane A (thread = query row = TMEM lane)
+//   warps 4-7  softmax + epilogue of lane B
+//   warp 8     TMA producer (one thread)
+//   warp 9     MMA issuer (one thread); owns the TMEM allocation (512 columns)
+// TMEM columns: lane L uses S/P at [256L, 256L+BS) and O at [256L+128, 256L+128+D).
+// P (bf16) overwrites the first BS/2 columns of S; the next S of that lane is issued after
+// the PV that reads P, and tcgen05 MMAs of one thread execute in issue order.
+//
+// Shared memory: Q tile per lane + a ring of kStages K/V tiles, consumed strictly in the
+// order the MMA thread uses them; the producer walks the identical schedule.
+// Online softmax in the exp2 domain with lazy rescaling: the running max is only raised
+// when a row's max grows by more than 8 (log2 units), so O is rarely touched; the final
+// O / l and LSE are exact either way.
+#include "common.cuh"
+
+namespace bsa {
+
+struct FwdParams {
+  Geo g;
+  int r;
+  int n_items;
+  const int* idx;
+  const int* cnt;
+  __nv_bfloat16* o;
+  float* lse;
+};
+
+constexpr int kFwdThreads = 320;
+constexpr int kFwdStages = 5;
+constexpr int kTileM = 128;
+
+template <int BS, int D>
+struct FwdLayout {
+  static constexpr int kQBytes = kTileM * D * 2;
+  static constexpr int kKVBytes = BS * D * 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kRingOff = 2 * kQBytes;
+  static constexpr int kBarOff = kRingOff + kFwdStages * kKVBytes;
+  // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] fin
+  static constexpr int kNumBars = 2 * 5 + 2 * kFwdStages + 1;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
+};
+
+// Cursor over the items of one lane: items blockIdx.x + gridDim.x * (2k + lane), skipping
+// items with cnt == 0.  The producer and the MMA thread walk identical cursors.
+struct Cursor {
+  int k, item, cnt, n;
+};
+
+__device__ __forceinline__ int load_cnt(const FwdParams& p, int item) {
+  int c = __ldg(p.cnt + item);
+  if (c < 0 || c > p.r) {
+    set_status(DEV_BAD_INDEX);
+    c = c < 0 ? 0 : p.r;
+  }
+  return c;
+}
+
+__device__ __forceinline__ int load_idx(const FwdParams& p, int item, int n) {
+  int j = __ldg(p.idx + (size_t)item * p.r + n);
+  if (j < 0 || j >= p.g.NBk) {
+    set_status(DEV_BAD_INDEX);
+    j = 0;
+  }
+  return j;
+}
+
+__device__ __forceinline__ bool cursor_seek(const FwdParams& p, Cursor& c, int lane) {
+  for (;; ++c.k) {
+    const int item = blockIdx.x + gridDim.x * (2 * c.k + lane);
+    if (item >= p.n_items) { c.item = -1; return false; }
+    const int n = load_cnt(p, item);
+    if (n > 0) { c.item = item; c.cnt = n; c.n = 0; return true; }
+  }
+}
+__device__ __forceinline__ bool cursor_next(const FwdParams& p, Cursor& c, int lane) {
+  if (++c.n < c.cnt) return true;
+  ++c.k;
+  return cursor_seek(p, c, lane);
+}
+
+template <int BS, int D>
+__global__ void __launch_bounds__(kFwdThreads, 1)
+    bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
+                   const __grid_constant__ CUtensorMap tmVc, const FwdParams p) {
+  using L = FwdLayout<BS, D>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 2;
+  uint64_t* kv_full = bars + 4;
+  uint64_t* kv_empty = kv_full + kFwdStages;
+  uint64_t* s_full = kv_empty + kFwdStages;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* o_full = p_full + 2;
+  uint64_t* fin_bar = o_full + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const Geo& g = p.g;
+
+  if (tid == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&q_full[i], 1);
+      mbar_init(&q_empty[i], 1);
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], 128);
+      mbar_init(&o_full[i], 1);
+    }
+    for (int s = 0; s < kFwdStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(fin_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(tmem_holder, 512);
+    tmem_relinquish();
+  }
+  if (warp == 8 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  if (warp == 8) {
+    // ================================================================ TMA producer
+    if (lane == 0) {
+      Cursor cur[2] = {{0, -1, 0, 0}, {0, -1, 0, 0}};
+      bool act[2];
+      act[0] = cursor_seek(p, cur[0], 0);
+      act[1] = cursor_seek(p, cur[1], 1);
+      int seq = 0, qloads[2] = {0, 0};
+      int stage_loads[kFwdStages];
+      for (int s = 0; s < kFwdStages; ++s) stage_loads[s] = 0;
+      bool ok = true;
+      auto kv_tile = [&](int Lw, bool is_v) -> bool {
+        const int stage = seq % kFwdStages, round = seq / kFwdStages;
+        if (round > 0 && !mbar_wait(&kv_empty[stage], (round - 1) & 1, abort_flag)) return false;
+        const Cursor& c = cur[Lw];
+        const int j = load_idx(p, c.item, c.n);
+        const int bhx = c.item / g.NBq;
+        const CUtensorMap* map;
+        int row;
+        if (j < g.NBc) { map = is_v ? &tmVc : &tmKc; row = (bhx * g.NBc + j) * BS; }
+        else { map = is_v ? &tmV : &tmK; row = (bhx * g.NBq + (j - g.NBc)) * BS; }
+        unsigned char* dst = smem + L::kRingOff + stage * L::kKVBytes;
+        mbar_expect_tx(&kv_full[stage], L::kKVBytes);
+#pragma unroll
+        for (int half = 0; half < D / 64; ++half)
+          tma_load_2d(dst + half * BS * 128, map, half * 64, row, &kv_full[stage]);
+        stage_loads[stage]++;
+        ++seq;
+        return true;
+      };
+      auto s_loads = [&](int Lw) -> bool {
+        Cursor& c = cur[Lw];
+        if (c.n == 0) {
+          if (qloads[Lw] > 0 && !mbar_wait(&q_empty[Lw], (qloads[Lw] - 1) & 1, abort_flag))
+            return false;
+          unsigned char* dst = smem + L::kQOff + Lw * L::kQBytes;
+          mbar_expect_tx(&q_full[Lw], L::kQBytes);
+#pragma unroll
+          for (int half = 0; half < D / 64; ++half)
+            tma_load_2d(dst + half * kTileM * 128, &tmQ, half * 64, c.item * BS, &q_full[Lw]);
+          qloads[Lw]++;
+        }
+        return kv_tile(Lw, false);
+      };
+      for (int Lw = 0; Lw < 2 && ok; ++Lw)
+        if (act[Lw]) ok = s_loads(Lw);
+      while (ok && (act[0] || act[1])) {
+        for (int Lw = 0; Lw < 2 && ok; ++Lw) {
+          if (!act[Lw]) continue;
+          ok = kv_tile(Lw, true);
+          if (!ok) break;
+          act[Lw] = cursor_next(p, cur[Lw], Lw);
+          if (act[Lw]) ok = s_loads(Lw);
+        }
+      }
+      // drain: every issued TMA load must land before the CTA may exit
+      for (int s = 0; s < kFwdStages; ++s)
+        if (stage_loads[s] > 0) mbar_wait_drain(&kv_full[s], (stage_loads[s] - 1) & 1);
+      for (int Lw = 0; Lw < 2; ++Lw)
+        if (qloads[Lw] > 0) mbar_wait_drain(&q_full[Lw], (qloads[Lw] - 1) & 1);
+    }
+  } else if (warp == 9) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kTileM, BS, 0, 0);
+      constexpr uint32_t idPV = idesc_bf16(kTileM, D, 0, 1);
+      Cursor cur[2] = {{0, -1, 0, 0}, {0, -1, 0, 0}};
+      bool act[2];
+      act[0] = cursor_seek(p, cur[0], 0);
+      act[1] = cursor_seek(p, cur[1], 1);
+      int seq = 0, qcons[2] = {0, 0}, pcons[2] = {0, 0};
+      bool ok = true;
+      const uint32_t q_s = smem_u32(smem + L::kQOff);
+      const uint32_t ring_s = smem_u32(smem + L::kRingOff);
+      auto issue_S = [&](int Lw) -> bool {
+        Cursor& c = cur[Lw];
+        if (c.n == 0) {
+          if (!mbar_wait(&q_full[Lw], qcons[Lw] & 1, abort_flag)) return false;
+          qcons[Lw]++;
+        }
+        const int stage = seq % kFwdStages;
+        if (!mbar_wait(&kv_full[stage], (seq / kFwdStages) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t qa = q_s + Lw * L::kQBytes, ka = ring_s + stage * L::kKVBytes;
+        const uint32_t d_s = tmem_base + Lw * 256;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t ad = smem_desc_sw128(qa + (kk / 4) * (kTileM * 128) + (kk % 4) * 32, 16, 1024);
+          const uint64_t bd = smem_desc_sw128(ka + (kk / 4) * (BS * 128) + (kk % 4) * 32, 16, 1024);
+          mma_ss(d_s, ad, bd, idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&kv_empty[stage]);
+        mma_commit(&s_full[Lw]);
+        if (c.n == c.cnt - 1) mma_commit(&q_empty[Lw]);
+        ++seq;
+        return true;
+      };
+      auto issue_PV = [&](int Lw) -> bool {
+        Cursor& c = cur[Lw];
+        if (!mbar_wait(&p_full[Lw], pcons[Lw] & 1, abort_flag)) return false;
+        pcons[Lw]++;
+        const int stage = seq % kFwdStages;
+        if (!mbar_wait(&kv_full[stage], (seq / kFwdStages) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t va = ring_s + stage * L::kKVBytes;
+        const uint32_t d_o = tmem_base + Lw * 256 + 128, a_p = tmem_base + Lw * 256;
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk) {
+          const uint64_t bd = smem_desc_sw128(va + kk * 2048, BS * 128, 1024);
+          mma_ts(d_o, a_p + kk * 8, bd, idPV, (c.n > 0 || kk > 0) ? 1u : 0u);
+        }
+        mma_commit(&kv_empty[stage]);
+        if (c.n == c.cnt - 1) mma_commit(&o_full[Lw]);
+        ++seq;
+        return true;
+      };
+      for (int Lw = 0; Lw < 2 && ok; ++Lw)
+        if (act[Lw]) ok = issue_S(Lw);
+      while (ok && (act[0] || act[1])) {
+        for (int Lw = 0; Lw < 2 && ok; ++Lw) {
+          if (!act[Lw]) continue;
+          ok = issue_PV(Lw);
+          if (!ok) break;
+          act[Lw] = cursor_next(p, cur[Lw], Lw);
+          if (act[Lw]) ok = issue_S(Lw);
+        }
+      }
+      // all MMAs issued by this thread must finish before TMEM is released
+      mma_commit(fin_bar);
+      mbar_wait_drain(fin_bar, 0);
+    }
+  } else {
+    // ================================================================ softmax + epilogue
+    const int Lw = warp / 4;
+    const int row = 32 * (warp % 4) + lane;
+    const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
+    const uint32_t t_s = tmem_base + t_lane + Lw * 256;
+    const uint32_t t_o = t_s + 128;
+    const float sl2 = g.scale * 1.4426950408889634f;
+    int scons = 0, ocons = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = blockIdx.x + gridDim.x * (2 * k + Lw);
+      if (item >= p.n_items) break;
+      const int cnt = load_cnt(p, item);
+      const int i = item % g.NBq;
+      // this row's query slot (rows >= BS belong to the tile's padding and are discarded)
+      bool qvalid = false;
+      if (row < BS) {
+        int vt, vh, vw;
+        block_extent(g, g.T, i, vt, vh, vw);
+        const int lt = row / (g.bh * g.bw), lh = (row / g.bw) % g.bh, lw = row % g.bw;
+        qvalid = lt < vt && lh < vh && lw < vw;
+      }
+      float m = -INFINITY, l = 0.f;
+      for (int n = 0; n < cnt; ++n) {
+        bool w_ok = mbar_wait(&s_full[Lw], scons & 1, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) { ok = false; break; }
+        ++scons;
+        tc_fence_after();
+        const int j = load_idx(p, item, n);
+        float s[BS];
+#pragma unroll
+        for (int c = 0; c < BS / 32; ++c) {
+          uint32_t r32[32];
+          tmem_ld32(t_s + c * 32, r32);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r32[e]);
+        }
+        // pad keys of a partial block get -inf
+        int vt, vh, vw;
+        if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
+        else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
+        if (vt < g.bt || vh < g.bh || vw < g.bw) {
+#pragma unroll
+          for (int c = 0; c < BS; ++c) {
+            const int lt = c / (g.bh * g.bw), lh = (c / g.bw) % g.bh, lw = c % g.bw;
+            if (!(lt < vt && lh < vh && lw < vw)) s[c] = -INFINITY;
+          }
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int c = 0; c < BS; ++c) mx = fmaxf(mx, s[c]);
+        mx *= sl2;
+        // lazy rescale: a row raises its running max only when it grew by more than 8
+        // (log2 units).  tcgen05.ld/st are warp-collective, so the warp rescales together
+        // (alpha = 1 for rows that keep their max).  The PV of step n-1 has completed: the
+        // S of step n was issued after it and has completed.
+        const float m_new = (n == 0 || mx > m + 8.0f) ? mx : m;
+        const bool resc = n > 0 && m_new != m;
+        if (__any_sync(0xffffffffu, resc)) {
+          const float alpha = resc ? exp2f(m - m_new) : 1.0f;
+          l *= alpha;
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t r32[32];
+            tmem_ld32(t_o + c * 32, r32);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r32[e] = __float_as_uint(__uint_as_float(r32[e]) * alpha);
+            tmem_st32(t_o + c * 32, r32);
+          }
+        }
+        m = m_new;
+        // P = exp2(s * scale * log2e - m) as bf16 pairs into the first BS/2 columns of S,
+        // 16 columns (32 keys) at a time; all of S is already in registers.
+        float lsum = 0.f;
+#pragma unroll
+        for (int c = 0; c < BS / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float p0 = exp2f(fmaf(s[c * 32 + 2 * e], sl2, -m));
+            const float p1 = exp2f(fmaf(s[c * 32 + 2 * e + 1], sl2, -m));
+            lsum += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(t_s + c * 16, pk);
+        }
+        l += lsum;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[Lw]);
+      }
+      if (!ok) break;
+      float* lse_row = p.lse + (size_t)item * BS;
+      __nv_bfloat16* o_row = p.o + ((size_t)item * BS + row) * D;
+      if (cnt == 0) {
+        if (row < BS) {
+          uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(o_row)[c] = z;
+          lse_row[row] = -INFINITY;
+        }
+        continue;
+      }
+      bool w_ok = mbar_wait(&o_full[Lw], ocons & 1, abort_flag);
+      w_ok = __all_sync(0xffffffffu, w_ok);
+      if (!w_ok) { ok = false; break; }
+      ++ocons;
+      tc_fence_after();
+      const float inv_l = qvalid ? 1.0f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t r32[32];
+        tmem_ld32(t_o + c * 32, r32);
+        tmem_wait_ld();
+        if (row < BS) {
+          uint4 v[4];
+          uint32_t* v32 = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            v32[e] = pack_bf16x2(__uint_as_float(r32[2 * e]) * inv_l,
+                                 __uint_as_float(r32[2 * e + 1]) * inv_l);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) reinterpret_cast<uint4*>(o_row + c * 32)[e] = v[e];
+        }
+      }
+      if (row < BS) lse_row[row] = qvalid ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 9) tmem_dealloc(tmem_base, 512);
+}
+
+cudaError_t launch_fwd(const CUtensorMap* maps, const FwdParams& p, int n_sm, cudaStream_t s) {
+  const int bs = p.g.BS, d = p.g.D;
+  int grid = min(n_sm, (p.n_items + 1) / 2);
+  if (grid < 1) grid = 1;
+#define BSA_LAUNCH_FWD(BSv, Dv)                                                                    \
+  do {                                                                                             \
+    auto kern = bsa_fwd_kernel<BSv, Dv>;                                                           \
+    const int smem = FwdLayout<BSv, Dv>::kAlloc;                                                   \
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); \
+    if (e != cudaSuccess) return e;                                                                \
+    kern<<<grid, kFwdThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);         \
+    return cudaGetLastError();                                                                     \
+  } while (0)
+  if (bs == 128 && d == 128) BSA_LAUNCH_FWD(128, 128);
+  if (bs == 128 && d == 64) BSA_LAUNCH_FWD(128, 64);
+  if (bs == 32 && d == 128) BSA_LAUNCH_FWD(32, 128);
+  if (bs == 32 && d == 64) BSA_LAUNCH_FWD(32, 64);
+#undef BSA_LAUNCH_FWD
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace bsa

@@ -1,0 +1,398 @@
+// bsa_lib.cu -- libbsa.so: the C ABI declared in include/bsa.h.
+//
+// One translation unit (the kernel files are included below) so that every kernel shares
+// the single per-device status word without relocatable device code.  Host code here
+// validates arguments, derives the block geometry, encodes TMA tensor maps and enqueues the
+// kernels on the caller's stream.  It allocates no device memory.
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+
+#include "prologue.cu"
+#include "route.cu"
+#include "attn_fwd.cu"
+#include "attn_bwd.cu"
+
+namespace bsa {
+namespace {
+
+thread_local std::string t_detail;
+
+bsa_status_t fail(bsa_status_t s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_detail = buf;
+  return s;
+}
+
+bsa_status_t cuda_fail(cudaError_t e, const char* where) {
+  return fail(BSA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+// ---------------------------------------------------------------- device checks (cached)
+struct DevInfo {
+  int checked = 0;  // 0 unknown, 1 ok, -1 unsupported
+  int n_sm = 0;
+};
+DevInfo g_dev[64];
+std::mutex g_dev_mu;
+
+bsa_status_t check_device(int* n_sm) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(BSA_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (d.checked == 0) {
+    int major = 0, minor = 0, sms = 0;
+    if ((e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev)) != cudaSuccess ||
+        (e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+      return cuda_fail(e, "cudaDeviceGetAttribute");
+    d.checked = (major == 10 && minor == 0) ? 1 : -1;
+    d.n_sm = sms;
+  }
+  if (d.checked < 0)
+    return fail(BSA_ERR_UNSUPPORTED, "libbsa is built for sm_100a only (B200)");
+  if (n_sm) *n_sm = d.n_sm;
+  return BSA_OK;
+}
+
+// ---------------------------------------------------------------- geometry
+bsa_status_t make_geo(const bsa_geom_t* gi, Geo* out) {
+  if (gi == nullptr) return fail(BSA_ERR_INVALID_ARG, "geometry is NULL");
+  const bsa_geom_t& a = *gi;
+  if (a.batch < 1 || a.heads < 1 || a.t_frames < 1 || a.grid_h < 1 || a.grid_w < 1)
+    return fail(BSA_ERR_INVALID_ARG, "batch, heads, t_frames, grid_h, grid_w must be >= 1");
+  if (a.head_dim != 64 && a.head_dim != 128)
+    return fail(BSA_ERR_UNSUPPORTED, "head_dim %d (supported: 64, 128)", a.head_dim);
+  if (a.blk_t < 1 || a.blk_h < 1 || a.blk_w < 1)
+    return fail(BSA_ERR_INVALID_ARG, "block dims must be >= 1");
+  const long bs = (long)a.blk_t * a.blk_h * a.blk_w;
+  if (bs != 32 && bs != 128)
+    return fail(BSA_ERR_UNSUPPORTED, "block size %ld tokens (supported: 32, 128)", bs);
+  if (a.cached_t < 0 || a.cached_t % a.blk_t)
+    return fail(BSA_ERR_INVALID_ARG, "cached_t %d must be >= 0 and a multiple of blk_t",
+                a.cached_t);
+  if (a.causal_chunk_t < 0 || (a.causal_chunk_t && a.causal_chunk_t % a.blk_t))
+    return fail(BSA_ERR_INVALID_ARG, "causal_chunk_t %d must be 0 or a multiple of blk_t",
+                a.causal_chunk_t);
+  if (!(a.softmax_scale >= 0.f) || std::isinf(a.softmax_scale))
+    return fail(BSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
+  Geo g;
+  g.B = a.batch; g.H = a.heads; g.D = a.head_dim;
+  g.T = a.t_frames; g.GH = a.grid_h; g.GW = a.grid_w; g.Tc = a.cached_t;
+  g.bt = a.blk_t; g.bh = a.blk_h; g.bw = a.blk_w; g.BS = (int)bs;
+  g.nbh = (a.grid_h + a.blk_h - 1) / a.blk_h;
+  g.nbw = (a.grid_w + a.blk_w - 1) / a.blk_w;
+  g.nbt_q = (a.t_frames + a.blk_t - 1) / a.blk_t;
+  g.nbt_c = a.cached_t / a.blk_t;
+  const long per_t = (long)g.nbh * g.nbw;
+  const long nbq = per_t * g.nbt_q, nbc = per_t * g.nbt_c;
+  if (nbq + nbc > 4096)
+    return fail(BSA_ERR_UNSUPPORTED, "%ld key blocks per head (supported: <= 4096)", nbq + nbc);
+  const long rows = (long)g.B * g.H * (nbq + nbc) * bs;
+  if (rows >= (1L << 31) - 256)
+    return fail(BSA_ERR_UNSUPPORTED, "problem too large for 32-bit TMA row coordinates");
+  g.NBq = (int)nbq; g.NBc = (int)nbc; g.NBk = (int)(nbq + nbc);
+  g.chunk = a.causal_chunk_t;
+  g.scale = a.softmax_scale > 0.f ? a.softmax_scale : 1.0f / std::sqrt((float)a.head_dim);
+  *out = g;
+  return BSA_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// ---------------------------------------------------------------- TMA tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bsa_status_t get_encoder(EncodeTiledFn* fn) {
+  std::call_once(g_encode_once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  if (!g_encode) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  *fn = g_encode;
+  return BSA_OK;
+}
+
+// 2D view [rows, D] of a blocked bf16 tensor, box = [64 columns, box_rows rows], 128B swizzle.
+bsa_status_t encode_blocked(CUtensorMap* map, const void* ptr, long rows, int D, int box_rows) {
+  EncodeTiledFn enc;
+  bsa_status_t st = get_encoder(&enc);
+  if (st != BSA_OK) return st;
+  cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims,
+                   strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(BSA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return BSA_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct RouteWs {
+  size_t qpool, kpool, total;
+};
+RouteWs route_ws(const Geo& g) {
+  RouteWs w;
+  w.qpool = 0;
+  w.kpool = align256((size_t)g.B * g.H * g.NBq * g.D * sizeof(float));
+  w.total = w.kpool + align256((size_t)g.B * g.H * g.NBq * g.D * sizeof(float));
+  return w;
+}
+
+}  // namespace
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+int32_t bsa_abi_version(void) { return BSA_ABI_VERSION; }
+
+const char* bsa_error_string(bsa_status_t s) {
+  switch (s) {
+    case BSA_OK: return "ok";
+    case BSA_ERR_INVALID_ARG: return "invalid argument";
+    case BSA_ERR_UNSUPPORTED: return "unsupported device or shape";
+    case BSA_ERR_CUDA: return "CUDA error";
+    case BSA_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+    case BSA_ERR_BAD_INDEX: return "block index or count out of range";
+    case BSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+  }
+  return "unknown status";
+}
+
+const char* bsa_last_error_detail(void) { return t_detail.c_str(); }
+
+size_t bsa_workspace_size(const bsa_geom_t* gi, int32_t top_r, int32_t which) {
+  Geo g;
+  if (make_geo(gi, &g) != BSA_OK || top_r < 1) return 0;
+  if (which == BSA_WS_ROUTE) return route_ws(g).total;
+  if (which == BSA_WS_FWD) return 0;
+  if (which == BSA_WS_BWD) return bwd_ws_layout(g, top_r).total;
+  return 0;
+}
+
+bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
+                                    const void* q_raster, const void* k_raster,
+                                    const void* v_raster, const float* gamma_q,
+                                    const float* gamma_k, float eps, float rope_theta,
+                                    void* q_blk, void* k_blk, void* v_blk, float* q_pool,
+                                    float* k_pool, bsa_stream_t stream) {
+  t_detail.clear();
+  Geo g;
+  bsa_status_t st = make_geo(gi, &g);
+  if (st != BSA_OK) return st;
+  if (frames < 1) return fail(BSA_ERR_INVALID_ARG, "frames must be >= 1");
+  if (t_offset < 0) return fail(BSA_ERR_INVALID_ARG, "t_offset must be >= 0");
+  if (!(eps >= 0.f) || !(rope_theta >= 0.f) || std::isinf(rope_theta))
+    return fail(BSA_ERR_INVALID_ARG, "eps and rope_theta must be finite and >= 0");
+  const void* xs[3] = {q_raster, k_raster, v_raster};
+  void* ys[3] = {q_blk, k_blk, v_blk};
+  bool any = false;
+  for (int i = 0; i < 3; ++i) {
+    if ((xs[i] == nullptr) != (ys[i] == nullptr))
+      return fail(BSA_ERR_INVALID_ARG, "input %d and its output must both be given or both NULL", i);
+    if (xs[i] && (!aligned(xs[i], 16) || !aligned(ys[i], 16)))
+      return fail(BSA_ERR_INVALID_ARG, "tensor %d not 16-byte aligned", i);
+    any |= xs[i] != nullptr;
+  }
+  if (!any) return fail(BSA_ERR_INVALID_ARG, "no tensor to process");
+  if ((q_pool && !q_raster) || (k_pool && !k_raster))
+    return fail(BSA_ERR_INVALID_ARG, "a pool output needs its tensor");
+  if ((q_pool && !aligned(q_pool, 16)) || (k_pool && !aligned(k_pool, 16)))
+    return fail(BSA_ERR_INVALID_ARG, "pool outputs must be 16-byte aligned");
+  if (((long)frames * g.GH * g.GW) * (long)g.B * g.H * g.D >= (1L << 40))
+    return fail(BSA_ERR_UNSUPPORTED, "tensor too large");
+  st = check_device(nullptr);
+  if (st != BSA_OK) return st;
+  PrologueArgs a;
+  a.g = g;
+  a.frames = frames;
+  a.t_offset = t_offset;
+  a.nbt = (frames + g.bt - 1) / g.bt;
+  for (int i = 0; i < 3; ++i) {
+    a.x[i] = static_cast<const __nv_bfloat16*>(xs[i]);
+    a.y[i] = static_cast<__nv_bfloat16*>(ys[i]);
+  }
+  a.gamma[0] = gamma_q;
+  a.gamma[1] = gamma_k;
+  a.pool[0] = q_pool;
+  a.pool[1] = k_pool;
+  a.eps = eps;
+  a.theta = rope_theta;
+  a.dh = 2 * (g.D / 6);
+  a.dw = a.dh;
+  a.dt = g.D - 2 * a.dh;
+  cudaError_t e = launch_prologue(a, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+  return BSA_OK;
+}
+
+bsa_status_t bsa_route(const bsa_geom_t* gi, int32_t top_r, const void* q_blk,
+                       const void* k_blk, const float* q_pool, const float* k_pool,
+                       const float* kpool_cache, int32_t* idx, int32_t* cnt, void* ws,
+                       size_t ws_bytes, bsa_stream_t stream) {
+  t_detail.clear();
+  Geo g;
+  bsa_status_t st = make_geo(gi, &g);
+  if (st != BSA_OK) return st;
+  if (top_r < 1) return fail(BSA_ERR_INVALID_ARG, "top_r must be >= 1");
+  if (!idx || !cnt) return fail(BSA_ERR_INVALID_ARG, "idx and cnt are required");
+  if ((!q_pool && !q_blk) || (!k_pool && !k_blk))
+    return fail(BSA_ERR_INVALID_ARG, "need q_blk or q_pool, and k_blk or k_pool");
+  if (g.NBc > 0 && !kpool_cache)
+    return fail(BSA_ERR_INVALID_ARG, "kpool_cache is required when cached_t > 0");
+  const void* ptrs[5] = {q_blk, k_blk, q_pool, k_pool, kpool_cache};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return fail(BSA_ERR_INVALID_ARG, "inputs must be 16-byte aligned");
+  const RouteWs w = route_ws(g);
+  if ((!q_pool || !k_pool) && (ws == nullptr || ws_bytes < w.total || !aligned(ws, 256)))
+    return fail(BSA_ERR_WORKSPACE, "route needs %zu workspace bytes (256-byte aligned)", w.total);
+  int n_sm = 0;
+  st = check_device(&n_sm);
+  if (st != BSA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (!q_pool) {
+    float* out = reinterpret_cast<float*>(static_cast<char*>(ws) + w.qpool);
+    if ((e = launch_pool(static_cast<const __nv_bfloat16*>(q_blk), g.T, g.NBq, g, out, s)) != cudaSuccess)
+      return cuda_fail(e, "pool launch");
+    q_pool = out;
+  }
+  if (!k_pool) {
+    float* out = reinterpret_cast<float*>(static_cast<char*>(ws) + w.kpool);
+    if ((e = launch_pool(static_cast<const __nv_bfloat16*>(k_blk), g.T, g.NBq, g, out, s)) != cudaSuccess)
+      return cuda_fail(e, "pool launch");
+    k_pool = out;
+  }
+  SelectArgs a;
+  a.g = g;
+  a.r = top_r;
+  a.qt = select_rows_per_cta(g);
+  a.qpool = q_pool;
+  a.kpool = k_pool;
+  a.kpool_cache = kpool_cache;
+  a.idx = idx;
+  a.cnt = cnt;
+  if ((e = launch_select(a, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  return BSA_OK;
+}
+
+bsa_status_t bsa_attn_fwd(const bsa_geom_t* gi, int32_t top_r, const void* q_blk,
+                          const void* k_blk, const void* v_blk, const void* k_cache_blk,
+                          const void* v_cache_blk, const int32_t* idx, const int32_t* cnt,
+                          void* o_blk, float* lse, bsa_stream_t stream) {
+  t_detail.clear();
+  Geo g;
+  bsa_status_t st = make_geo(gi, &g);
+  if (st != BSA_OK) return st;
+  if (top_r < 1) return fail(BSA_ERR_INVALID_ARG, "top_r must be >= 1");
+  if (!q_blk || !k_blk || !v_blk || !idx || !cnt || !o_blk || !lse)
+    return fail(BSA_ERR_INVALID_ARG, "q, k, v, idx, cnt, o and lse are required");
+  if (g.NBc > 0 && (!k_cache_blk || !v_cache_blk))
+    return fail(BSA_ERR_INVALID_ARG, "k_cache_blk and v_cache_blk are required when cached_t > 0");
+  const void* ptrs[7] = {q_blk, k_blk, v_blk, k_cache_blk, v_cache_blk, o_blk, lse};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int n_sm = 0;
+  st = check_device(&n_sm);
+  if (st != BSA_OK) return st;
+  const long bh = (long)g.B * g.H;
+  CUtensorMap maps[5];
+  if ((st = encode_blocked(&maps[0], q_blk, bh * g.NBq * g.BS, g.D, kTileM)) != BSA_OK) return st;
+  if ((st = encode_blocked(&maps[1], k_blk, bh * g.NBq * g.BS, g.D, g.BS)) != BSA_OK) return st;
+  if ((st = encode_blocked(&maps[2], v_blk, bh * g.NBq * g.BS, g.D, g.BS)) != BSA_OK) return st;
+  if (g.NBc > 0) {
+    if ((st = encode_blocked(&maps[3], k_cache_blk, bh * g.NBc * g.BS, g.D, g.BS)) != BSA_OK) return st;
+    if ((st = encode_blocked(&maps[4], v_cache_blk, bh * g.NBc * g.BS, g.D, g.BS)) != BSA_OK) return st;
+  } else {
+    maps[3] = maps[1];
+    maps[4] = maps[2];
+  }
+  FwdParams p;
+  p.g = g;
+  p.r = top_r;
+  p.n_items = (int)(bh * g.NBq);
+  p.idx = idx;
+  p.cnt = cnt;
+  p.o = static_cast<__nv_bfloat16*>(o_blk);
+  p.lse = lse;
+  cudaError_t e = launch_fwd(maps, p, n_sm, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "fwd launch");
+  return BSA_OK;
+}
+
+bsa_status_t bsa_attn_bwd(const bsa_geom_t* gi, int32_t top_r, const void* q_blk,
+                          const void* k_blk, const void* v_blk, const void* k_cache_blk,
+                          const void* v_cache_blk, const void* o_blk, const float* lse,
+                          const void* do_blk, const int32_t* idx, const int32_t* cnt,
+                          void* dq_blk, void* dk_blk, void* dv_blk, void* ws, size_t ws_bytes,
+                          bsa_stream_t stream) {
+  t_detail.clear();
+  Geo g;
+  bsa_status_t st = make_geo(gi, &g);
+  if (st != BSA_OK) return st;
+  if (top_r < 1) return fail(BSA_ERR_INVALID_ARG, "top_r must be >= 1");
+  if (!q_blk || !k_blk || !v_blk || !o_blk || !lse || !do_blk || !idx || !cnt || !dq_blk ||
+      !dk_blk || !dv_blk)
+    return fail(BSA_ERR_INVALID_ARG, "missing tensor argument");
+  if (g.NBc > 0 && (!k_cache_blk || !v_cache_blk))
+    return fail(BSA_ERR_INVALID_ARG, "k_cache_blk and v_cache_blk are required when cached_t > 0");
+  const void* ptrs[11] = {q_blk, k_blk, v_blk, k_cache_blk, v_cache_blk, o_blk, lse, do_blk,
+                          dq_blk, dk_blk, dv_blk};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  const BwdWs w = bwd_ws_layout(g, top_r);
+  if (ws == nullptr || ws_bytes < w.total || !aligned(ws, 256))
+    return fail(BSA_ERR_WORKSPACE, "bwd needs %zu workspace bytes (256-byte aligned)", w.total);
+  int n_sm = 0;
+  st = check_device(&n_sm);
+  if (st != BSA_OK) return st;
+  BwdPtrs P;
+  P.q = q_blk; P.k = k_blk; P.v = v_blk; P.kc = k_cache_blk; P.vc = v_cache_blk;
+  P.o = o_blk; P.lse = lse; P.dO = do_blk; P.idx = idx; P.cnt = cnt;
+  P.dq = dq_blk; P.dk = dk_blk; P.dv = dv_blk; P.ws = static_cast<char*>(ws);
+  return run_bwd(g, top_r, P, w, n_sm, reinterpret_cast<cudaStream_t>(stream));
+}
+
+bsa_status_t bsa_device_status(bsa_stream_t stream) {
+  t_detail.clear();
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  uint32_t v = 0, zero = 0;
+  e = cudaMemcpyFromSymbol(&v, g_dev_status, sizeof(v));
+  if (e != cudaSuccess) return cuda_fail(e, "read status word");
+  if (v) {
+    e = cudaMemcpyToSymbol(g_dev_status, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status word");
+  }
+  if (v & DEV_TIMEOUT) return fail(BSA_ERR_TIMEOUT, "device status 0x%x", v);
+  if (v & DEV_BAD_INDEX) return fail(BSA_ERR_BAD_INDEX, "device status 0x%x", v);
+  return BSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,215 @@
+// prologue.cu -- fused QK-RMSNorm + 3D RoPE + raster -> blocked relayout (+ block means).
+//
+// Source: "美团LongCat-Video揭秘：13.6B参数长视频生成模型如何终结画面漂移？", section 三 模型架构
+// (the DiT uses 3D RoPE position encoding and RMSNorm + QKNorm).  The RoPE channel split and
+// pairing, the norm placement (before RoPE) and eps are this library's documented readings.
+//
+// HBM-bound: every (token, head) row of q, k, v is read once (D bf16) and written once to
+// its slot of the blocked layout; pad slots are written as zeros.  One CTA handles one
+// block of the padded grid for up to 8 heads; D/8 lanes own one row (16-byte vectors), so a
+// warp moves 512 contiguous bytes per instruction on both sides.  The cos/sin table of the
+// block's (t, h, w) positions is built once per CTA in shared memory (fp64 angles).
+#include "common.cuh"
+
+namespace bsa {
+
+struct PrologueArgs {
+  Geo g;
+  int frames, t_offset, nbt;  // grid being processed: frames, RoPE frame offset, t-blocks
+  const __nv_bfloat16* x[3];
+  __nv_bfloat16* y[3];
+  const float* gamma[2];
+  float* pool[2];
+  float eps, theta;
+  int dt, dh, dw;  // RoPE axis widths (channels)
+};
+
+constexpr int kPrologueThreads = 256;
+constexpr int kHeadsPerCta = 8;
+
+template <int D>
+__global__ void __launch_bounds__(kPrologueThreads)
+    prologue_kernel(const PrologueArgs a) {
+  constexpr int LPR = D / 8;                     // lanes per row
+  constexpr int RPP = kPrologueThreads / LPR;    // rows per pass
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* pool_s = reinterpret_cast<float*>(smem_raw);            // [2][8][D]
+  float2* tab = reinterpret_cast<float2*>(pool_s + 2 * kHeadsPerCta * D);
+
+  const Geo& g = a.g;
+  const int blk = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int per_t = g.nbh * g.nbw;
+  const int ibt = blk / per_t, ibh = (blk % per_t) / g.nbw, ibw = blk % g.nbw;
+  int vt, vh, vw;
+  block_extent(g, a.frames, blk, vt, vh, vw);
+  const int nvalid = max(vt, 0) * max(vh, 0) * max(vw, 0);
+  const bool rope = a.theta > 0.f;
+
+  // ---- cos/sin table: axis t rows [0,bt), h rows [bt, bt+bh), w rows after; each row
+  //      holds that axis' pairs.
+  const int pt = a.dt / 2, ph = a.dh / 2, pw = a.dw / 2;
+  const int off_h = g.bt * pt, off_w = off_h + g.bh * ph, ntab = off_w + g.bw * pw;
+  if (rope) {
+    for (int e = tid; e < ntab; e += kPrologueThreads) {
+      int pos, i, width;
+      if (e < off_h) {
+        pos = a.t_offset + ibt * g.bt + e / pt; i = e % pt; width = a.dt;
+      } else if (e < off_w) {
+        int r = e - off_h; pos = ibh * g.bh + r / ph; i = r % ph; width = a.dh;
+      } else {
+        int r = e - off_w; pos = ibw * g.bw + r / pw; i = r % pw; width = a.dw;
+      }
+      double ang = (double)pos * pow((double)a.theta, -2.0 * (double)i / (double)width);
+      double s, c;
+      sincos(ang, &s, &c);
+      tab[e] = make_float2((float)c, (float)s);
+    }
+  }
+  for (int e = tid; e < 2 * kHeadsPerCta * D; e += kPrologueThreads) pool_s[e] = 0.f;
+  __syncthreads();
+
+  const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
+  const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
+  const int rows = heads_here * g.BS;
+  const size_t n_raster = (size_t)a.frames * g.GH * g.GW;
+
+  // RoPE coordinates of this lane's 4 channel pairs: axis (0 t, 1 h, 2 w) and pair index.
+  int ax[4], pi[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    int p = c0 / 2 + q;
+    if (2 * p < a.dt) { ax[q] = 0; pi[q] = p; }
+    else if (2 * p < a.dt + a.dh) { ax[q] = 1; pi[q] = p - pt; }
+    else { ax[q] = 2; pi[q] = p - pt - ph; }
+  }
+
+  for (int which = 0; which < 3; ++which) {
+    const __nv_bfloat16* __restrict__ x = a.x[which];
+    __nv_bfloat16* __restrict__ y = a.y[which];
+    if (x == nullptr) continue;
+    const bool qk = which < 2;
+    const float* gam = qk ? a.gamma[which] : nullptr;
+    const bool do_rope = qk && rope;
+    const bool do_pool = qk && a.pool[which] != nullptr;
+    float gv[8];
+    if (gam) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) gv[e] = gam[c0 + e];
+    }
+    float psum[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    int cur_h = -1;
+    for (int base = 0; base < rows; base += RPP) {
+      const int row = base + rid;
+      const bool in = row < rows;
+      const int hl = in ? row / g.BS : cur_h, slot = row % g.BS;
+      const int h = hg * kHeadsPerCta + hl;
+      const int lt = slot / (g.bh * g.bw), lh = (slot / g.bw) % g.bh, lw = slot % g.bw;
+      const bool valid = in && lt < vt && lh < vh && lw < vw;
+      float v[8];
+      if (valid) {
+        const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
+        const size_t n = ((size_t)t * g.GH + hh) * g.GW + ww;
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
+            x + (((size_t)b * n_raster + n) * g.H + h) * D + c0));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2 f = __bfloat1622float2(p2[e]);
+          v[2 * e] = f.x; v[2 * e + 1] = f.y;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+      }
+      if (gam) {  // RMSNorm over the row: every lane takes part in the shuffles
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float rs = rsqrtf(ss * (1.0f / D) + a.eps);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = v[e] * rs * gv[e];
+      }
+      if (do_rope && valid) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float2 cs;
+          if (ax[q] == 0) cs = tab[lt * pt + pi[q]];
+          else if (ax[q] == 1) cs = tab[off_h + lh * ph + pi[q]];
+          else cs = tab[off_w + lw * pw + pi[q]];
+          const float x0 = v[2 * q], x1 = v[2 * q + 1];
+          v[2 * q] = x0 * cs.x - x1 * cs.y;
+          v[2 * q + 1] = x0 * cs.y + x1 * cs.x;
+        }
+      }
+      uint4 outv;
+      uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o32[e] = valid ? pack_bf16x2(v[2 * e], v[2 * e + 1]) : 0u;
+      if (in) {
+        *reinterpret_cast<uint4*>(
+            y + ((((size_t)b * g.H + h) * (size_t)(a.nbt * per_t) + blk) * g.BS + slot) * D +
+            c0) = outv;
+      }
+      if (do_pool && in) {
+        if (hl != cur_h) {
+          if (cur_h >= 0) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              atomicAdd(&pool_s[(which * kHeadsPerCta + cur_h) * D + c0 + e], psum[e]);
+              psum[e] = 0.f;
+            }
+          }
+          cur_h = hl;
+        }
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&outv);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float2 f = __bfloat1622float2(p2[e]);
+          psum[2 * e] += f.x; psum[2 * e + 1] += f.y;
+        }
+      }
+    }
+    if (do_pool && cur_h >= 0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        atomicAdd(&pool_s[(which * kHeadsPerCta + cur_h) * D + c0 + e], psum[e]);
+    }
+  }
+  __syncthreads();
+  for (int which = 0; which < 2; ++which) {
+    float* out = a.pool[which];
+    if (out == nullptr || a.x[which] == nullptr) continue;
+    const float inv = nvalid > 0 ? 1.0f / (float)nvalid : 0.f;
+    for (int e = tid; e < heads_here * D; e += kPrologueThreads) {
+      const int hl = e / D, d = e % D, h = hg * kHeadsPerCta + hl;
+      out[(((size_t)b * g.H + h) * (size_t)(a.nbt * per_t) + blk) * D + d] =
+          pool_s[(which * kHeadsPerCta + hl) * D + d] * inv;
+    }
+  }
+}
+
+size_t prologue_smem_bytes(const Geo& g, int dt, int dh, int dw) {
+  return (size_t)2 * kHeadsPerCta * g.D * sizeof(float) +
+         (size_t)(g.bt * (dt / 2) + g.bh * (dh / 2) + g.bw * (dw / 2)) * sizeof(float2);
+}
+
+cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s) {
+  const Geo& g = a.g;
+  dim3 grid(a.nbt * g.nbh * g.nbw, (g.H + kHeadsPerCta - 1) / kHeadsPerCta, g.B);
+  size_t smem = prologue_smem_bytes(g, a.dt, a.dh, a.dw);
+  if (g.D == 128) {
+    cudaFuncSetAttribute(prologue_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    prologue_kernel<128><<<grid, kPrologueThreads, smem, s>>>(a);
+  } else {
+    cudaFuncSetAttribute(prologue_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+    prologue_kernel<64><<<grid, kPrologueThreads, smem, s>>>(a);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace bsa

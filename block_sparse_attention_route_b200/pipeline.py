@@ -1,0 +1,100 @@
+"""The BSA call chain on device buffers: prologue -> route -> sparse attention fwd (-> bwd).
+
+``BsaPipeline`` owns the device buffers of one geometry (allocated once with torch) and
+issues the C-ABI calls on one stream; it does no arithmetic itself.
+"""
+from __future__ import annotations
+
+from typing import Dict, Optional
+
+import torch
+
+from . import (WS_BWD, WS_ROUTE, Geometry, blocked_shape, bsa_attn_bwd, bsa_attn_fwd,
+               bsa_route, bsa_workspace_size, rope3d_qknorm_prologue)
+
+
+class BsaPipeline:
+    """Device buffers + calls for one geometry.
+
+    Inputs are raster bf16 [B, N, H, D] tensors on the device.  ``forward`` fills
+    ``self.o`` / ``self.lse`` (blocked), ``self.idx`` / ``self.cnt``; ``backward`` fills
+    ``self.dq`` / ``self.dk`` / ``self.dv`` (blocked).
+    """
+
+    def __init__(self, g: Geometry, top_r: int, *, rope_theta: float = 10000.0,
+                 qknorm: bool = True, eps: float = 1e-6, with_bwd: bool = False,
+                 device: str = "cuda"):
+        self.g, self.r, self.theta, self.eps, self.qknorm = g, top_r, rope_theta, eps, qknorm
+        dev = torch.device(device)
+        bf = dict(dtype=torch.bfloat16, device=dev)
+        shp = blocked_shape(g)
+        self.q = torch.empty(shp, **bf)
+        self.k = torch.empty(shp, **bf)
+        self.v = torch.empty(shp, **bf)
+        self.o = torch.empty(shp, **bf)
+        self.lse = torch.empty(shp[:4], dtype=torch.float32, device=dev)
+        self.q_pool = torch.empty(shp[:3] + (g.head_dim,), dtype=torch.float32, device=dev)
+        self.k_pool = torch.empty_like(self.q_pool)
+        self.idx = torch.empty((g.batch, g.heads, g.nbq, top_r), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((g.batch, g.heads, g.nbq), dtype=torch.int32, device=dev)
+        self.ws_route = torch.empty(max(bsa_workspace_size(g, top_r, WS_ROUTE), 256),
+                                    dtype=torch.uint8, device=dev)
+        self.kc = self.vc = self.kc_pool = None
+        if g.cached_t:
+            cshp = blocked_shape(g, g.cached_t)
+            self.kc = torch.empty(cshp, **bf)
+            self.vc = torch.empty(cshp, **bf)
+            self.kc_pool = torch.empty(cshp[:3] + (g.head_dim,), dtype=torch.float32, device=dev)
+        self.gamma_q = self.gamma_k = None
+        if with_bwd:
+            self.do = torch.empty(shp, **bf)
+            self.dq = torch.empty(shp, **bf)
+            self.dk = torch.empty(shp, **bf)
+            self.dv = torch.empty(shp, **bf)
+            self.ws_bwd = torch.empty(max(bsa_workspace_size(g, top_r, WS_BWD), 256),
+                                      dtype=torch.uint8, device=dev)
+
+    def set_gamma(self, gamma_q: Optional[torch.Tensor], gamma_k: Optional[torch.Tensor]):
+        self.gamma_q, self.gamma_k = gamma_q, gamma_k
+
+    def load_cache(self, kc_raster: torch.Tensor, vc_raster: torch.Tensor, stream=None):
+        """Relayout (and norm/rotate) the cached frames' K/V and their block means, once."""
+        g = self.g
+        rope3d_qknorm_prologue(g, g.cached_t, 0, None, kc_raster, vc_raster, None,
+                               self.gamma_k if self.qknorm else None, self.eps,
+                               self.theta, None, self.kc, self.vc, None, self.kc_pool,
+                               stream=stream)
+
+    def prologue(self, q_raster, k_raster, v_raster, stream=None):
+        g = self.g
+        rope3d_qknorm_prologue(g, g.t_frames, g.cached_t, q_raster, k_raster, v_raster,
+                               self.gamma_q if self.qknorm else None,
+                               self.gamma_k if self.qknorm else None, self.eps, self.theta,
+                               self.q, self.k, self.v, self.q_pool, self.k_pool, stream=stream)
+
+    def route(self, stream=None, use_pools: bool = True):
+        bsa_route(self.g, self.r, self.q, self.k, self.q_pool if use_pools else None,
+                  self.k_pool if use_pools else None, self.kc_pool, self.idx, self.cnt,
+                  self.ws_route, stream=stream)
+
+    def attn_fwd(self, stream=None):
+        bsa_attn_fwd(self.g, self.r, self.q, self.k, self.v, self.kc, self.vc, self.idx,
+                     self.cnt, self.o, self.lse, stream=stream)
+
+    def forward(self, q_raster, k_raster, v_raster, stream=None) -> Dict[str, torch.Tensor]:
+        self.prologue(q_raster, k_raster, v_raster, stream)
+        self.route(stream)
+        self.attn_fwd(stream)
+        return {"o": self.o, "lse": self.lse, "idx": self.idx, "cnt": self.cnt}
+
+    def load_grad(self, do_raster, stream=None):
+        """Relayout the upstream gradient dO (raster) into the blocked layout."""
+        g = self.g
+        rope3d_qknorm_prologue(g, g.t_frames, 0, None, None, do_raster, None, None, 0.0, 0.0,
+                               None, None, self.do, None, None, stream=stream)
+
+    def backward(self, stream=None):
+        bsa_attn_bwd(self.g, self.r, self.q, self.k, self.v, self.kc, self.vc, self.o,
+                     self.lse, self.do, self.idx, self.cnt, self.dq, self.dk, self.dv,
+                     self.ws_bwd, stream=stream)
+        return {"dq": self.dq, "dk": self.dk, "dv": self.dv}

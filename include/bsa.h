@@ -1,0 +1,178 @@
+/*
+ * bsa.h -- C ABI of the B200 (sm_100a) block sparse attention library (libbsa.so).
+ *
+ * Block Sparse Attention (BSA) over 3D latent video tokens: the token grid (latent frames x
+ * rows x columns) is split into 3D blocks; every query block scores every key block with
+ * block-pooled q.k, keeps its top-r key blocks, and exact softmax attention runs over the
+ * selected blocks only, with an optional block-causal mask and cached conditioning-frame
+ * keys/values.  Sources (web pages describing the LongCat-Video model):
+ *   - "LongCat-Video : Generate 1 minute long AI videos with this model", section "Sparse
+ *     attention" (small 3D cubes, each looks at the few most relevant ones, chosen by
+ *     similarity) and section "The core idea" (KV caching of conditioning frames);
+ *   - "LongCat-Video视频生成模型发布 迈出世界模型探索第一步", section 块稀疏注意力（BSA）
+ *     (split the 3D tokens into blocks, keep only the top-r key blocks);
+ *   - "美团LongCat-Video揭秘：13.6B参数长视频生成模型如何终结画面漂移？", section 三 模型架构
+ *     (3D RoPE; RMSNorm + QKNorm);
+ *   - "LongCat-Video 高效長視頻生成探索世界模型的第壹步", section 2.1 (Block-Causal
+ *     attention enabling a cache for continuation) and 2.2 (the sparse attention module
+ *     ships forward and backward code).
+ *
+ * LAYOUTS (all tensors contiguous, row-major, device memory unless stated)
+ *   raster  : bf16 [B, N, H, D], N = frames * grid_h * grid_w tokens ordered (t, h, w).
+ *   blocked : bf16 [B, H, NB, BS, D].  The grid is padded up to whole blocks; blocks are
+ *             numbered (block-t, block-h, block-w) row-major; the BS = blk_t*blk_h*blk_w
+ *             slots of a block are ordered (local t, local h, local w) row-major.  Pad
+ *             slots hold zeros (written by the prologue, written as zeros in O/dQ/dK/dV).
+ *   pooled  : fp32 [B, H, NB, D], mean over the valid (non-pad) tokens of each block.
+ *   idx     : int32 [B, H, NBq, top_r], selected global key-block ids in ascending order,
+ *             -1 after the first cnt entries.  cnt: int32 [B, H, NBq].
+ *   lse     : fp32 [B, H, NBq, BS], natural-log log-sum-exp of the scaled logits of each
+ *             query slot; -inf for pad slots.
+ *   Query blocks cover the current frames (NBq blocks).  Key blocks are numbered globally:
+ *   first the NBc blocks of the cached frames (read from the *_cache tensors, blocked over
+ *   cached_t frames), then the NBq blocks of the current frames.
+ *
+ * OWNERSHIP AND ORDERING
+ *   The caller allocates every buffer; the library allocates no device memory per call.
+ *   Scratch memory is the caller's workspace (see bsa_workspace_size).  Every call enqueues
+ *   work on `stream` and returns without waiting.  Argument errors are returned before
+ *   anything is enqueued.  Device-side failures (a bounded wait that ran out, an index out
+ *   of range) set a per-device status word that bsa_device_status() reports; kernels never
+ *   trap.  Devices other than sm_100 return BSA_ERR_UNSUPPORTED; there is no fallback.
+ */
+#ifndef BSA_H_
+#define BSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BSA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define BSA_API __attribute__((visibility("default")))
+#else
+#define BSA_API
+#endif
+
+typedef struct CUstream_st* bsa_stream_t; /* same handle as cudaStream_t; NULL = legacy default stream */
+
+typedef enum bsa_status {
+  BSA_OK = 0,
+  BSA_ERR_INVALID_ARG = 1,  /* bad pointer, size, shape or alignment; nothing was enqueued */
+  BSA_ERR_UNSUPPORTED = 2,  /* device is not sm_100, or a shape outside the supported set */
+  BSA_ERR_CUDA = 3,         /* a CUDA runtime/driver call failed */
+  BSA_ERR_TIMEOUT = 4,      /* a kernel's bounded wait ran out (reported by bsa_device_status) */
+  BSA_ERR_BAD_INDEX = 5,    /* idx/cnt held a value out of range (reported by bsa_device_status) */
+  BSA_ERR_WORKSPACE = 6     /* workspace pointer NULL/misaligned or smaller than required */
+} bsa_status_t;
+
+/* Geometry of one problem.  Supported: head_dim in {64, 128}; blk_t*blk_h*blk_w in {32, 128};
+ * cached_t and causal_chunk_t multiples of blk_t. */
+typedef struct bsa_geom {
+  int32_t batch;          /* B */
+  int32_t heads;          /* H */
+  int32_t head_dim;       /* D */
+  int32_t t_frames;       /* current latent frames (query tokens and current key tokens) */
+  int32_t grid_h;         /* latent rows (valid, before padding) */
+  int32_t grid_w;         /* latent columns (valid, before padding) */
+  int32_t cached_t;       /* leading latent frames whose K/V come from the cache (0 = none);
+                             current frame f sits at absolute frame cached_t + f */
+  int32_t blk_t, blk_h, blk_w; /* 3D block shape */
+  int32_t causal_chunk_t; /* 0 = no mask; else key block j is allowed for query block i iff
+                             floor(t0(j)/C) <= floor(t0(i)/C), t0 = first absolute frame */
+  float softmax_scale;    /* logits = q.k * scale; 0 selects 1/sqrt(head_dim) */
+} bsa_geom_t;
+
+enum { BSA_WS_ROUTE = 1, BSA_WS_FWD = 2, BSA_WS_BWD = 3 };
+
+/* ABI version of the loaded library (BSA_ABI_VERSION). */
+BSA_API int32_t bsa_abi_version(void);
+
+/* Bytes of workspace `which` (BSA_WS_*) needs for this geometry; 0 on invalid arguments.
+ * Workspace must be 256-byte aligned.  ROUTE: pooled q/k means.  FWD: none (returns 0).
+ * BWD: fp32 dQ accumulator, row sums of dO*O and the key-block -> query-block index. */
+BSA_API size_t bsa_workspace_size(const bsa_geom_t* g, int32_t top_r, int32_t which);
+
+/* Fused QK-RMSNorm + 3D RoPE prologue and raster -> blocked relayout.
+ * Source: "美团LongCat-Video揭秘…", section 三 模型架构 (3D RoPE; RMSNorm + QKNorm).
+ * Processes `frames` frames of the (grid_h, grid_w) grid of g (pass g->t_frames for the
+ * current tokens, g->cached_t for a cache).  For q and k, per (token, head):
+ *   y = x / sqrt(mean_d(x^2) + eps) * gamma      (skipped when gamma is NULL)
+ *   then 3D RoPE when rope_theta > 0: channels [0,d_t) turn with the absolute frame
+ *   (t_offset + t), [d_t, d_t+d_h) with the row, [d_t+d_h, D) with the column, where
+ *   d_h = d_w = 2*floor(D/6) and d_t = D - 2*d_h; the adjacent pair (2p, 2p+1) of an axis
+ *   of width d_a turns by pos * rope_theta^(-2i/d_a), i = the pair's index in that axis.
+ * v is relaid out only (any tensor that needs the layout alone, e.g. dO, can go here).
+ * Each of q/k/v may be NULL (then its output must be NULL too).  q_pool / k_pool (nullable)
+ * receive the fp32 block means of the bf16-rounded q / k outputs.  Arithmetic in fp32,
+ * outputs rounded to bf16 (round to nearest even).  Raster inputs: bf16 [B, frames*gh*gw,
+ * H, D]; outputs blocked over `frames` (pad slots zero).  gamma: fp32 [D] device arrays. */
+BSA_API bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* g, int32_t frames, int32_t t_offset,
+                                    const void* q_raster, const void* k_raster,
+                                    const void* v_raster, const float* gamma_q,
+                                    const float* gamma_k, float eps, float rope_theta,
+                                    void* q_blk, void* k_blk, void* v_blk, float* q_pool,
+                                    float* k_pool, bsa_stream_t stream);
+
+/* Block-pooled top-r routing.
+ * Sources: "LongCat-Video : Generate 1 minute long AI videos with this model", section
+ * "Sparse attention" (blocks chosen by similarity); "LongCat-Video视频生成模型发布…",
+ * section 块稀疏注意力（BSA） (keep the top-r key blocks).
+ * For every (b, h, query block i): s_ij = qbar_i . kbar_j (fp32, unscaled) over all key
+ * blocks j, -inf where the block-causal rule forbids j; keeps the top_r largest (ties to
+ * the lower j), writes them ascending to idx with cnt = min(top_r, #allowed).
+ * qbar/kbar are block means over valid tokens: taken from q_pool/k_pool when given
+ * (e.g. from the prologue), else computed from q_blk/k_blk into the workspace.
+ * kpool_cache: fp32 [B, H, NBc, D] means of the cached key blocks (required iff
+ * cached_t > 0).  ws: BSA_WS_ROUTE bytes (may be NULL when both pools are given). */
+BSA_API bsa_status_t bsa_route(const bsa_geom_t* g, int32_t top_r, const void* q_blk,
+                       const void* k_blk, const float* q_pool, const float* k_pool,
+                       const float* kpool_cache, int32_t* idx, int32_t* cnt, void* ws,
+                       size_t ws_bytes, bsa_stream_t stream);
+
+/* Sparse attention forward over the selected blocks (tcgen05 tensor cores, TMA).
+ * Source: "LongCat-Video视频生成模型发布…", section 块稀疏注意力（BSA）.
+ * For every (b, h, query block i) and valid query slot:
+ *   O = softmax(q K_S^T * scale) V_S, LSE = log sum exp(q K_S^T * scale), over the valid
+ *   key tokens of the blocks S = idx[b,h,i,0:cnt].  Pad query slots get O = 0, LSE = -inf;
+ *   cnt = 0 gives O = 0, LSE = -inf.
+ * q_blk: blocked over the current frames; k_blk/v_blk: current key blocks; k_cache_blk /
+ * v_cache_blk: blocked over cached_t frames (required iff cached_t > 0).  bf16 operands,
+ * fp32 accumulation, O rounded to bf16.  All blocked tensors 16-byte aligned. */
+BSA_API bsa_status_t bsa_attn_fwd(const bsa_geom_t* g, int32_t top_r, const void* q_blk,
+                          const void* k_blk, const void* v_blk, const void* k_cache_blk,
+                          const void* v_cache_blk, const int32_t* idx, const int32_t* cnt,
+                          void* o_blk, float* lse, bsa_stream_t stream);
+
+/* Sparse attention backward for a fixed routing (the forward's idx/cnt).
+ * Source: "LongCat-Video 高效長視頻生成探索世界模型的第壹步", section 2.2 (forward and
+ * backward of the sparse attention for training).  With P the softmax of the forward and
+ * Delta = rowsum(dO * O):  dV_j += P^T dO,  dS = P * (dO V^T - Delta),
+ * dQ_i += scale * dS K_j,  dK_j += scale * dS^T Q_i, summed over the selected pairs.
+ * Gradients reach current keys/values only (cached ones are constants).  Outputs dq_blk,
+ * dk_blk, dv_blk are bf16 blocked (pad slots 0); ws: BSA_WS_BWD bytes. */
+BSA_API bsa_status_t bsa_attn_bwd(const bsa_geom_t* g, int32_t top_r, const void* q_blk,
+                          const void* k_blk, const void* v_blk, const void* k_cache_blk,
+                          const void* v_cache_blk, const void* o_blk, const float* lse,
+                          const void* do_blk, const int32_t* idx, const int32_t* cnt,
+                          void* dq_blk, void* dk_blk, void* dv_blk, void* ws,
+                          size_t ws_bytes, bsa_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the current device's status word.
+ * Returns BSA_OK, BSA_ERR_TIMEOUT or BSA_ERR_BAD_INDEX (or BSA_ERR_CUDA). */
+BSA_API bsa_status_t bsa_device_status(bsa_stream_t stream);
+
+/* Static string for a status code. */
+BSA_API const char* bsa_error_string(bsa_status_t s);
+
+/* Detail of the last argument error on the calling thread ("" if none). */
+BSA_API const char* bsa_last_error_detail(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H_ */

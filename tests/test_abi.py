@@ -1,0 +1,87 @@
+"""C-ABI library checks that need no GPU: it loads, exports every declared entry point,
+and rejects bad arguments on the host before touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import block_sparse_attention_route_b200 as bsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "bsa.h")).read()
+    return re.findall(r"BSA_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+
+
+def test_library_exports_every_declared_symbol():
+    names = _declared()
+    assert set(names) >= {"rope3d_qknorm_prologue", "bsa_route", "bsa_attn_fwd", "bsa_attn_bwd",
+                          "bsa_workspace_size", "bsa_device_status", "bsa_error_string"}
+    L = bsa.lib()
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.bsa_abi_version() == 1
+
+
+def test_error_strings():
+    for code in range(7):
+        assert bsa.bsa_error_string(code)
+
+
+def _g(**kw):
+    base = dict(batch=1, heads=32, head_dim=128, t_frames=24, grid_h=45, grid_w=80)
+    base.update(kw)
+    return bsa.Geometry(**base)
+
+
+def test_workspace_sizes_720p():
+    g = _g()
+    nbq = 720
+    assert g.nbq == nbq
+    route = bsa.bsa_workspace_size(g, 72, bsa.WS_ROUTE)
+    assert route == 2 * 32 * nbq * 128 * 4
+    assert bsa.bsa_workspace_size(g, 72, bsa.WS_FWD) == 0
+    bwd = bsa.bsa_workspace_size(g, 72, bsa.WS_BWD)
+    assert bwd >= 32 * nbq * 128 * 128 * 4  # at least the fp32 dQ accumulator
+
+
+@pytest.mark.parametrize("bad", [dict(head_dim=96), dict(blk=(4, 4, 4)), dict(cached_t=3),
+                                 dict(causal_chunk_t=6), dict(batch=0), dict(grid_w=0),
+                                 dict(softmax_scale=-1.0)])
+def test_bad_geometry_rejected_on_host(bad):
+    g = _g(**bad)
+    assert bsa.bsa_workspace_size(g, 8, bsa.WS_ROUTE) == 0
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_route(g, 8, 16, 16, None, None, None, 16, 16, None, stream=0)
+    assert ei.value.code in (1, 2)
+
+
+def test_bad_arguments_rejected_on_host():
+    g = _g()
+    with pytest.raises(bsa.BsaError) as ei:  # top_r < 1
+        bsa.bsa_attn_fwd(g, 0, 16, 16, 16, None, None, 16, 16, 16, 16, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # missing output
+        bsa.bsa_attn_fwd(g, 8, 16, 16, 16, None, None, 16, 16, None, 16, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # misaligned pointer
+        bsa.bsa_attn_fwd(g, 8, 17, 16, 16, None, None, 16, 16, 16, 16, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # cache geometry without cache tensors
+        bsa.bsa_attn_fwd(_g(cached_t=12, t_frames=12), 8, 16, 16, 16, None, None, 16, 16, 16, 16,
+                         stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # route without workspace
+        bsa.bsa_route(g, 8, 16, 16, None, None, None, 16, 16, None, stream=0)
+    assert ei.value.code == 6
+    with pytest.raises(bsa.BsaError) as ei:  # prologue: output without input
+        bsa.rope3d_qknorm_prologue(g, 24, 0, None, None, None, None, None, 1e-6, 1e4, 16, None,
+                                   None, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # bwd workspace too small
+        bsa.bsa_attn_bwd(g, 8, *([16] * 3), None, None, 16, 16, 16, 16, 16, 16, 16, 16, 16,
+                         stream=0)
+    assert ei.value.code == 6
