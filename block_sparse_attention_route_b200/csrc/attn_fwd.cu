@@ -11,11 +11,15 @@
 // order so the CTAs running at once share one head's K/V in L2.  Each CTA keeps two items
 // in flight ("lanes" A and B) so one lane's softmax overlaps the other lane's MMAs.
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads = 3 warpgroups):
 //   warps 0-3  softmax + epilogue of lane A (thread = query row = TMEM lane)
 //   warps 4-7  softmax + epilogue of lane B
 //   warp 8     TMA producer (one thread)
 //   warp 9     MMA issuer (one thread); owns the TMEM allocation (512 columns)
+//   warps 10-11 idle
+// Registers: launched at 168 per thread (384 x 168 = 64512); the producer/MMA warpgroup
+// drops to kRegsCtl and the two softmax warpgroups rise to kRegsSoftmax:
+// 256 * 208 + 128 * 80 = 63488 <= 64512.
 // TMEM columns: lane L uses S/P at [256L, 256L+BS) and O at [256L+128, 256L+128+D).
 // P (bf16) overwrites the first BS/2 columns of S; the next S of that lane is issued after
 // the PV that reads P, and tcgen05 MMAs of one thread execute in issue order.
@@ -39,7 +43,11 @@ struct FwdParams {
   float* lse;
 };
 
-constexpr int kFwdThreads = 320;
+constexpr int kFwdThreads = 384;
+constexpr int kRegsSoftmax = 208;
+constexpr int kRegsCtl = 80;
+static_assert(256 * kRegsSoftmax + 128 * kRegsCtl <= kFwdThreads * 168,
+              "register re-split exceeds the launch allocation");
 constexpr int kFwdStages = 5;
 constexpr int kTileM = 128;
 
@@ -148,7 +156,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  // every role ends here: all TMEM traffic done, then warp 9 releases the columns
+  auto teardown = [&]() {
+    tc_fence_before();
+    named_bar_sync(1, kFwdThreads);
+    tc_fence_after();
+    if (warp == 9) tmem_dealloc(tmem_base, 512);
+  };
 
+  if (warp >= 8) {
+  regs_dec<kRegsCtl>();
   if (warp == 8) {
     // ================================================================ TMA producer
     if (lane == 0) {
@@ -280,7 +297,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mma_commit(fin_bar);
       mbar_wait_drain(fin_bar, 0);
     }
+  }
+  teardown();
   } else {
+    regs_inc<kRegsSoftmax>();
     // ================================================================ softmax + epilogue
     const int Lw = warp / 4;
     const int row = 32 * (warp % 4) + lane;
@@ -312,24 +332,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
         const int j = load_idx(p, item, n);
         float s[BS];
-#pragma unroll
-        for (int c = 0; c < BS / 32; ++c) {
-          uint32_t r32[32];
-          tmem_ld32(t_s + c * 32, r32);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) s[c * 32 + e] = __uint_as_float(r32[e]);
+        {
+          uint32_t* sr = reinterpret_cast<uint32_t*>(s);
+          if constexpr (BS == 128) tmem_ld128_wait(t_s, sr);
+          else tmem_ld32_wait(t_s, sr);
         }
-        // pad keys of a partial block get -inf
+        // pad keys of a partial block get -inf (mask built without divisions per column)
         int vt, vh, vw;
         if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
         else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
         if (vt < g.bt || vh < g.bh || vw < g.bw) {
+          uint32_t vm[BS / 32];
+          block_valid_mask<BS>(g, vt, vh, vw, vm);
 #pragma unroll
-          for (int c = 0; c < BS; ++c) {
-            const int lt = c / (g.bh * g.bw), lh = (c / g.bw) % g.bh, lw = c % g.bw;
-            if (!(lt < vt && lh < vh && lw < vw)) s[c] = -INFINITY;
-          }
+          for (int c = 0; c < BS; ++c)
+            if (!((vm[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
         }
         float mx = -INFINITY;
 #pragma unroll
@@ -342,17 +359,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const float m_new = (n == 0 || mx > m + 8.0f) ? mx : m;
         const bool resc = n > 0 && m_new != m;
         if (__any_sync(0xffffffffu, resc)) {
-          const float alpha = resc ? exp2f(m - m_new) : 1.0f;
+          const float alpha = resc ? fast_exp2(m - m_new) : 1.0f;
           l *= alpha;
 #pragma unroll
           for (int c = 0; c < D / 32; ++c) {
             uint32_t r32[32];
-            tmem_ld32(t_o + c * 32, r32);
-            tmem_wait_ld();
+            tmem_ld32_wait(t_o + c * 32, r32);
 #pragma unroll
             for (int e = 0; e < 32; ++e) r32[e] = __float_as_uint(__uint_as_float(r32[e]) * alpha);
             tmem_st32(t_o + c * 32, r32);
           }
+          tmem_wait_st();
         }
         m = m_new;
         // P = exp2(s * scale * log2e - m) as bf16 pairs into the first BS/2 columns of S,
@@ -363,8 +380,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = exp2f(fmaf(s[c * 32 + 2 * e], sl2, -m));
-            const float p1 = exp2f(fmaf(s[c * 32 + 2 * e + 1], sl2, -m));
+            const float p0 = fast_exp2(fmaf(s[c * 32 + 2 * e], sl2, -m));
+            const float p1 = fast_exp2(fmaf(s[c * 32 + 2 * e + 1], sl2, -m));
             lsum += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
@@ -396,8 +413,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t r32[32];
-        tmem_ld32(t_o + c * 32, r32);
-        tmem_wait_ld();
+        tmem_ld32_wait(t_o + c * 32, r32);
         if (row < BS) {
           uint4 v[4];
           uint32_t* v32 = reinterpret_cast<uint32_t*>(v);
@@ -411,12 +427,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       }
       if (row < BS) lse_row[row] = qvalid ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
+    teardown();
   }
-
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  if (warp == 9) tmem_dealloc(tmem_base, 512);
 }
 
 cudaError_t launch_fwd(const CUtensorMap* maps, const FwdParams& p, int n_sm, cudaStream_t s) {
