@@ -50,6 +50,10 @@ static_assert(256 * kRegsSoftmax + 128 * kRegsCtl <= kFwdThreads * 168,
               "register re-split exceeds the launch allocation");
 constexpr int kFwdStages = 5;
 constexpr int kTileM = 128;
+// softmax arithmetic options (see the design doc for the measurements behind the defaults)
+constexpr bool kPolyExp = false;   // half of the exponentials on the FMA pipe
+constexpr bool kMax3 = true;       // 3-input max for the row max
+constexpr bool kPacked = true;     // f32x2 FMA / ADD for the exponent argument and row sum
 
 template <int BS, int D>
 struct FwdLayout {
@@ -168,129 +172,135 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   regs_dec<kRegsCtl>();
   if (warp == 8) {
     // ================================================================ TMA producer
+    // Walks the same schedule as the MMA thread: for each lane in turn, the V tile of the
+    // current step, then (after advancing) the Q tile of a new item and the next K tile.
+    // All state lives in registers (the two lanes are unrolled statically).
     if (lane == 0) {
-      Cursor cur[2] = {{0, -1, 0, 0}, {0, -1, 0, 0}};
-      bool act[2];
-      act[0] = cursor_seek(p, cur[0], 0);
-      act[1] = cursor_seek(p, cur[1], 1);
-      int seq = 0, qloads[2] = {0, 0};
-      int stage_loads[kFwdStages];
-      for (int s = 0; s < kFwdStages; ++s) stage_loads[s] = 0;
+      Cursor c0{0, -1, 0, 0}, c1{0, -1, 0, 0};
+      bool a0 = cursor_seek(p, c0, 0), a1 = cursor_seek(p, c1, 1);
+      int seq = 0, ql0 = 0, ql1 = 0;
       bool ok = true;
-      auto kv_tile = [&](int Lw, bool is_v) -> bool {
+      unsigned char* ring = smem + L::kRingOff;
+      auto kv_tile = [&](const Cursor& c, bool is_v) -> bool {
         const int stage = seq % kFwdStages, round = seq / kFwdStages;
         if (round > 0 && !mbar_wait(&kv_empty[stage], (round - 1) & 1, abort_flag)) return false;
-        const Cursor& c = cur[Lw];
         const int j = load_idx(p, c.item, c.n);
         const int bhx = c.item / g.NBq;
         const CUtensorMap* map;
         int row;
         if (j < g.NBc) { map = is_v ? &tmVc : &tmKc; row = (bhx * g.NBc + j) * BS; }
         else { map = is_v ? &tmV : &tmK; row = (bhx * g.NBq + (j - g.NBc)) * BS; }
-        unsigned char* dst = smem + L::kRingOff + stage * L::kKVBytes;
+        unsigned char* dst = ring + stage * L::kKVBytes;
         mbar_expect_tx(&kv_full[stage], L::kKVBytes);
 #pragma unroll
         for (int half = 0; half < D / 64; ++half)
           tma_load_2d(dst + half * BS * 128, map, half * 64, row, &kv_full[stage]);
-        stage_loads[stage]++;
         ++seq;
         return true;
       };
-      auto s_loads = [&](int Lw) -> bool {
-        Cursor& c = cur[Lw];
-        if (c.n == 0) {
-          if (qloads[Lw] > 0 && !mbar_wait(&q_empty[Lw], (qloads[Lw] - 1) & 1, abort_flag))
-            return false;
-          unsigned char* dst = smem + L::kQOff + Lw * L::kQBytes;
-          mbar_expect_tx(&q_full[Lw], L::kQBytes);
+      auto q_tile = [&](const Cursor& c, int lw, int& ql) -> bool {
+        if (ql > 0 && !mbar_wait(&q_empty[lw], (ql - 1) & 1, abort_flag)) return false;
+        unsigned char* dst = smem + L::kQOff + lw * L::kQBytes;
+        mbar_expect_tx(&q_full[lw], L::kQBytes);
 #pragma unroll
-          for (int half = 0; half < D / 64; ++half)
-            tma_load_2d(dst + half * kTileM * 128, &tmQ, half * 64, c.item * BS, &q_full[Lw]);
-          qloads[Lw]++;
-        }
-        return kv_tile(Lw, false);
+        for (int half = 0; half < D / 64; ++half)
+          tma_load_2d(dst + half * kTileM * 128, &tmQ, half * 64, c.item * BS, &q_full[lw]);
+        ++ql;
+        return true;
       };
-      for (int Lw = 0; Lw < 2 && ok; ++Lw)
-        if (act[Lw]) ok = s_loads(Lw);
-      while (ok && (act[0] || act[1])) {
-        for (int Lw = 0; Lw < 2 && ok; ++Lw) {
-          if (!act[Lw]) continue;
-          ok = kv_tile(Lw, true);
+      if (a0) ok = q_tile(c0, 0, ql0) && kv_tile(c0, false);
+      if (ok && a1) ok = q_tile(c1, 1, ql1) && kv_tile(c1, false);
+      while (ok && (a0 || a1)) {
+        if (a0) {
+          ok = kv_tile(c0, true);
           if (!ok) break;
-          act[Lw] = cursor_next(p, cur[Lw], Lw);
-          if (act[Lw]) ok = s_loads(Lw);
+          a0 = cursor_next(p, c0, 0);
+          if (a0) ok = (c0.n > 0 || q_tile(c0, 0, ql0)) && kv_tile(c0, false);
+          if (!ok) break;
+        }
+        if (a1) {
+          ok = kv_tile(c1, true);
+          if (!ok) break;
+          a1 = cursor_next(p, c1, 1);
+          if (a1) ok = (c1.n > 0 || q_tile(c1, 1, ql1)) && kv_tile(c1, false);
         }
       }
       // drain: every issued TMA load must land before the CTA may exit
-      for (int s = 0; s < kFwdStages; ++s)
-        if (stage_loads[s] > 0) mbar_wait_drain(&kv_full[s], (stage_loads[s] - 1) & 1);
-      for (int Lw = 0; Lw < 2; ++Lw)
-        if (qloads[Lw] > 0) mbar_wait_drain(&q_full[Lw], (qloads[Lw] - 1) & 1);
+      for (int st = 0; st < kFwdStages; ++st) {
+        const int loads = seq / kFwdStages + (st < seq % kFwdStages ? 1 : 0);
+        if (loads > 0) mbar_wait_drain(&kv_full[st], (loads - 1) & 1);
+      }
+      if (ql0 > 0) mbar_wait_drain(&q_full[0], (ql0 - 1) & 1);
+      if (ql1 > 0) mbar_wait_drain(&q_full[1], (ql1 - 1) & 1);
     }
   } else if (warp == 9) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTileM, BS, 0, 0);
       constexpr uint32_t idPV = idesc_bf16(kTileM, D, 0, 1);
-      Cursor cur[2] = {{0, -1, 0, 0}, {0, -1, 0, 0}};
-      bool act[2];
-      act[0] = cursor_seek(p, cur[0], 0);
-      act[1] = cursor_seek(p, cur[1], 1);
-      int seq = 0, qcons[2] = {0, 0}, pcons[2] = {0, 0};
+      Cursor c0{0, -1, 0, 0}, c1{0, -1, 0, 0};
+      bool a0 = cursor_seek(p, c0, 0), a1 = cursor_seek(p, c1, 1);
+      int seq = 0, qc0 = 0, qc1 = 0, pc0 = 0, pc1 = 0;
       bool ok = true;
-      const uint32_t q_s = smem_u32(smem + L::kQOff);
-      const uint32_t ring_s = smem_u32(smem + L::kRingOff);
-      auto issue_S = [&](int Lw) -> bool {
-        Cursor& c = cur[Lw];
+      // descriptor bases; per-MMA descriptors add (byte offset >> 4) to the start field
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+      const uint64_t dq1 = smem_desc_sw128(smem_u32(smem + L::kQOff + L::kQBytes), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
+      const uint64_t dv = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
+      auto issue_S = [&](const Cursor& c, int lw, uint64_t dq, int& qc) -> bool {
         if (c.n == 0) {
-          if (!mbar_wait(&q_full[Lw], qcons[Lw] & 1, abort_flag)) return false;
-          qcons[Lw]++;
+          if (!mbar_wait(&q_full[lw], qc & 1, abort_flag)) return false;
+          ++qc;
         }
         const int stage = seq % kFwdStages;
         if (!mbar_wait(&kv_full[stage], (seq / kFwdStages) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t qa = q_s + Lw * L::kQBytes, ka = ring_s + stage * L::kKVBytes;
-        const uint32_t d_s = tmem_base + Lw * 256;
+        const uint32_t d_s = tmem_base + lw * 256;
+        const uint64_t kb = dk + (uint64_t)((stage * L::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t ad = smem_desc_sw128(qa + (kk / 4) * (kTileM * 128) + (kk % 4) * 32, 16, 1024);
-          const uint64_t bd = smem_desc_sw128(ka + (kk / 4) * (BS * 128) + (kk % 4) * 32, 16, 1024);
+          const uint64_t ad = dq + (uint64_t)(((kk / 4) * (kTileM * 128) + (kk % 4) * 32) >> 4);
+          const uint64_t bd = kb + (uint64_t)(((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4);
           mma_ss(d_s, ad, bd, idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(&kv_empty[stage]);
-        mma_commit(&s_full[Lw]);
-        if (c.n == c.cnt - 1) mma_commit(&q_empty[Lw]);
+        mma_commit(&s_full[lw]);
+        if (c.n == c.cnt - 1) mma_commit(&q_empty[lw]);
         ++seq;
         return true;
       };
-      auto issue_PV = [&](int Lw) -> bool {
-        Cursor& c = cur[Lw];
-        if (!mbar_wait(&p_full[Lw], pcons[Lw] & 1, abort_flag)) return false;
-        pcons[Lw]++;
+      auto issue_PV = [&](const Cursor& c, int lw, int& pc) -> bool {
+        if (!mbar_wait(&p_full[lw], pc & 1, abort_flag)) return false;
+        ++pc;
         const int stage = seq % kFwdStages;
         if (!mbar_wait(&kv_full[stage], (seq / kFwdStages) & 1, abort_flag)) return false;
         tc_fence_after();
-        const uint32_t va = ring_s + stage * L::kKVBytes;
-        const uint32_t d_o = tmem_base + Lw * 256 + 128, a_p = tmem_base + Lw * 256;
+        const uint32_t d_o = tmem_base + lw * 256 + 128, a_p = tmem_base + lw * 256;
+        const uint64_t vb = dv + (uint64_t)((stage * L::kKVBytes) >> 4);
 #pragma unroll
-        for (int kk = 0; kk < BS / 16; ++kk) {
-          const uint64_t bd = smem_desc_sw128(va + kk * 2048, BS * 128, 1024);
-          mma_ts(d_o, a_p + kk * 8, bd, idPV, (c.n > 0 || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_ts(d_o, a_p + kk * 8, vb + (uint64_t)((kk * 2048) >> 4), idPV,
+                 (c.n > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&kv_empty[stage]);
-        if (c.n == c.cnt - 1) mma_commit(&o_full[Lw]);
+        if (c.n == c.cnt - 1) mma_commit(&o_full[lw]);
         ++seq;
         return true;
       };
-      for (int Lw = 0; Lw < 2 && ok; ++Lw)
-        if (act[Lw]) ok = issue_S(Lw);
-      while (ok && (act[0] || act[1])) {
-        for (int Lw = 0; Lw < 2 && ok; ++Lw) {
-          if (!act[Lw]) continue;
-          ok = issue_PV(Lw);
+      if (a0) ok = issue_S(c0, 0, dq0, qc0);
+      if (ok && a1) ok = issue_S(c1, 1, dq1, qc1);
+      while (ok && (a0 || a1)) {
+        if (a0) {
+          ok = issue_PV(c0, 0, pc0);
           if (!ok) break;
-          act[Lw] = cursor_next(p, cur[Lw], Lw);
-          if (act[Lw]) ok = issue_S(Lw);
+          a0 = cursor_next(p, c0, 0);
+          if (a0) ok = issue_S(c0, 0, dq0, qc0);
+          if (!ok) break;
+        }
+        if (a1) {
+          ok = issue_PV(c1, 1, pc1);
+          if (!ok) break;
+          a1 = cursor_next(p, c1, 1);
+          if (a1) ok = issue_S(c1, 1, dq1, qc1);
         }
       }
       // all MMAs issued by this thread must finish before TMEM is released
@@ -341,16 +351,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         int vt, vh, vw;
         if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
         else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
-        if (vt < g.bt || vh < g.bh || vw < g.bw) {
+        const bool partial = vt < g.bt || vh < g.bh || vw < g.bw;
+        if (partial) {
           uint32_t vm[BS / 32];
           block_valid_mask<BS>(g, vt, vh, vw, vm);
 #pragma unroll
           for (int c = 0; c < BS; ++c)
             if (!((vm[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
         }
-        float mx = -INFINITY;
+        // row max (four independent chains)
+        float mx;
+        if constexpr (kMax3) {
+          float a0 = s[0], a1 = s[1], a2 = s[2], a3 = s[3];
 #pragma unroll
-        for (int c = 0; c < BS; ++c) mx = fmaxf(mx, s[c]);
+          for (int c = 4; c + 8 <= BS; c += 8) {
+            a0 = max3f(a0, s[c], s[c + 1]);
+            a1 = max3f(a1, s[c + 2], s[c + 3]);
+            a2 = max3f(a2, s[c + 4], s[c + 5]);
+            a3 = max3f(a3, s[c + 6], s[c + 7]);
+          }
+          mx = max3f(max3f(a0, a1, a2), a3, fmaxf(s[BS - 4], fmaxf(s[BS - 3], fmaxf(s[BS - 2], s[BS - 1]))));
+        } else {
+          float a0 = s[0], a1 = s[1], a2 = s[2], a3 = s[3];
+#pragma unroll
+          for (int c = 4; c < BS; c += 4) {
+            a0 = fmaxf(a0, s[c]); a1 = fmaxf(a1, s[c + 1]);
+            a2 = fmaxf(a2, s[c + 2]); a3 = fmaxf(a3, s[c + 3]);
+          }
+          mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+        }
         mx *= sl2;
         // lazy rescale: a row raises its running max only when it grew by more than 8
         // (log2 units).  tcgen05.ld/st are warp-collective, so the warp rescales together
@@ -373,19 +402,42 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         m = m_new;
         // P = exp2(s * scale * log2e - m) as bf16 pairs into the first BS/2 columns of S,
-        // 16 columns (32 keys) at a time; all of S is already in registers.
+        // 16 columns (32 keys) at a time; all of S is already in registers.  Half of the
+        // exponentials go to the FMA pipe (polynomial), half to MUFU; blocks with pad keys
+        // use MUFU only, so masked keys get exactly 0.
+        const uint64_t sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(-m, -m);
+        uint64_t sum2 = f2pack(0.f, 0.f);
         float lsum = 0.f;
+        const bool poly = kPolyExp && !partial;
 #pragma unroll
         for (int c = 0; c < BS / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = fast_exp2(fmaf(s[c * 32 + 2 * e], sl2, -m));
-            const float p1 = fast_exp2(fmaf(s[c * 32 + 2 * e + 1], sl2, -m));
-            lsum += p0 + p1;
+            const float s0 = s[c * 32 + 2 * e], s1 = s[c * 32 + 2 * e + 1];
+            float x0, x1, p0, p1;
+            if constexpr (kPacked) {
+              f2unpack(fma2(f2pack(s0, s1), sl2x2, nmx2), x0, x1);
+            } else {
+              x0 = fmaf(s0, sl2, -m);
+              x1 = fmaf(s1, sl2, -m);
+            }
+            if (poly && (e & 1)) {
+              exp2_poly2(f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f)), p0, p1);
+            } else {
+              p0 = fast_exp2(x0);
+              p1 = fast_exp2(x1);
+            }
+            if constexpr (kPacked) sum2 = add2(sum2, f2pack(p0, p1));
+            else lsum += p0 + p1;
             pk[e] = pack_bf16x2(p0, p1);
           }
           tmem_st16(t_s + c * 16, pk);
+        }
+        if constexpr (kPacked) {
+          float l0, l1;
+          f2unpack(sum2, l0, l1);
+          lsum = l0 + l1;
         }
         l += lsum;
         tmem_wait_st();
