@@ -1,18 +1,40 @@
-// attn_bwd.cu -- sparse flash-attention backward (placeholder until the kernels land).
+// attn_bwd.cu -- sparse flash-attention backward over the forward's selected blocks (sm_100a).
+//
+// Source: "LongCat-Video 高效長視頻生成探索世界模型的第壹步", section 2.2 (the sparse attention
+// module ships forward and backward code for training and inference).  For the forward
+// O = softmax(scale * Q K_S^T) V_S with LSE, and upstream gradient dO:
+//   P = exp(scale * S - LSE),  dP = dO V^T,  Delta = rowsum(dO * O),  dS = P * (dP - Delta)
+//   dV_j += P^T dO_i,  dK_j += scale * dS^T Q_i,  dQ_i += scale * dS K_j
+// summed over every selected (query block i, key block j) pair.
+//
+// Four kernels, all on the caller's stream, no atomics (results are deterministic):
+//   bwd_prep      Delta and log2-scaled LSE per query row (HBM-bound, one warp per row).
+//   bwd_revidx    per (b, h): the key-block -> query-block index (CSR, lists ordered by i).
+//   bwd_dkdv      key-major over current key blocks j: K_j, V_j stay in shared memory, the
+//                 Q_i / dO_i tiles of the query blocks that selected j stream through a TMA
+//                 ring; S^T and dP^T go to TMEM, P^T and dS^T (bf16) overwrite them and feed
+//                 the dV / dK MMAs straight from TMEM; dV, dK accumulate in TMEM.
+//   bwd_dq        query-major like the forward: Q_i, dO_i stay, K_j / V_j stream; S is double
+//                 buffered so the next S and dP run on the tensor cores while the current
+//                 dS is formed; dS (bf16) overwrites S and feeds dQ += dS K_j from TMEM.
+// Splitting dQ from dK/dV costs two extra MMAs per pair (S and dP are recomputed) but needs
+// no fp32 atomics, and the two 512-column TMEM plans fit exactly.
 #include "common.cuh"
 
 namespace bsa {
 
 struct BwdWs {
-  size_t dq_acc, delta, total;
+  size_t delta, lse2, rev_off, rev_list, total;
 };
 inline size_t bwd_align(size_t x) { return (x + 255) & ~size_t(255); }
 BwdWs bwd_ws_layout(const Geo& g, int r) {
-  (void)r;
   BwdWs w;
-  w.dq_acc = 0;
-  w.delta = bwd_align((size_t)g.B * g.H * g.NBq * g.BS * g.D * 4);
-  w.total = w.delta + bwd_align((size_t)g.B * g.H * g.NBq * g.BS * 4);
+  const size_t rows = (size_t)g.B * g.H * g.NBq * g.BS;
+  w.delta = 0;
+  w.lse2 = bwd_align(rows * 4);
+  w.rev_off = w.lse2 + bwd_align(rows * 4);
+  w.rev_list = w.rev_off + bwd_align((size_t)g.B * g.H * (g.NBk + 1) * 4);
+  w.total = w.rev_list + bwd_align((size_t)g.B * g.H * g.NBq * r * 4);
   return w;
 }
 struct BwdPtrs {
@@ -22,8 +44,760 @@ struct BwdPtrs {
   void *dq, *dk, *dv;
   char* ws;
 };
-bsa_status_t run_bwd(const Geo&, int, const BwdPtrs&, const BwdWs&, int, cudaStream_t) {
-  return BSA_ERR_UNSUPPORTED;
+
+struct BwdParams {
+  Geo g;
+  int r;
+  int n_items;            // dkdv: B*H*NBq current key blocks; dq: B*H*NBq query blocks
+  const int* idx;
+  const int* cnt;
+  const int* rev_off;     // [B*H][NBk+1]
+  const int* rev_list;    // [B*H][NBq*r]
+  const float* delta;     // [B*H*NBq*BS]
+  const float* lse2;      // [B*H*NBq*BS], +inf for pad rows
+  __nv_bfloat16* out0;    // dkdv: dK, dq: dQ
+  __nv_bfloat16* out1;    // dkdv: dV
+};
+
+// ------------------------------------------------------------------------------ prep
+// Delta = rowsum(dO * O) and lse2 = LSE * log2(e) (+inf where LSE = -inf: pad rows or empty
+// selections, so exp2(s - lse2) = 0 there).
+template <int D>
+__global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
+                                                       const __nv_bfloat16* __restrict__ dO,
+                                                       const float* __restrict__ lse,
+                                                       float* __restrict__ delta,
+                                                       float* __restrict__ lse2, size_t rows) {
+  constexpr int LPR = D / 8;  // lanes per row (16-byte vectors)
+  const size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const size_t row = t / LPR;
+  const int c = (int)(t % LPR);
+  float acc = 0.f;
+  if (row < rows) {
+    const uint4 a = __ldg(reinterpret_cast<const uint4*>(o + row * D) + c);
+    const uint4 b = __ldg(reinterpret_cast<const uint4*>(dO + row * D) + c);
+    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 fa = __bfloat1622float2(a2[e]), fb = __bfloat1622float2(b2[e]);
+      acc = fmaf(fa.x, fb.x, fmaf(fa.y, fb.y, acc));
+    }
+  }
+#pragma unroll
+  for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (row < rows && c == 0) {
+    delta[row] = acc;
+    const float l = lse[row];
+    lse2[row] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+  }
+}
+
+// ------------------------------------------------------------------------------ reverse index
+// One CTA per (b, h).  Counts how often each key block is selected, scans the counts into
+// offsets, then fills each key block's list with the query blocks that selected it, in
+// increasing query-block order (rows are visited in order; a row never repeats a block).
+constexpr int kRevThreads = 256;
+__global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams p, int* rev_off,
+                                                                int* rev_list) {
+  extern __shared__ int rsm[];  // cnt/cursor [NBk], scan scratch [kRevThreads]
+  const Geo& g = p.g;
+  const int bh = blockIdx.x;
+  int* cntk = rsm;
+  int* part = rsm + g.NBk;
+  const int tid = threadIdx.x;
+  for (int j = tid; j < g.NBk; j += kRevThreads) cntk[j] = 0;
+  __syncthreads();
+  const int* idx = p.idx + (size_t)bh * g.NBq * p.r;
+  const int* cnt = p.cnt + (size_t)bh * g.NBq;
+  for (int e = tid; e < g.NBq * p.r; e += kRevThreads) {
+    const int i = e / p.r, n = e % p.r;
+    int c = cnt[i];
+    if (c < 0 || c > p.r) { set_status(DEV_BAD_INDEX); c = min(max(c, 0), p.r); }
+    if (n < c) {
+      const int j = idx[e];
+      if (j >= 0 && j < g.NBk) atomicAdd(&cntk[j], 1);
+      else set_status(DEV_BAD_INDEX);
+    }
+  }
+  __syncthreads();
+  // exclusive scan: each thread scans a contiguous chunk, then the chunk totals
+  const int per = (g.NBk + kRevThreads - 1) / kRevThreads;
+  const int j0 = tid * per, j1 = min(g.NBk, j0 + per);
+  int s = 0;
+  for (int j = j0; j < j1; ++j) s += cntk[j];
+  part[tid] = s;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int t = 0; t < kRevThreads; ++t) { const int v = part[t]; part[t] = run; run += v; }
+  }
+  __syncthreads();
+  int run = part[tid];
+  int* off = rev_off + (size_t)bh * (g.NBk + 1);
+  for (int j = j0; j < j1; ++j) { const int v = cntk[j]; off[j] = run; cntk[j] = run; run += v; }
+  if (tid == kRevThreads - 1) off[g.NBk] = run;
+  __syncthreads();
+  if (tid < 32) {  // one warp fills rows in order; entries of a row have distinct blocks
+    int* list = rev_list + (size_t)bh * g.NBq * p.r;
+    for (int i = 0; i < g.NBq; ++i) {
+      const int c = min(max(cnt[i], 0), p.r);
+      for (int n = tid; n < c; n += 32) {
+        const int j = idx[(size_t)i * p.r + n];
+        if (j >= 0 && j < g.NBk) list[cntk[j]++] = i;
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// ------------------------------------------------------------------------------ common
+constexpr int kBwdThreads = 192;  // warps 0-3 elementwise (thread = TMEM lane), 4 TMA, 5 MMA
+constexpr int kBwdStages = 2;  // Q_i + dO_i stages of the key-major pass (64 KB each)
+constexpr int kTile = 128;
+
+// ------------------------------------------------------------------------------ dK / dV
+// Work item = current key block (b, h, jc), jc in [0, NBq) (global id NBc + jc).  Steps =
+// the query blocks that selected it.  TMEM: S^T [0,128), dP^T [128,256), dV [256,384),
+// dK [384,512); P^T (bf16) overwrites S^T, dS^T (bf16) overwrites dP^T.
+template <int BS, int D>
+struct DkdvLayout {
+  static constexpr int kKVBytes = BS * D * 2;      // K_j or V_j
+  static constexpr int kTileBytes = BS * D * 2;    // Q_i or dO_i (BS query rows)
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kKVBytes;
+  static constexpr int kRingOff = 2 * kKVBytes;     // stage s: Q at +0, dO at +kTileBytes
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  static constexpr int kVecOff = kRingOff + kBwdStages * kStageBytes;  // lse2 / delta per stage
+  static constexpr int kVecBytes = 2 * BS * 4;
+  static constexpr int kBarOff = kVecOff + kBwdStages * kVecBytes;
+  // kv_full, kv_empty(unused), st_full[S], st_empty[S], s_full, p_full, acc_full, fin
+  static constexpr int kNumBars = 2 + 2 * kBwdStages + 4;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kAlloc = kMiscOff + 16 + 1024;
+};
+
+template <int BS, int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bsa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                        const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                        const BwdParams p) {
+  using L = DkdvLayout<BS, D>;
+  static_assert(BS == 128, "the key-major pass maps one key row to one TMEM lane");
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* kv_full = bars;           // K_j, V_j landed (one phase per item)
+  uint64_t* kv_empty = bars + 1;      // K_j, V_j no longer needed (one phase per item)
+  uint64_t* st_full = bars + 2;       // [kBwdStages] Q_i, dO_i, lse2_i, delta_i landed
+  uint64_t* st_empty = st_full + kBwdStages;
+  uint64_t* s_full = st_empty + kBwdStages;  // S^T and dP^T in TMEM
+  uint64_t* p_full = s_full + 1;             // P^T and dS^T in TMEM (128 arrivals)
+  uint64_t* acc_full = p_full + 1;           // dV and dK of the item complete
+  uint64_t* fin_bar = acc_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const Geo& g = p.g;
+
+  if (tid == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(kv_empty, 1);
+    for (int s = 0; s < kBwdStages; ++s) { mbar_init(&st_full[s], 1); mbar_init(&st_empty[s], 1); }
+    mbar_init(s_full, 1);
+    mbar_init(p_full, 128);
+    mbar_init(acc_full, 1);
+    mbar_init(fin_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 5) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  // item -> (bh, current key block jc); steps = rev list of global key block NBc + jc
+  auto item_range = [&](int item, int& beg, int& end) {
+    const int bh = item / g.NBq, jc = item % g.NBq;
+    const int* off = p.rev_off + (size_t)bh * (g.NBk + 1) + g.NBc + jc;
+    beg = off[0];
+    end = off[1];
+    if (beg < 0 || end < beg || end > g.NBq * p.r) { set_status(DEV_BAD_INDEX); beg = end = 0; }
+  };
+
+  if (warp == 4) {
+    // ====================================================== TMA producer
+    if (lane == 0) {
+      int seq = 0, items = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        int beg, end;
+        item_range(item, beg, end);
+        const int bh = item / g.NBq, jc = item % g.NBq;
+        // K_j, V_j for the item (wait until the previous item's MMAs released them)
+        if (items > 0 && !mbar_wait(kv_empty, (items - 1) & 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(kv_full, 2 * L::kKVBytes);
+        const int krow = (bh * g.NBq + jc) * BS;
+#pragma unroll
+        for (int half = 0; half < D / 64; ++half) {
+          tma_load_2d(smem + L::kKOff + half * BS * 128, &tmK, half * 64, krow, kv_full);
+          tma_load_2d(smem + L::kVOff + half * BS * 128, &tmV, half * 64, krow, kv_full);
+        }
+        ++items;
+        const int* list = p.rev_list + (size_t)bh * g.NBq * p.r;
+        for (int e = beg; e < end; ++e) {
+          int i = list[e];
+          if (i < 0 || i >= g.NBq) { set_status(DEV_BAD_INDEX); i = 0; }
+          const int stage = seq % kBwdStages, round = seq / kBwdStages;
+          if (round > 0 && !mbar_wait(&st_empty[stage], (round - 1) & 1, abort_flag)) { ok = false; break; }
+          unsigned char* dst = smem + L::kRingOff + stage * L::kStageBytes;
+          unsigned char* vec = smem + L::kVecOff + stage * L::kVecBytes;
+          mbar_expect_tx(&st_full[stage], L::kStageBytes + L::kVecBytes);
+          const int qrow = (bh * g.NBq + i) * BS;
+#pragma unroll
+          for (int half = 0; half < D / 64; ++half) {
+            tma_load_2d(dst + half * BS * 128, &tmQ, half * 64, qrow, &st_full[stage]);
+            tma_load_2d(dst + L::kTileBytes + half * BS * 128, &tmdO, half * 64, qrow, &st_full[stage]);
+          }
+          bulk_load(vec, p.lse2 + (size_t)qrow, BS * 4, &st_full[stage]);
+          bulk_load(vec + BS * 4, p.delta + (size_t)qrow, BS * 4, &st_full[stage]);
+          ++seq;
+        }
+      }
+      // drain every copy still in flight
+      for (int st = 0; st < kBwdStages; ++st) {
+        const int loads = seq / kBwdStages + (st < seq % kBwdStages ? 1 : 0);
+        if (loads > 0) mbar_wait_drain(&st_full[st], (loads - 1) & 1);
+      }
+      if (items > 0) mbar_wait_drain(kv_full, (items - 1) & 1);
+    }
+  } else if (warp == 5) {
+    // ====================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idSS = idesc_bf16(kTile, BS, 0, 0);   // S^T, dP^T: both K-major
+      constexpr uint32_t idTS = idesc_bf16(kTile, D, 0, 1);    // dV, dK: B MN-major
+      const uint64_t dK0 = smem_desc_sw128(smem_u32(smem + L::kKOff), 16, 1024);
+      const uint64_t dV0 = smem_desc_sw128(smem_u32(smem + L::kVOff), 16, 1024);
+      const uint64_t dR0 = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
+      const uint64_t dRmn = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
+      const uint32_t t_s = tmem_base, t_dp = tmem_base + 128, t_dv = tmem_base + 256,
+                     t_dk = tmem_base + 384;
+      int seq = 0, items = 0, steps = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        int beg, end;
+        item_range(item, beg, end);
+        if (!mbar_wait(kv_full, items & 1, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        for (int e = beg; e < end; ++e) {
+          const int stage = seq % kBwdStages;
+          if (!mbar_wait(&st_full[stage], (seq / kBwdStages) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t rq = dR0 + (uint64_t)((stage * L::kStageBytes) >> 4);
+          const uint64_t rdo = rq + (uint64_t)(L::kTileBytes >> 4);
+          // S^T = K Q^T, dP^T = V dO^T  (K-dim = D)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
+            mma_ss(t_s, dK0 + off, rq + off, idSS, kk > 0 ? 1u : 0u);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
+            mma_ss(t_dp, dV0 + off, rdo + off, idSS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full);
+          if (!mbar_wait(p_full, steps & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          ++steps;
+          // dV += P^T dO, dK += dS^T Q  (K-dim = the BS query rows; B operands MN-major)
+          const uint64_t mq = dRmn + (uint64_t)((stage * L::kStageBytes) >> 4);
+          const uint64_t mdo = mq + (uint64_t)(L::kTileBytes >> 4);
+          const uint32_t acc0 = (e > beg) ? 1u : 0u;
+#pragma unroll
+          for (int kk = 0; kk < BS / 16; ++kk)
+            mma_ts(t_dv, t_s + kk * 8, mdo + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
+#pragma unroll
+          for (int kk = 0; kk < BS / 16; ++kk)
+            mma_ts(t_dk, t_dp + kk * 8, mq + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
+          mma_commit(&st_empty[stage]);
+          ++seq;
+        }
+        if (!ok) break;
+        mma_commit(kv_empty);
+        if (end > beg) mma_commit(acc_full);
+        ++items;
+      }
+      mma_commit(fin_bar);
+      mbar_wait_drain(fin_bar, 0);
+    }
+  } else {
+    // ====================================================== elementwise + epilogue
+    const int row = 32 * (warp % 4) + lane;  // key slot within the block
+    const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
+    const uint32_t t_s = tmem_base + t_lane, t_dp = t_s + 128, t_dv = t_s + 256, t_dk = t_s + 384;
+    const float sl2 = g.scale * 1.4426950408889634f;
+    int seq = 0, steps = 0, items = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      int beg, end;
+      item_range(item, beg, end);
+      const int jc = item % g.NBq;
+      int vt, vh, vw;
+      block_extent(g, g.T, jc, vt, vh, vw);
+      const int lt = row / (g.bh * g.bw), lh = (row / g.bw) % g.bh, lw = row % g.bw;
+      const bool kvalid = lt < vt && lh < vh && lw < vw;
+      for (int e = beg; e < end; ++e) {
+        const int stage = seq % kBwdStages;
+        bool w_ok = mbar_wait(s_full, steps & 1, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) { ok = false; break; }
+        tc_fence_after();
+        const float* vec = reinterpret_cast<const float*>(smem + L::kVecOff + stage * L::kVecBytes);
+        const float* lse2 = vec;
+        const float* dlt = vec + BS;
+        // 32 query columns at a time: P^T = exp2(S^T*sl2 - lse2[q]),
+        // dS^T = P^T * (dP^T - delta[q]); bf16 results overwrite already-read columns.
+#pragma unroll 1
+        for (int c = 0; c < BS / 32; ++c) {
+          uint32_t sr[32], dr[32], pk[16], dk[16];
+          tmem_ld32_wait(t_s + c * 32, sr);
+          tmem_ld32_wait(t_dp + c * 32, dr);
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const int q0 = c * 32 + 2 * e2;
+            const float2 ld = *reinterpret_cast<const float2*>(lse2 + q0);
+            const float2 dd = *reinterpret_cast<const float2*>(dlt + q0);
+            const float l0 = ld.x, l1 = ld.y, d0 = dd.x, d1 = dd.y;
+            float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -l0));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -l1));
+            if (!kvalid) { p0 = 0.f; p1 = 0.f; }
+            const float s0 = p0 * (__uint_as_float(dr[2 * e2]) - d0);
+            const float s1 = p1 * (__uint_as_float(dr[2 * e2 + 1]) - d1);
+            pk[e2] = pack_bf16x2(p0, p1);
+            dk[e2] = pack_bf16x2(s0, s1);
+          }
+          tmem_st16(t_s + c * 16, pk);
+          tmem_st16(t_dp + c * 16, dk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(p_full);
+        ++steps;
+        ++seq;
+      }
+      if (!ok) break;
+      // epilogue: dV, dK rows of this key block (zeros for pad keys / no selections)
+      const size_t orow = (size_t)item * BS + row;
+      __nv_bfloat16* dv_row = p.out1 + orow * D;
+      __nv_bfloat16* dk_row = p.out0 + orow * D;
+      if (end > beg) {
+        bool w_ok = mbar_wait(acc_full, items & 1, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32], bk[32];
+          tmem_ld32_wait(t_dv + c * 32, a);
+          tmem_ld32_wait(t_dk + c * 32, bk);
+          uint4 va[4], vb[4];
+          uint32_t* a32 = reinterpret_cast<uint32_t*>(va);
+          uint32_t* b32 = reinterpret_cast<uint32_t*>(vb);
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            a32[e2] = kvalid ? pack_bf16x2(__uint_as_float(a[2 * e2]), __uint_as_float(a[2 * e2 + 1])) : 0u;
+            b32[e2] = kvalid ? pack_bf16x2(__uint_as_float(bk[2 * e2]) * g.scale,
+                                           __uint_as_float(bk[2 * e2 + 1]) * g.scale)
+                             : 0u;
+          }
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) {
+            reinterpret_cast<uint4*>(dv_row + c * 32)[e2] = va[e2];
+            reinterpret_cast<uint4*>(dk_row + c * 32)[e2] = vb[e2];
+          }
+        }
+      } else {
+        const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+        for (int c = 0; c < D / 8; ++c) {
+          reinterpret_cast<uint4*>(dv_row)[c] = z;
+          reinterpret_cast<uint4*>(dk_row)[c] = z;
+        }
+      }
+      if (end > beg) ++items;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem_base, 512);
+}
+
+// ------------------------------------------------------------------------------ dQ
+// Work item = query block (b, h, i); steps = its selected key blocks (cached ones included).
+// TMEM: S0 [0,128), S1 [128,256), dP [256,384), dQ [384,512); dS (bf16) overwrites the S
+// buffer it came from.  MMA order per step n: dP(n) once the previous dP was read out,
+// dQ += dS(n-1) K_{n-1}, S(n+1); so the tensor cores run while dS(n) is formed.
+template <int BS, int D>
+struct DqLayout {
+  static constexpr int kTileBytes = kTile * D * 2;  // Q_i / dO_i (128-row tiles)
+  static constexpr int kKVBytes = BS * D * 2;
+  static constexpr int kQOff = 0;
+  static constexpr int kDOOff = kTileBytes;
+  static constexpr int kRingOff = 2 * kTileBytes;
+  static constexpr int kStages = 5;
+  static constexpr int kBarOff = kRingOff + kStages * kKVBytes;
+  // q_full, q_empty, kv_full[5], kv_empty[5], s_full[2], dp_free, ds_full[2], dq_full, fin
+  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 1 + 2 + 2;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kAlloc = kMiscOff + 16 + 1024;
+};
+
+template <int BS, int D>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bsa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                      const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                      const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
+                      const BwdParams p) {
+  using L = DqLayout<BS, D>;
+  constexpr int S = L::kStages;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* q_empty = bars + 1;
+  uint64_t* kv_full = bars + 2;
+  uint64_t* kv_empty = kv_full + S;
+  uint64_t* s_full = kv_empty + S;   // [2] S(n) and dP(n) complete (committed after dP)
+  uint64_t* dp_free = s_full + 2;    // dP read out (128 arrivals)
+  uint64_t* ds_full = dp_free + 1;   // [2] dS(n) in TMEM (128 arrivals)
+  uint64_t* dq_full = ds_full + 2;
+  uint64_t* fin_bar = dq_full + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const Geo& g = p.g;
+
+  if (tid == 0) {
+    mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
+    for (int s = 0; s < S; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&s_full[b], 1); mbar_init(&ds_full[b], 128); }
+    mbar_init(dp_free, 128);
+    mbar_init(dq_full, 1);
+    mbar_init(fin_bar, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 5) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+
+  auto item_cnt = [&](int item) {
+    int c = __ldg(p.cnt + item);
+    if (c < 0 || c > p.r) { set_status(DEV_BAD_INDEX); c = min(max(c, 0), p.r); }
+    return c;
+  };
+  auto item_idx = [&](int item, int n) {
+    int j = __ldg(p.idx + (size_t)item * p.r + n);
+    if (j < 0 || j >= g.NBk) { set_status(DEV_BAD_INDEX); j = 0; }
+    return j;
+  };
+
+  if (warp == 4) {
+    // ====================================================== TMA producer: per step K_n, V_n
+    if (lane == 0) {
+      int seq = 0, qloads = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const int cnt = item_cnt(item);
+        if (cnt == 0) continue;
+        if (qloads > 0 && !mbar_wait(q_empty, (qloads - 1) & 1, abort_flag)) { ok = false; break; }
+        mbar_expect_tx(q_full, 2 * L::kTileBytes);
+#pragma unroll
+        for (int half = 0; half < D / 64; ++half) {
+          tma_load_2d(smem + L::kQOff + half * kTile * 128, &tmQ, half * 64, item * BS, q_full);
+          tma_load_2d(smem + L::kDOOff + half * kTile * 128, &tmdO, half * 64, item * BS, q_full);
+        }
+        ++qloads;
+        const int bhx = item / g.NBq;
+        for (int n = 0; n < cnt && ok; ++n) {
+          const int j = item_idx(item, n);
+          const CUtensorMap *mk, *mv;
+          int row;
+          if (j < g.NBc) { mk = &tmKc; mv = &tmVc; row = (bhx * g.NBc + j) * BS; }
+          else { mk = &tmK; mv = &tmV; row = (bhx * g.NBq + (j - g.NBc)) * BS; }
+          for (int t = 0; t < 2; ++t) {  // K_n then V_n
+            const int stage = seq % S, round = seq / S;
+            if (round > 0 && !mbar_wait(&kv_empty[stage], (round - 1) & 1, abort_flag)) { ok = false; break; }
+            unsigned char* dst = smem + L::kRingOff + stage * L::kKVBytes;
+            mbar_expect_tx(&kv_full[stage], L::kKVBytes);
+#pragma unroll
+            for (int half = 0; half < D / 64; ++half)
+              tma_load_2d(dst + half * BS * 128, t == 0 ? mk : mv, half * 64, row, &kv_full[stage]);
+            ++seq;
+          }
+        }
+      }
+      for (int st = 0; st < S; ++st) {
+        const int loads = seq / S + (st < seq % S ? 1 : 0);
+        if (loads > 0) mbar_wait_drain(&kv_full[st], (loads - 1) & 1);
+      }
+      if (qloads > 0) mbar_wait_drain(q_full, (qloads - 1) & 1);
+    }
+  } else if (warp == 5) {
+    // ====================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kTile, BS, 0, 0);
+      constexpr uint32_t idQ = idesc_bf16(kTile, D, 0, 1);
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+      const uint64_t ddo = smem_desc_sw128(smem_u32(smem + L::kDOOff), 16, 1024);
+      const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
+      const uint64_t dkmn = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
+      const uint32_t t_dp = tmem_base + 256, t_dq = tmem_base + 384;
+      int qcons = 0, dp_issued = 0, dsw0 = 0, dsw1 = 0;
+      bool ok = true;
+      // the ring holds K_n at seq_base + 2n and V_n at seq_base + 2n + 1
+      int seq_base = 0;
+      auto wait_tile = [&](int seq) -> bool {
+        if (!mbar_wait(&kv_full[seq % S], (seq / S) & 1, abort_flag)) return false;
+        tc_fence_after();
+        return true;
+      };
+      auto issue_S = [&](int n) -> bool {  // S(n) = Q K_n^T into buffer n & 1
+        const int seq = seq_base + 2 * n;
+        if (!wait_tile(seq)) return false;
+        const uint64_t kb = dk + (uint64_t)(((seq % S) * L::kKVBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t offq = ((kk / 4) * (kTile * 128) + (kk % 4) * 32) >> 4;
+          const uint32_t offk = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
+          mma_ss(tmem_base + (n & 1) * 128, dq0 + offq, kb + offk, idS, kk > 0 ? 1u : 0u);
+        }
+        return true;
+      };
+      // dP(n) = dO V_n^T once the previous dP has been read out; then signal S(n) + dP(n)
+      auto issue_dP = [&](int n) -> bool {
+        const int seq = seq_base + 2 * n + 1;
+        if (dp_issued > 0) {
+          if (!mbar_wait(dp_free, (dp_issued - 1) & 1, abort_flag)) return false;
+          tc_fence_after();
+        }
+        if (!wait_tile(seq)) return false;
+        const uint64_t vb = dk + (uint64_t)(((seq % S) * L::kKVBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t offq = ((kk / 4) * (kTile * 128) + (kk % 4) * 32) >> 4;
+          const uint32_t offk = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
+          mma_ss(t_dp, ddo + offq, vb + offk, idS, kk > 0 ? 1u : 0u);
+        }
+        ++dp_issued;
+        mma_commit(&kv_empty[seq % S]);  // V_n done
+        mma_commit(&s_full[n & 1]);
+        return true;
+      };
+      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+        const int cnt = item_cnt(item);
+        if (cnt == 0) continue;
+        if (!mbar_wait(q_full, qcons & 1, abort_flag)) { ok = false; break; }
+        ++qcons;
+        tc_fence_after();
+        ok = issue_S(0) && issue_dP(0);
+        if (ok && cnt > 1) ok = issue_S(1);
+        for (int n = 0; n < cnt && ok; ++n) {
+          if (n + 1 < cnt) { ok = issue_dP(n + 1); if (!ok) break; }
+          // dQ += dS(n) K_n  (dS(n) sits in S buffer n & 1)
+          const int b = n & 1;
+          int& dsw = b ? dsw1 : dsw0;
+          if (!mbar_wait(&ds_full[b], dsw & 1, abort_flag)) { ok = false; break; }
+          ++dsw;
+          tc_fence_after();
+          const int kseq = seq_base + 2 * n;
+          const uint64_t kb = dkmn + (uint64_t)(((kseq % S) * L::kKVBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < BS / 16; ++kk)
+            mma_ts(t_dq, tmem_base + b * 128 + kk * 8, kb + (uint64_t)((kk * 2048) >> 4), idQ,
+                   (n > 0 || kk > 0) ? 1u : 0u);
+          mma_commit(&kv_empty[kseq % S]);  // K_n done
+          if (n + 2 < cnt) { ok = issue_S(n + 2); if (!ok) break; }
+        }
+        if (!ok) break;
+        mma_commit(q_empty);
+        mma_commit(dq_full);
+        seq_base += 2 * cnt;
+      }
+      mma_commit(fin_bar);
+      mbar_wait_drain(fin_bar, 0);
+    }
+  } else {
+    // ====================================================== elementwise + epilogue
+    const int row = 32 * (warp % 4) + lane;  // query row of the 128-row tile
+    const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
+    const uint32_t t_dp = tmem_base + t_lane + 256, t_dq = tmem_base + t_lane + 384;
+    const float sl2 = g.scale * 1.4426950408889634f;
+    int sfc[2] = {0, 0}, dqc = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+      const int cnt = item_cnt(item);
+      const size_t qrow = (size_t)item * BS + row;
+      __nv_bfloat16* dq_row = p.out0 + qrow * D;
+      if (cnt == 0) {
+        if (row < BS) {
+          const uint4 z = make_uint4(0, 0, 0, 0);
+#pragma unroll
+          for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dq_row)[c] = z;
+        }
+        continue;
+      }
+      const float l2 = row < BS ? p.lse2[qrow] : INFINITY;   // +inf: pad row -> P = 0
+      const float dl = row < BS ? p.delta[qrow] : 0.f;
+      for (int n = 0; n < cnt; ++n) {
+        const int b = n & 1;
+        bool w_ok = mbar_wait(&s_full[b], sfc[b] & 1, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) { ok = false; break; }
+        ++sfc[b];
+        tc_fence_after();
+        // dP row first, then release its columns for dP(n+1)
+        uint32_t dpr[BS];
+        if constexpr (BS == 128) tmem_ld128_wait(t_dp, dpr);
+        else tmem_ld32_wait(t_dp, dpr);
+        tc_fence_before();
+        mbar_arrive(dp_free);
+        // pad keys of a partial key block: P = 0
+        const int j = item_idx(item, n);
+        int vt, vh, vw;
+        if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
+        else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
+        uint32_t vm[BS / 32];
+#pragma unroll
+        for (int w2 = 0; w2 < BS / 32; ++w2) vm[w2] = 0xFFFFFFFFu;
+        if (vt < g.bt || vh < g.bh || vw < g.bw) block_valid_mask<BS>(g, vt, vh, vw, vm);
+        const uint32_t t_s = tmem_base + t_lane + b * 128;
+#pragma unroll
+        for (int c = 0; c < BS / 32; ++c) {
+          uint32_t sr[32], pk[16];
+          tmem_ld32_wait(t_s + c * 32, sr);
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const int k0 = c * 32 + 2 * e2;
+            float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -l2));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -l2));
+            if (!((vm[k0 >> 5] >> (k0 & 31)) & 1u)) p0 = 0.f;
+            if (!((vm[(k0 + 1) >> 5] >> ((k0 + 1) & 31)) & 1u)) p1 = 0.f;
+            const float d0 = p0 * (__uint_as_float(dpr[k0]) - dl);
+            const float d1 = p1 * (__uint_as_float(dpr[k0 + 1]) - dl);
+            pk[e2] = pack_bf16x2(d0, d1);
+          }
+          tmem_st16(t_s + c * 16, pk);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&ds_full[b]);
+      }
+      if (!ok) break;
+      bool w_ok = mbar_wait(dq_full, dqc & 1, abort_flag);
+      w_ok = __all_sync(0xffffffffu, w_ok);
+      if (!w_ok) { ok = false; break; }
+      ++dqc;
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32_wait(t_dq + c * 32, a);
+        if (row < BS) {
+          uint4 v[4];
+          uint32_t* v32 = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2)
+            v32[e2] = (l2 == INFINITY) ? 0u
+                                       : pack_bf16x2(__uint_as_float(a[2 * e2]) * g.scale,
+                                                     __uint_as_float(a[2 * e2 + 1]) * g.scale);
+#pragma unroll
+          for (int e2 = 0; e2 < 4; ++e2) reinterpret_cast<uint4*>(dq_row + c * 32)[e2] = v[e2];
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 5) tmem_dealloc(tmem_base, 512);
+}
+
+// ------------------------------------------------------------------------------ host side
+// maps: 0 Q (box 128 rows), 1 K, 2 V, 3 K cache, 4 V cache (box BS rows), 5 dO (box 128 rows)
+bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, const CUtensorMap* maps,
+                     int n_sm, cudaStream_t s) {
+  if (g.BS != 128) return BSA_ERR_UNSUPPORTED;  // the key-major pass needs 128-token blocks
+  float* delta = reinterpret_cast<float*>(P.ws + w.delta);
+  float* lse2 = reinterpret_cast<float*>(P.ws + w.lse2);
+  int* rev_off = reinterpret_cast<int*>(P.ws + w.rev_off);
+  int* rev_list = reinterpret_cast<int*>(P.ws + w.rev_list);
+  const size_t rows = (size_t)g.B * g.H * g.NBq * g.BS;
+  {
+    const size_t threads = rows * (g.D / 8);
+    const unsigned blocks = (unsigned)((threads + 255) / 256);
+    if (g.D == 128)
+      bwd_prep_kernel<128><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(P.o),
+                                                  static_cast<const __nv_bfloat16*>(P.dO), P.lse,
+                                                  delta, lse2, rows);
+    else
+      bwd_prep_kernel<64><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(P.o),
+                                                 static_cast<const __nv_bfloat16*>(P.dO), P.lse,
+                                                 delta, lse2, rows);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  BwdParams bp;
+  bp.g = g;
+  bp.r = r;
+  bp.n_items = g.B * g.H * g.NBq;
+  bp.idx = P.idx;
+  bp.cnt = P.cnt;
+  bp.rev_off = rev_off;
+  bp.rev_list = rev_list;
+  bp.delta = delta;
+  bp.lse2 = lse2;
+  {
+    const size_t smem = (size_t)(g.NBk + kRevThreads) * 4;
+    if (cudaFuncSetAttribute(bwd_revidx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+      return BSA_ERR_CUDA;
+    bwd_revidx_kernel<<<g.B * g.H, kRevThreads, smem, s>>>(bp, rev_off, rev_list);
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
+  }
+  const int grid = max(1, min(n_sm, bp.n_items));
+#define BSA_LAUNCH_BWD(Dv)                                                                        \
+  do {                                                                                            \
+    BwdParams a = bp;                                                                             \
+    a.out0 = static_cast<__nv_bfloat16*>(P.dk);                                                   \
+    a.out1 = static_cast<__nv_bfloat16*>(P.dv);                                                   \
+    auto k1 = bsa_bwd_dkdv_kernel<128, Dv>;                                                       \
+    const int s1 = DkdvLayout<128, Dv>::kAlloc;                                                   \
+    if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, s1) != cudaSuccess) \
+      return BSA_ERR_CUDA;                                                                        \
+    k1<<<grid, kBwdThreads, s1, s>>>(maps[1], maps[2], maps[0], maps[5], a);                      \
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;                                   \
+    BwdParams c = bp;                                                                             \
+    c.out0 = static_cast<__nv_bfloat16*>(P.dq);                                                   \
+    c.out1 = nullptr;                                                                             \
+    auto k2 = bsa_bwd_dq_kernel<128, Dv>;                                                         \
+    const int s2 = DqLayout<128, Dv>::kAlloc;                                                     \
+    if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, s2) != cudaSuccess) \
+      return BSA_ERR_CUDA;                                                                        \
+    k2<<<grid, kBwdThreads, s2, s>>>(maps[0], maps[5], maps[1], maps[2], maps[3], maps[4], c);   \
+    if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;                                   \
+  } while (0)
+  if (g.D == 128) BSA_LAUNCH_BWD(128);
+  else BSA_LAUNCH_BWD(64);
+#undef BSA_LAUNCH_BWD
+  return BSA_OK;
 }
 
 }  // namespace bsa

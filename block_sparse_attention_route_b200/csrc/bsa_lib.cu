@@ -372,11 +372,28 @@ bsa_status_t bsa_attn_bwd(const bsa_geom_t* gi, int32_t top_r, const void* q_blk
   int n_sm = 0;
   st = check_device(&n_sm);
   if (st != BSA_OK) return st;
+  if (g.BS != 128)
+    return fail(BSA_ERR_UNSUPPORTED, "backward supports 128-token blocks (got %d)", g.BS);
+  const long bh = (long)g.B * g.H;
+  CUtensorMap maps[6];
+  if ((st = encode_blocked(&maps[0], q_blk, bh * g.NBq * g.BS, g.D, kTileM)) != BSA_OK) return st;
+  if ((st = encode_blocked(&maps[1], k_blk, bh * g.NBq * g.BS, g.D, g.BS)) != BSA_OK) return st;
+  if ((st = encode_blocked(&maps[2], v_blk, bh * g.NBq * g.BS, g.D, g.BS)) != BSA_OK) return st;
+  if (g.NBc > 0) {
+    if ((st = encode_blocked(&maps[3], k_cache_blk, bh * g.NBc * g.BS, g.D, g.BS)) != BSA_OK) return st;
+    if ((st = encode_blocked(&maps[4], v_cache_blk, bh * g.NBc * g.BS, g.D, g.BS)) != BSA_OK) return st;
+  } else {
+    maps[3] = maps[1];
+    maps[4] = maps[2];
+  }
+  if ((st = encode_blocked(&maps[5], do_blk, bh * g.NBq * g.BS, g.D, kTileM)) != BSA_OK) return st;
   BwdPtrs P;
   P.q = q_blk; P.k = k_blk; P.v = v_blk; P.kc = k_cache_blk; P.vc = v_cache_blk;
   P.o = o_blk; P.lse = lse; P.dO = do_blk; P.idx = idx; P.cnt = cnt;
   P.dq = dq_blk; P.dk = dk_blk; P.dv = dv_blk; P.ws = static_cast<char*>(ws);
-  return run_bwd(g, top_r, P, w, n_sm, reinterpret_cast<cudaStream_t>(stream));
+  st = run_bwd(g, top_r, P, w, maps, n_sm, reinterpret_cast<cudaStream_t>(stream));
+  if (st != BSA_OK) return fail(st, "bwd launch failed");
+  return BSA_OK;
 }
 
 bsa_status_t bsa_device_status(bsa_stream_t stream) {
