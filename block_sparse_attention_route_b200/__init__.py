@@ -18,6 +18,7 @@ from typing import Optional
 __all__ = [
     "Geometry", "BsaError", "lib", "bsa_workspace_size", "rope3d_qknorm_prologue", "bsa_route",
     "bsa_attn_fwd", "bsa_attn_bwd", "bsa_device_status", "bsa_error_string", "blocked_shape",
+    "bsa_selftest_bounded_wait",
     "WS_ROUTE", "WS_FWD", "WS_BWD",
 ]
 
@@ -113,6 +114,7 @@ def lib() -> ctypes.CDLL:
             "bsa_attn_fwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P]),
             "bsa_attn_bwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
             "bsa_device_status": (I32, [P]),
+            "bsa_selftest_bounded_wait": (I32, [I32, P]),
             "bsa_error_string": (ctypes.c_char_p, [I32]),
             "bsa_last_error_detail": (ctypes.c_char_p, []),
         }
@@ -194,6 +196,10 @@ def bsa_attn_bwd(g: Geometry, top_r: int, q_blk, k_blk, v_blk, k_cache_blk, v_ca
         _ptr(v_cache_blk), _ptr(o_blk), _ptr(lse), _ptr(do_blk), _ptr(idx), _ptr(cnt),
         _ptr(dq_blk), _ptr(dk_blk), _ptr(dv_blk), _ptr(ws), nbytes, _stream(stream)),
         "bsa_attn_bwd")
+
+
+def bsa_selftest_bounded_wait(limit_us: int, stream=None):
+    _check(lib().bsa_selftest_bounded_wait(limit_us, _stream(stream)), "bsa_selftest_bounded_wait")
 
 
 def bsa_device_status(stream=None) -> int:

@@ -19,6 +19,22 @@
 #include "attn_bwd.cu"
 
 namespace bsa {
+
+// Self-test of the bounded wait: one warp waits on an mbarrier that nothing ever arrives on,
+// with the caller's limit, through the same mbar_wait every kernel uses; it must give up,
+// record DEV_TIMEOUT and return (the context stays usable).
+__global__ void selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  __syncthreads();
+  mbar_wait(&bar, 0, &abort_flag, limit_ns);
+}
+
 namespace {
 
 thread_local std::string t_detail;
@@ -393,6 +409,19 @@ bsa_status_t bsa_attn_bwd(const bsa_geom_t* gi, int32_t top_r, const void* q_blk
   P.dq = dq_blk; P.dk = dk_blk; P.dv = dv_blk; P.ws = static_cast<char*>(ws);
   st = run_bwd(g, top_r, P, w, maps, n_sm, reinterpret_cast<cudaStream_t>(stream));
   if (st != BSA_OK) return fail(st, "bwd launch failed");
+  return BSA_OK;
+}
+
+bsa_status_t bsa_selftest_bounded_wait(int32_t limit_us, bsa_stream_t stream) {
+  t_detail.clear();
+  if (limit_us < 1 || limit_us > 1000000)
+    return fail(BSA_ERR_INVALID_ARG, "limit_us must be in [1, 1e6]");
+  bsa_status_t st = check_device(nullptr);
+  if (st != BSA_OK) return st;
+  selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      (uint64_t)limit_us * 1000ull);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
   return BSA_OK;
 }
 

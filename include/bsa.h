@@ -166,6 +166,13 @@ BSA_API bsa_status_t bsa_attn_bwd(const bsa_geom_t* g, int32_t top_r, const void
  * Returns BSA_OK, BSA_ERR_TIMEOUT or BSA_ERR_BAD_INDEX (or BSA_ERR_CUDA). */
 BSA_API bsa_status_t bsa_device_status(bsa_stream_t stream);
 
+/* Failure-path self test: enqueues one kernel that waits, through the same bounded wait every
+ * kernel uses, on a barrier that nothing signals; after `limit_us` microseconds (1..1e6) it
+ * gives up and records a timeout, which the next bsa_device_status() returns as
+ * BSA_ERR_TIMEOUT.  The device stays usable.  No page counterpart: this tests the library's
+ * own hang protection without hanging the GPU. */
+BSA_API bsa_status_t bsa_selftest_bounded_wait(int32_t limit_us, bsa_stream_t stream);
+
 /* Static string for a status code. */
 BSA_API const char* bsa_error_string(bsa_status_t s);
 

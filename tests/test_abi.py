@@ -45,7 +45,10 @@ def test_workspace_sizes_720p():
     assert route == 2 * 32 * nbq * 128 * 4
     assert bsa.bsa_workspace_size(g, 72, bsa.WS_FWD) == 0
     bwd = bsa.bsa_workspace_size(g, 72, bsa.WS_BWD)
-    assert bwd >= 32 * nbq * 128 * 128 * 4  # at least the fp32 dQ accumulator
+    up = lambda x: -(-x // 256) * 256  # noqa: E731
+    rows = 32 * nbq * 128
+    # Delta + log2 LSE per query row, reverse-index offsets and lists
+    assert bwd == 2 * up(rows * 4) + up(32 * (nbq + 1) * 4) + up(32 * nbq * 72 * 4)
 
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(blk=(4, 4, 4)), dict(cached_t=3),

@@ -263,3 +263,18 @@ def test_bad_index_reports_status_without_fault(torch_cuda):
     torch.cuda.synchronize()
     assert bsa.bsa_device_status() == 5
     assert bsa.bsa_device_status() == 0  # cleared
+
+
+def test_bounded_wait_times_out_and_context_survives(torch_cuda):
+    """A wait on a barrier that nothing signals gives up after its limit and reports
+    BSA_ERR_TIMEOUT; the next launches on the same context still work and pass parity."""
+    import time
+    import block_sparse_attention_route_b200 as bsa
+    t0 = time.perf_counter()
+    bsa.bsa_selftest_bounded_wait(50000)  # 50 ms
+    assert bsa.bsa_device_status() == 4
+    assert time.perf_counter() - t0 < 5.0
+    assert bsa.bsa_device_status() == 0
+    w = WORKLOADS["tiny"]
+    pipe, _ = run_forward(w)
+    check_attention(w, pipe, [0, 1])
