@@ -18,7 +18,7 @@ from typing import Optional
 __all__ = [
     "Geometry", "BsaError", "lib", "bsa_workspace_size", "rope3d_qknorm_prologue", "bsa_route",
     "bsa_attn_fwd", "bsa_attn_bwd", "bsa_device_status", "bsa_error_string", "blocked_shape",
-    "bsa_selftest_bounded_wait",
+    "bsa_selftest_bounded_wait", "bsa_route_noalloc",
     "WS_ROUTE", "WS_FWD", "WS_BWD",
 ]
 
@@ -115,6 +115,7 @@ def lib() -> ctypes.CDLL:
             "bsa_attn_bwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
             "bsa_device_status": (I32, [P]),
             "bsa_selftest_bounded_wait": (I32, [I32, P]),
+            "bsa_route_noalloc": (I32, [G, I32, P, P, P, P, P, P]),
             "bsa_error_string": (ctypes.c_char_p, [I32]),
             "bsa_last_error_detail": (ctypes.c_char_p, []),
         }
@@ -178,6 +179,13 @@ def bsa_route(g: Geometry, top_r: int, q_blk, k_blk, q_pool, k_pool, kpool_cache
     _check(lib().bsa_route(
         ctypes.byref(g.c()), top_r, _ptr(q_blk), _ptr(k_blk), _ptr(q_pool), _ptr(k_pool),
         _ptr(kpool_cache), _ptr(idx), _ptr(cnt), _ptr(ws), nbytes, _stream(stream)), "bsa_route")
+
+
+def bsa_route_noalloc(g: Geometry, top_r: int, q_blk, k_blk, kpool_cache, idx, cnt, stream=None):
+    """bsa_route without a workspace (the library's fixed scratch array; see include/bsa.h)."""
+    _check(lib().bsa_route_noalloc(
+        ctypes.byref(g.c()), top_r, _ptr(q_blk), _ptr(k_blk), _ptr(kpool_cache), _ptr(idx),
+        _ptr(cnt), _stream(stream)), "bsa_route_noalloc")
 
 
 def bsa_attn_fwd(g: Geometry, top_r: int, q_blk, k_blk, v_blk, k_cache_blk, v_cache_blk, idx,

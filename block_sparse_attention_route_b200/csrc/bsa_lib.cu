@@ -442,3 +442,5 @@ bsa_status_t bsa_device_status(bsa_stream_t stream) {
 }
 
 }  // extern "C"
+
+#include "route_noalloc.cu"

@@ -166,6 +166,20 @@ BSA_API bsa_status_t bsa_attn_bwd(const bsa_geom_t* g, int32_t top_r, const void
  * Returns BSA_OK, BSA_ERR_TIMEOUT or BSA_ERR_BAD_INDEX (or BSA_ERR_CUDA). */
 BSA_API bsa_status_t bsa_device_status(bsa_stream_t stream);
 
+/* Routing without a caller workspace, for callers that cannot allocate device memory when they
+ * route (a serving engine that reserved the whole device up front, a host framework whose
+ * allocator owns all memory, a latency-critical path where cudaMalloc could synchronise the
+ * device).  Same result as bsa_route with q_pool = k_pool = NULL (means computed from q_blk and
+ * k_blk); the means live in a 16 MiB array inside the library, held on every device that loads
+ * it until the process exits.  Rejects geometries with B*H*NBq*D*8 > 16 MiB (after 256-byte
+ * rounding of each half) with BSA_ERR_UNSUPPORTED.  Allocates nothing.  The first call on a
+ * device looks up that array's device address (cudaGetSymbolAddress) and caches it: make it
+ * before any stream capture.  Calls share the array, so calls that overlap on the GPU race.
+ * No page counterpart: this entry point exists for callers that cannot allocate. */
+BSA_API bsa_status_t bsa_route_noalloc(const bsa_geom_t* g, int32_t top_r, const void* q_blk,
+                                       const void* k_blk, const float* kpool_cache, int32_t* idx,
+                                       int32_t* cnt, bsa_stream_t stream);
+
 /* Failure-path self test: enqueues one kernel that waits, through the same bounded wait every
  * kernel uses, on a barrier that nothing signals; after `limit_us` microseconds (1..1e6) it
  * gives up and records a timeout, which the next bsa_device_status() returns as
