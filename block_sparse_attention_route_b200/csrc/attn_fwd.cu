@@ -11,15 +11,18 @@
 // order so the CTAs running at once share one head's K/V in L2.  Each CTA keeps two items
 // in flight ("lanes" A and B) so one lane's softmax overlaps the other lane's MMAs.
 //
-// Warp roles (384 threads = 3 warpgroups):
-//   warps 0-3  softmax + epilogue of lane A (thread = query row = TMEM lane)
-//   warps 4-7  softmax + epilogue of lane B
-//   warp 8     TMA producer (one thread)
-//   warp 9     MMA issuer (one thread); owns the TMEM allocation (512 columns)
-//   warps 10-11 idle
-// Registers: launched at 168 per thread (384 x 168 = 64512); the producer/MMA warpgroup
-// drops to kRegsCtl and the two softmax warpgroups rise to kRegsSoftmax:
-// 256 * 208 + 128 * 80 = 63488 <= 64512.
+// Warp roles (640 threads = 5 warpgroups):
+//   warps 0-7   softmax + epilogue of lane A: warps 0-3 take the left half of every S row
+//               (keys 0..BS/2-1), warps 4-7 the right half; thread = query row = TMEM lane
+//   warps 8-15  the same for lane B
+//   warp 16     TMA producer (one thread)
+//   warp 17     MMA issuer (one thread); owns the TMEM allocation (512 columns)
+//   warps 18-19 idle
+// The two threads of a row exchange their partial row maxima through shared memory behind a
+// named barrier of the lane's 256 threads, so both apply the same running max; each keeps a
+// partial row sum, combined once per item.  Registers: launched at 96 per thread
+// (640 x 96 = 61440); the control warpgroup drops to kRegsCtl and the softmax warpgroups
+// rise to kRegsSoftmax: 512 * 104 + 128 * 56 = 60416 <= 61440.
 // TMEM columns: lane L uses S/P at [256L, 256L+BS) and O at [256L+128, 256L+128+D).
 // P (bf16) overwrites the first BS/2 columns of S; the next S of that lane is issued after
 // the PV that reads P, and tcgen05 MMAs of one thread execute in issue order.
@@ -43,12 +46,14 @@ struct FwdParams {
   float* lse;
 };
 
-constexpr int kFwdThreads = 384;
-constexpr int kRegsSoftmax = 208;
-constexpr int kRegsCtl = 80;
-static_assert(256 * kRegsSoftmax + 128 * kRegsCtl <= kFwdThreads * 168,
+constexpr int kFwdThreads = 640;
+constexpr int kProducerWarp = 16, kMmaWarp = 17;
+constexpr int kRegsLaunch = 96;  // 65536 / 640 rounded down to a multiple of 8
+constexpr int kRegsSoftmax = 104;
+constexpr int kRegsCtl = 56;
+static_assert(512 * kRegsSoftmax + 128 * kRegsCtl <= kFwdThreads * kRegsLaunch,
               "register re-split exceeds the launch allocation");
-constexpr int kFwdStages = 5;
+constexpr int kFwdStages = 4;
 constexpr int kTileM = 128;
 // softmax arithmetic options (see the design doc for the measurements behind the defaults)
 constexpr bool kPolyExp = false;   // half of the exponentials on the FMA pipe
@@ -65,7 +70,9 @@ struct FwdLayout {
   // barriers: q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] fin
   static constexpr int kNumBars = 2 * 5 + 2 * kFwdStages + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kBytes = kMiscOff + 16;
+  static constexpr int kXchOff = kMiscOff + 16;              // float [2 lanes][2 halves][128]
+  static constexpr int kSumOff = kXchOff + 2 * 2 * 128 * 4;  // float [2 lanes][2 halves][128]
+  static constexpr int kBytes = kSumOff + 2 * 2 * 128 * 4;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
@@ -136,7 +143,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], 128);
+      mbar_init(&p_full[i], 256);
       mbar_init(&o_full[i], 1);
     }
     for (int s = 0; s < kFwdStages; ++s) {
@@ -147,11 +154,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 9) {
+  if (warp == kMmaWarp) {
     tmem_alloc(tmem_holder, 512);
     tmem_relinquish();
   }
-  if (warp == 8 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -165,12 +172,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tc_fence_before();
     named_bar_sync(1, kFwdThreads);
     tc_fence_after();
-    if (warp == 9) tmem_dealloc(tmem_base, 512);
+    if (warp == kMmaWarp) tmem_dealloc(tmem_base, 512);
   };
 
-  if (warp >= 8) {
+  if (warp >= kProducerWarp) {
   regs_dec<kRegsCtl>();
-  if (warp == 8) {
+  if (warp == kProducerWarp) {
     // ================================================================ TMA producer
     // Walks the same schedule as the MMA thread: for each lane in turn, the V tile of the
     // current step, then (after advancing) the Q tile of a new item and the next K tile.
@@ -233,7 +240,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       if (ql0 > 0) mbar_wait_drain(&q_full[0], (ql0 - 1) & 1);
       if (ql1 > 0) mbar_wait_drain(&q_full[1], (ql1 - 1) & 1);
     }
-  } else if (warp == 9) {
+  } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTileM, BS, 0, 0);
@@ -312,11 +319,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else {
     regs_inc<kRegsSoftmax>();
     // ================================================================ softmax + epilogue
-    const int Lw = warp / 4;
-    const int row = 32 * (warp % 4) + lane;
-    const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
-    const uint32_t t_s = tmem_base + t_lane + Lw * 256;
-    const uint32_t t_o = t_s + 128;
+    constexpr int HC = BS / 2;  // S columns (keys) per thread
+    constexpr int HO = D / 2;   // O columns per thread
+    const int Lw = warp / 8, hf = (warp / 4) & 1, quarter = warp & 3;
+    const int row = 32 * quarter + lane;
+    const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
+    const uint32_t t_s = tmem_base + t_lane + Lw * 256;   // S / P of this lane
+    const uint32_t t_sh = t_s + hf * HC;                  // this thread's S columns
+    const uint32_t t_ph = t_s + hf * (HC / 2);            // this thread's P columns (bf16 pairs)
+    const uint32_t t_oh = t_s + 128 + hf * HO;            // this thread's O columns
+    float* xch = reinterpret_cast<float*>(smem + L::kXchOff) + Lw * 256;
+    float* xsum = reinterpret_cast<float*>(smem + L::kSumOff) + Lw * 256;
+    const int bar_id = 2 + Lw;
     const float sl2 = g.scale * 1.4426950408889634f;
     int scons = 0, ocons = 0;
     bool ok = true;
@@ -341,121 +355,117 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ++scons;
         tc_fence_after();
         const int j = load_idx(p, item, n);
-        float s[BS];
+        float s[HC];
         {
           uint32_t* sr = reinterpret_cast<uint32_t*>(s);
-          if constexpr (BS == 128) tmem_ld128_wait(t_s, sr);
-          else tmem_ld32_wait(t_s, sr);
+          if constexpr (HC == 64) tmem_ld64_wait(t_sh, sr);
+          else tmem_ld16_wait(t_sh, sr);
         }
         // pad keys of a partial block get -inf (mask built without divisions per column)
         int vt, vh, vw;
         if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
         else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
-        const bool partial = vt < g.bt || vh < g.bh || vw < g.bw;
-        if (partial) {
+        if (vt < g.bt || vh < g.bh || vw < g.bw) {
           uint32_t vm[BS / 32];
           block_valid_mask<BS>(g, vt, vh, vw, vm);
 #pragma unroll
-          for (int c = 0; c < BS; ++c)
-            if (!((vm[c >> 5] >> (c & 31)) & 1u)) s[c] = -INFINITY;
+          for (int c = 0; c < HC; ++c) {
+            const int kc = hf * HC + c;
+            if (!((vm[kc >> 5] >> (kc & 31)) & 1u)) s[c] = -INFINITY;
+          }
         }
-        // row max (four independent chains)
         float mx;
-        if constexpr (kMax3) {
+        {
           float a0 = s[0], a1 = s[1], a2 = s[2], a3 = s[3];
 #pragma unroll
-          for (int c = 4; c + 8 <= BS; c += 8) {
+          for (int c = 4; c + 8 <= HC; c += 8) {
             a0 = max3f(a0, s[c], s[c + 1]);
             a1 = max3f(a1, s[c + 2], s[c + 3]);
             a2 = max3f(a2, s[c + 4], s[c + 5]);
             a3 = max3f(a3, s[c + 6], s[c + 7]);
           }
-          mx = max3f(max3f(a0, a1, a2), a3, fmaxf(s[BS - 4], fmaxf(s[BS - 3], fmaxf(s[BS - 2], s[BS - 1]))));
-        } else {
-          float a0 = s[0], a1 = s[1], a2 = s[2], a3 = s[3];
-#pragma unroll
-          for (int c = 4; c < BS; c += 4) {
-            a0 = fmaxf(a0, s[c]); a1 = fmaxf(a1, s[c + 1]);
-            a2 = fmaxf(a2, s[c + 2]); a3 = fmaxf(a3, s[c + 3]);
-          }
-          mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3));
+          mx = max3f(max3f(a0, a1, a2), a3,
+                     fmaxf(s[HC - 4], fmaxf(s[HC - 3], fmaxf(s[HC - 2], s[HC - 1]))));
         }
-        mx *= sl2;
+        // exchange the half-row maxima (the partner's S columns are read by now, so the P
+        // stores below may overwrite them)
+        xch[hf * 128 + row] = mx;
+        named_bar_sync(bar_id, 256);
+        mx = fmaxf(mx, xch[(1 - hf) * 128 + row]) * sl2;
         // lazy rescale: a row raises its running max only when it grew by more than 8
-        // (log2 units).  tcgen05.ld/st are warp-collective, so the warp rescales together
-        // (alpha = 1 for rows that keep their max).  The PV of step n-1 has completed: the
-        // S of step n was issued after it and has completed.
+        // (log2 units); both threads of a row take the same decision.  tcgen05.ld/st are
+        // warp-collective, so a warp rescales together (alpha = 1 for rows that keep their
+        // max).  The PV of step n-1 has completed: the S of step n was issued after it.
         const float m_new = (n == 0 || mx > m + 8.0f) ? mx : m;
         const bool resc = n > 0 && m_new != m;
         if (__any_sync(0xffffffffu, resc)) {
           const float alpha = resc ? fast_exp2(m - m_new) : 1.0f;
           l *= alpha;
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < HO / 32; ++c) {
             uint32_t r32[32];
-            tmem_ld32_wait(t_o + c * 32, r32);
+            tmem_ld32_wait(t_oh + c * 32, r32);
 #pragma unroll
             for (int e = 0; e < 32; ++e) r32[e] = __float_as_uint(__uint_as_float(r32[e]) * alpha);
-            tmem_st32(t_o + c * 32, r32);
+            tmem_st32(t_oh + c * 32, r32);
           }
           tmem_wait_st();
         }
         m = m_new;
-        // P = exp2(s * scale * log2e - m) as bf16 pairs into the first BS/2 columns of S,
-        // 16 columns (32 keys) at a time; all of S is already in registers.  Half of the
-        // exponentials go to the FMA pipe (polynomial), half to MUFU; blocks with pad keys
-        // use MUFU only, so masked keys get exactly 0.
+        // P = exp2(s * scale * log2e - m) as bf16 pairs into this half's P columns
         const uint64_t sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(-m, -m);
         uint64_t sum2 = f2pack(0.f, 0.f);
-        float lsum = 0.f;
-        const bool poly = kPolyExp && !partial;
 #pragma unroll
-        for (int c = 0; c < BS / 32; ++c) {
+        for (int c = 0; c < HC / 32; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float s0 = s[c * 32 + 2 * e], s1 = s[c * 32 + 2 * e + 1];
-            float x0, x1, p0, p1;
-            if constexpr (kPacked) {
-              f2unpack(fma2(f2pack(s0, s1), sl2x2, nmx2), x0, x1);
-            } else {
-              x0 = fmaf(s0, sl2, -m);
-              x1 = fmaf(s1, sl2, -m);
-            }
-            if (poly && (e & 1)) {
-              exp2_poly2(f2pack(fmaxf(x0, -126.f), fmaxf(x1, -126.f)), p0, p1);
-            } else {
-              p0 = fast_exp2(x0);
-              p1 = fast_exp2(x1);
-            }
-            if constexpr (kPacked) sum2 = add2(sum2, f2pack(p0, p1));
-            else lsum += p0 + p1;
+            float x0, x1;
+            f2unpack(fma2(f2pack(s[c * 32 + 2 * e], s[c * 32 + 2 * e + 1]), sl2x2, nmx2), x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            sum2 = add2(sum2, f2pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st16(t_s + c * 16, pk);
+          tmem_st16(t_ph + c * 16, pk);
         }
-        if constexpr (kPacked) {
+        if constexpr (HC % 32 != 0) {  // BS = 32: 16 keys per thread, 8 P columns
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float x0, x1;
+            f2unpack(fma2(f2pack(s[2 * e], s[2 * e + 1]), sl2x2, nmx2), x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            sum2 = add2(sum2, f2pack(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st8(t_ph, pk);
+        }
+        {
           float l0, l1;
           f2unpack(sum2, l0, l1);
-          lsum = l0 + l1;
+          l += l0 + l1;
         }
-        l += lsum;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[Lw]);
       }
       if (!ok) break;
       float* lse_row = p.lse + (size_t)item * BS;
-      __nv_bfloat16* o_row = p.o + ((size_t)item * BS + row) * D;
+      __nv_bfloat16* o_row = p.o + ((size_t)item * BS + row) * D + hf * HO;
       if (cnt == 0) {
         if (row < BS) {
           uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(o_row)[c] = z;
-          lse_row[row] = -INFINITY;
+          for (int c = 0; c < HO / 8; ++c) reinterpret_cast<uint4*>(o_row)[c] = z;
+          if (hf == 0) lse_row[row] = -INFINITY;
         }
         continue;
       }
+      // combine the two partial row sums (own buffer: the max exchange may already be in
+      // use for the next item)
+      xsum[hf * 128 + row] = l;
+      named_bar_sync(bar_id, 256);
+      l += xsum[(1 - hf) * 128 + row];
       bool w_ok = mbar_wait(&o_full[Lw], ocons & 1, abort_flag);
       w_ok = __all_sync(0xffffffffu, w_ok);
       if (!w_ok) { ok = false; break; }
@@ -463,9 +473,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       tc_fence_after();
       const float inv_l = qvalid ? 1.0f / l : 0.f;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < HO / 32; ++c) {
         uint32_t r32[32];
-        tmem_ld32_wait(t_o + c * 32, r32);
+        tmem_ld32_wait(t_oh + c * 32, r32);
         if (row < BS) {
           uint4 v[4];
           uint32_t* v32 = reinterpret_cast<uint32_t*>(v);
@@ -477,7 +487,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           for (int e = 0; e < 4; ++e) reinterpret_cast<uint4*>(o_row + c * 32)[e] = v[e];
         }
       }
-      if (row < BS) lse_row[row] = qvalid ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      if (row < BS && hf == 0)
+        lse_row[row] = qvalid ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      // the partner must have read this thread's partial sum before it is overwritten by
+      // the next item's: the next write happens after the next item's first exchange
+      // barrier, which the partner reaches only after reading it.
     }
     teardown();
   }
