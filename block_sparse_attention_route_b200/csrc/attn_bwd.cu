@@ -152,7 +152,13 @@ __global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams
 }
 
 // ------------------------------------------------------------------------------ common
-constexpr int kBwdThreads = 192;  // warps 0-3 elementwise (thread = TMEM lane), 4 TMA, 5 MMA
+// warps 0-15 elementwise: warp w reads TMEM lanes 32*(w%4).. and owns the 32-column group
+// w/4 of every tile (S, dP: 4 x 32 columns); warp 16 TMA producer; warp 17 MMA issuer and
+// TMEM owner; warps 18-19 idle.  No row reductions are needed in the backward (P comes from
+// the stored LSE), so the column groups work independently; one named barrier per step
+// orders the loads of all groups before the bf16 stores that overwrite loaded columns.
+constexpr int kBwdThreads = 640;
+constexpr int kBwdProducer = 16, kBwdMma = 17, kBwdElem = 512;
 constexpr int kBwdStages = 2;  // Q_i + dO_i stages of the key-major pass (64 KB each)
 constexpr int kTile = 128;
 
@@ -206,13 +212,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(kv_empty, 1);
     for (int s = 0; s < kBwdStages; ++s) { mbar_init(&st_full[s], 1); mbar_init(&st_empty[s], 1); }
     mbar_init(s_full, 1);
-    mbar_init(p_full, 128);
+    mbar_init(p_full, kBwdElem);
     mbar_init(acc_full, 1);
     mbar_init(fin_bar, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 5) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  if (warp == kBwdMma) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (beg < 0 || end < beg || end > g.NBq * p.r) { set_status(DEV_BAD_INDEX); beg = end = 0; }
   };
 
-  if (warp == 4) {
+  if (warp == kBwdProducer) {
     // ====================================================== TMA producer
     if (lane == 0) {
       int seq = 0, items = 0;
@@ -273,7 +279,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (items > 0) mbar_wait_drain(kv_full, (items - 1) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == kBwdMma) {
     // ====================================================== MMA issuer
     if (lane == 0) {
       constexpr uint32_t idSS = idesc_bf16(kTile, BS, 0, 0);   // S^T, dP^T: both K-major
@@ -333,9 +339,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit(fin_bar);
       mbar_wait_drain(fin_bar, 0);
     }
-  } else {
+  } else if (warp < kBwdElem / 32) {
     // ====================================================== elementwise + epilogue
     const int row = 32 * (warp % 4) + lane;  // key slot within the block
+    const int cg = warp / 4;                 // 32-column group
     const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
     const uint32_t t_s = tmem_base + t_lane, t_dp = t_s + 128, t_dv = t_s + 256, t_dk = t_s + 384;
     const float sl2 = g.scale * 1.4426950408889634f;
@@ -358,29 +365,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float* vec = reinterpret_cast<const float*>(smem + L::kVecOff + stage * L::kVecBytes);
         const float* lse2 = vec;
         const float* dlt = vec + BS;
-        // 32 query columns at a time: P^T = exp2(S^T*sl2 - lse2[q]),
-        // dS^T = P^T * (dP^T - delta[q]); bf16 results overwrite already-read columns.
-#pragma unroll 1
-        for (int c = 0; c < BS / 32; ++c) {
+        // this group's 32 query columns: P^T = exp2(S^T*sl2 - lse2[q]),
+        // dS^T = P^T * (dP^T - delta[q]); bf16 results go to columns [16cg, 16cg+16), which
+        // another group may still be reading until the barrier.
+        {
           uint32_t sr[32], dr[32], pk[16], dk[16];
-          tmem_ld32_wait(t_s + c * 32, sr);
-          tmem_ld32_wait(t_dp + c * 32, dr);
+          tmem_ld32_wait(t_s + cg * 32, sr);
+          tmem_ld32_wait(t_dp + cg * 32, dr);
 #pragma unroll
           for (int e2 = 0; e2 < 16; ++e2) {
-            const int q0 = c * 32 + 2 * e2;
+            const int q0 = cg * 32 + 2 * e2;
             const float2 ld = *reinterpret_cast<const float2*>(lse2 + q0);
             const float2 dd = *reinterpret_cast<const float2*>(dlt + q0);
-            const float l0 = ld.x, l1 = ld.y, d0 = dd.x, d1 = dd.y;
-            float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -l0));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -l1));
+            float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -ld.x));
+            float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -ld.y));
             if (!kvalid) { p0 = 0.f; p1 = 0.f; }
-            const float s0 = p0 * (__uint_as_float(dr[2 * e2]) - d0);
-            const float s1 = p1 * (__uint_as_float(dr[2 * e2 + 1]) - d1);
+            const float s0 = p0 * (__uint_as_float(dr[2 * e2]) - dd.x);
+            const float s1 = p1 * (__uint_as_float(dr[2 * e2 + 1]) - dd.y);
             pk[e2] = pack_bf16x2(p0, p1);
             dk[e2] = pack_bf16x2(s0, s1);
           }
-          tmem_st16(t_s + c * 16, pk);
-          tmem_st16(t_dp + c * 16, dk);
+          named_bar_sync(1, kBwdElem);
+          tmem_st16(t_s + cg * 16, pk);
+          tmem_st16(t_dp + cg * 16, dk);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -398,33 +405,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         w_ok = __all_sync(0xffffffffu, w_ok);
         if (!w_ok) { ok = false; break; }
         tc_fence_after();
-#pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t a[32], bk[32];
-          tmem_ld32_wait(t_dv + c * 32, a);
-          tmem_ld32_wait(t_dk + c * 32, bk);
-          uint4 va[4], vb[4];
-          uint32_t* a32 = reinterpret_cast<uint32_t*>(va);
-          uint32_t* b32 = reinterpret_cast<uint32_t*>(vb);
+        constexpr int DC = D / 4;  // dV / dK columns of this group
+        uint32_t a[DC], bk[DC];
+        if constexpr (DC == 32) {
+          tmem_ld32_wait(t_dv + cg * DC, a);
+          tmem_ld32_wait(t_dk + cg * DC, bk);
+        } else {
+          tmem_ld16_wait(t_dv + cg * DC, a);
+          tmem_ld16_wait(t_dk + cg * DC, bk);
+        }
+        uint4 va[DC / 8], vb[DC / 8];
+        uint32_t* a32 = reinterpret_cast<uint32_t*>(va);
+        uint32_t* b32 = reinterpret_cast<uint32_t*>(vb);
 #pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            a32[e2] = kvalid ? pack_bf16x2(__uint_as_float(a[2 * e2]), __uint_as_float(a[2 * e2 + 1])) : 0u;
-            b32[e2] = kvalid ? pack_bf16x2(__uint_as_float(bk[2 * e2]) * g.scale,
-                                           __uint_as_float(bk[2 * e2 + 1]) * g.scale)
-                             : 0u;
-          }
+        for (int e2 = 0; e2 < DC / 2; ++e2) {
+          a32[e2] = kvalid ? pack_bf16x2(__uint_as_float(a[2 * e2]), __uint_as_float(a[2 * e2 + 1])) : 0u;
+          b32[e2] = kvalid ? pack_bf16x2(__uint_as_float(bk[2 * e2]) * g.scale,
+                                         __uint_as_float(bk[2 * e2 + 1]) * g.scale)
+                           : 0u;
+        }
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) {
-            reinterpret_cast<uint4*>(dv_row + c * 32)[e2] = va[e2];
-            reinterpret_cast<uint4*>(dk_row + c * 32)[e2] = vb[e2];
-          }
+        for (int e2 = 0; e2 < DC / 8; ++e2) {
+          reinterpret_cast<uint4*>(dv_row + cg * DC)[e2] = va[e2];
+          reinterpret_cast<uint4*>(dk_row + cg * DC)[e2] = vb[e2];
         }
       } else {
         const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          reinterpret_cast<uint4*>(dv_row)[c] = z;
-          reinterpret_cast<uint4*>(dk_row)[c] = z;
+        for (int c = 0; c < D / 32; ++c) {
+          reinterpret_cast<uint4*>(dv_row + cg * (D / 4))[c] = z;
+          reinterpret_cast<uint4*>(dk_row + cg * (D / 4))[c] = z;
         }
       }
       if (end > beg) ++items;
@@ -433,7 +443,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem_base, 512);
+  if (warp == kBwdMma) tmem_dealloc(tmem_base, 512);
 }
 
 // ------------------------------------------------------------------------------ dQ
@@ -486,14 +496,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_init(q_full, 1);
     mbar_init(q_empty, 1);
     for (int s = 0; s < S; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&s_full[b], 1); mbar_init(&ds_full[b], 128); }
-    mbar_init(dp_free, 128);
+    for (int b = 0; b < 2; ++b) { mbar_init(&s_full[b], 1); mbar_init(&ds_full[b], kBwdElem); }
+    mbar_init(dp_free, kBwdElem);
     mbar_init(dq_full, 1);
     mbar_init(fin_bar, 1);
     *abort_flag = 0;
     mbar_fence_init();
   }
-  if (warp == 5) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  if (warp == kBwdMma) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -510,7 +520,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     return j;
   };
 
-  if (warp == 4) {
+  if (warp == kBwdProducer) {
     // ====================================================== TMA producer: per step K_n, V_n
     if (lane == 0) {
       int seq = 0, qloads = 0;
@@ -551,7 +561,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       if (qloads > 0) mbar_wait_drain(q_full, (qloads - 1) & 1);
     }
-  } else if (warp == 5) {
+  } else if (warp == kBwdMma) {
     // ====================================================== MMA issuer
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTile, BS, 0, 0);
@@ -635,9 +645,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mma_commit(fin_bar);
       mbar_wait_drain(fin_bar, 0);
     }
-  } else {
+  } else if (warp < kBwdElem / 32) {
     // ====================================================== elementwise + epilogue
     const int row = 32 * (warp % 4) + lane;  // query row of the 128-row tile
+    const int cg = warp / 4;                 // 32-column group (BS / 4 keys)
     const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
     const uint32_t t_dp = tmem_base + t_lane + 256, t_dq = tmem_base + t_lane + 384;
     const float sl2 = g.scale * 1.4426950408889634f;
@@ -651,7 +662,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (row < BS) {
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int c = 0; c < D / 8; ++c) reinterpret_cast<uint4*>(dq_row)[c] = z;
+          for (int c = 0; c < D / 32; ++c) reinterpret_cast<uint4*>(dq_row + cg * (D / 4))[c] = z;
         }
         continue;
       }
@@ -664,10 +675,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!w_ok) { ok = false; break; }
         ++sfc[b];
         tc_fence_after();
-        // dP row first, then release its columns for dP(n+1)
-        uint32_t dpr[BS];
-        if constexpr (BS == 128) tmem_ld128_wait(t_dp, dpr);
-        else tmem_ld32_wait(t_dp, dpr);
+        // this group's BS/4 key columns of dP and S; release dP for dP(n+1) once read
+        constexpr int KC = BS / 4;
+        uint32_t dpr[KC], sr[KC], pk[KC / 2];
+        const uint32_t t_s = tmem_base + t_lane + b * 128;
+        if constexpr (KC == 32) {
+          tmem_ld32_wait(t_dp + cg * KC, dpr);
+          tmem_ld32_wait(t_s + cg * KC, sr);
+        } else {
+          tmem_ld16_wait(t_dp + cg * KC, dpr);
+          tmem_ld16_wait(t_s + cg * KC, sr);
+        }
         tc_fence_before();
         mbar_arrive(dp_free);
         // pad keys of a partial key block: P = 0
@@ -679,24 +697,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int w2 = 0; w2 < BS / 32; ++w2) vm[w2] = 0xFFFFFFFFu;
         if (vt < g.bt || vh < g.bh || vw < g.bw) block_valid_mask<BS>(g, vt, vh, vw, vm);
-        const uint32_t t_s = tmem_base + t_lane + b * 128;
 #pragma unroll
-        for (int c = 0; c < BS / 32; ++c) {
-          uint32_t sr[32], pk[16];
-          tmem_ld32_wait(t_s + c * 32, sr);
-#pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            const int k0 = c * 32 + 2 * e2;
-            float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -l2));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -l2));
-            if (!((vm[k0 >> 5] >> (k0 & 31)) & 1u)) p0 = 0.f;
-            if (!((vm[(k0 + 1) >> 5] >> ((k0 + 1) & 31)) & 1u)) p1 = 0.f;
-            const float d0 = p0 * (__uint_as_float(dpr[k0]) - dl);
-            const float d1 = p1 * (__uint_as_float(dpr[k0 + 1]) - dl);
-            pk[e2] = pack_bf16x2(d0, d1);
-          }
-          tmem_st16(t_s + c * 16, pk);
+        for (int e2 = 0; e2 < KC / 2; ++e2) {
+          const int k0 = cg * KC + 2 * e2;
+          float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -l2));
+          float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -l2));
+          if (!((vm[k0 >> 5] >> (k0 & 31)) & 1u)) p0 = 0.f;
+          if (!((vm[(k0 + 1) >> 5] >> ((k0 + 1) & 31)) & 1u)) p1 = 0.f;
+          pk[e2] = pack_bf16x2(p0 * (__uint_as_float(dpr[2 * e2]) - dl),
+                               p1 * (__uint_as_float(dpr[2 * e2 + 1]) - dl));
         }
+        // dS goes to columns [KC/2 * cg, ..): other groups may still be reading them
+        named_bar_sync(1, kBwdElem);
+        if constexpr (KC == 32) tmem_st16(t_s + cg * (KC / 2), pk);
+        else tmem_st8(t_s + cg * (KC / 2), pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ds_full[b]);
@@ -707,20 +721,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       if (!w_ok) { ok = false; break; }
       ++dqc;
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[32];
-        tmem_ld32_wait(t_dq + c * 32, a);
+      {
+        constexpr int DC = D / 4;
+        uint32_t a[DC];
+        if constexpr (DC == 32) tmem_ld32_wait(t_dq + cg * DC, a);
+        else tmem_ld16_wait(t_dq + cg * DC, a);
         if (row < BS) {
-          uint4 v[4];
+          uint4 v[DC / 8];
           uint32_t* v32 = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2)
+          for (int e2 = 0; e2 < DC / 2; ++e2)
             v32[e2] = (l2 == INFINITY) ? 0u
                                        : pack_bf16x2(__uint_as_float(a[2 * e2]) * g.scale,
                                                      __uint_as_float(a[2 * e2 + 1]) * g.scale);
 #pragma unroll
-          for (int e2 = 0; e2 < 4; ++e2) reinterpret_cast<uint4*>(dq_row + c * 32)[e2] = v[e2];
+          for (int e2 = 0; e2 < DC / 8; ++e2) reinterpret_cast<uint4*>(dq_row + cg * DC)[e2] = v[e2];
         }
       }
     }
@@ -728,7 +743,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 5) tmem_dealloc(tmem_base, 512);
+  if (warp == kBwdMma) tmem_dealloc(tmem_base, 512);
 }
 
 // ------------------------------------------------------------------------------ host side
