@@ -108,6 +108,10 @@ bsa_status_t make_geo(const bsa_geom_t* gi, Geo* out) {
   g.B = a.batch; g.H = a.heads; g.D = a.head_dim;
   g.T = a.t_frames; g.GH = a.grid_h; g.GW = a.grid_w; g.Tc = a.cached_t;
   g.bt = a.blk_t; g.bh = a.blk_h; g.bw = a.blk_w; g.BS = (int)bs;
+  g.lbh = 0;
+  while ((1 << g.lbh) < g.bh) ++g.lbh;
+  g.lbw = 0;
+  while ((1 << g.lbw) < g.bw) ++g.lbw;
   g.nbh = (a.grid_h + a.blk_h - 1) / a.blk_h;
   g.nbw = (a.grid_w + a.blk_w - 1) / a.blk_w;
   g.nbt_q = (a.t_frames + a.blk_t - 1) / a.blk_t;

@@ -22,7 +22,8 @@ struct Geo {
   int B, H, D;
   int T, GH, GW;        // current frames and valid grid
   int Tc;               // cached frames
-  int bt, bh, bw, BS;   // block shape
+  int bt, bh, bw, BS;   // block shape (powers of two: BS is 32 or 128)
+  int lbh, lbw;         // log2(bh), log2(bw): slot (lt, lh, lw) = (s >> (lbh+lbw), (s >> lbw) & (bh-1), s & (bw-1))
   int nbh, nbw;         // blocks along h and w
   int nbt_q, nbt_c;     // blocks along t for current / cached frames
   int NBq, NBc, NBk;    // query blocks, cached key blocks, all key blocks

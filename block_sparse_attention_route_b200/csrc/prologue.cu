@@ -6,9 +6,11 @@
 //
 // HBM-bound: every (token, head) row of q, k, v is read once (D bf16) and written once to
 // its slot of the blocked layout; pad slots are written as zeros.  One CTA handles one
-// block of the padded grid for up to 8 heads; D/8 lanes own one row (16-byte vectors), so a
-// warp moves 512 contiguous bytes per instruction on both sides.  The cos/sin table of the
-// block's (t, h, w) positions is built once per CTA in shared memory (fp64 angles).
+// block of the padded grid for 8 heads; D/8 lanes own one row (16-byte vectors).  Rows are
+// visited slot-major, head-minor, so consecutive row groups read consecutive heads of one
+// token (a contiguous 8 x D x 2-byte run of the raster) and every lane keeps one head.
+// The cos/sin table of the block's (t, h, w) positions is built once per CTA in shared
+// memory (fp64 angles).
 #include "common.cuh"
 
 namespace bsa {
@@ -71,7 +73,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
 
   const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
   const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
-  const int rows = heads_here * g.BS;
+  const int rows = kHeadsPerCta * g.BS;  // (slot, head) pairs; heads >= heads_here are skipped
   const size_t n_raster = (size_t)a.frames * g.GH * g.GW;
 
   // RoPE coordinates of this lane's 4 channel pairs: axis (0 t, 1 h, 2 w) and pair index.
@@ -101,10 +103,10 @@ __global__ void __launch_bounds__(kPrologueThreads)
     int cur_h = -1;
     for (int base = 0; base < rows; base += RPP) {
       const int row = base + rid;
-      const bool in = row < rows;
-      const int hl = in ? row / g.BS : cur_h, slot = row % g.BS;
+      const int hl = row % kHeadsPerCta, slot = row / kHeadsPerCta;
+      const bool in = row < rows && hl < heads_here;
       const int h = hg * kHeadsPerCta + hl;
-      const int lt = slot / (g.bh * g.bw), lh = (slot / g.bw) % g.bh, lw = slot % g.bw;
+      const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
       const bool valid = in && lt < vt && lh < vh && lw < vw;
       float v[8];
       if (valid) {

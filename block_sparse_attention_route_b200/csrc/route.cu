@@ -30,7 +30,7 @@ __global__ void __launch_bounds__(kPoolThreads)
   const __nv_bfloat16* base = x + (((size_t)b * g.H + h) * nb + blk) * (size_t)g.BS * D;
   float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
   for (int slot = rg; slot < g.BS; slot += RG) {
-    const int lt = slot / (g.bh * g.bw), lh = (slot / g.bw) % g.bh, lw = slot % g.bw;
+    const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
     if (lt < vt && lh < vh && lw < vw) {
       const uint4 raw = __ldg(reinterpret_cast<const uint4*>(base + (size_t)slot * D + cc * 8));
       const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
