@@ -22,9 +22,14 @@
 // S(n+2) into the buffer P(n) came from (tcgen05 MMAs of one thread run in issue order, so
 // S(n+2) is written after PV(n) has read P(n)).
 //
-// The four column groups of a row exchange partial row maxima through shared memory behind
-// a named barrier (one per step; the exchange slots alternate with the step parity) and keep
-// partial row sums, combined once per item.  Online softmax in the exp2 domain with lazy
+// The four column groups of a row (warps q, q+4, q+8, q+12: the same TMEM lanes) exchange
+// partial row maxima through shared memory behind a named barrier of those 128 threads (one
+// per step; the exchange slots alternate with the step parity) and keep partial row sums,
+// combined once per item.  The barrier also orders every group's read of S(n) before any
+// group overwrites it with P(n).  The four row quarters run independently: P-ready is one
+// mbarrier per S buffer, so the phases of one barrier are two steps apart and a quarter can
+// never arrive for step n+2 before the MMA thread has consumed step n (S(n+2) is issued only
+// after PV(n)).  Online softmax in the exp2 domain with lazy
 // rescaling: the running max is raised only when a row's max grows by more than 8 (log2
 // units), so O is rarely touched (and then only after the previous PV has completed, which
 // the pv_done barrier tells); the final O / l and LSE are exact either way.
@@ -59,8 +64,8 @@ struct FwdLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kQBytes;
   static constexpr int kBarOff = kRingOff + kFwdStages * kKVBytes;
-  // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full pv_done o_full fin
-  static constexpr int kNumBars = 4 + 2 * kFwdStages + 2 + 4;
+  // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done o_full fin
+  static constexpr int kNumBars = 4 + 2 * kFwdStages + 2 + 2 + 3;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kXchOff = kMiscOff + 16;               // float [2 parity][4 groups][128]
   static constexpr int kSumOff = kXchOff + 2 * 4 * 128 * 4;   // float [4 groups][128]
@@ -102,8 +107,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* kv_full = bars + 4;       // [S]
   uint64_t* kv_empty = kv_full + S;   // [S]
   uint64_t* s_full = kv_empty + S;    // [2] S(n) in buffer n & 1
-  uint64_t* p_full = s_full + 2;      // P(n) written (kSoftmaxThreads arrivals)
-  uint64_t* pv_done = p_full + 1;     // PV(n) complete
+  uint64_t* p_full = s_full + 2;      // [2] P(n) written into buffer n & 1 (kSoftmaxThreads arrivals)
+  uint64_t* pv_done = p_full + 2;     // PV(n) complete
   uint64_t* o_full = pv_done + 1;     // O of the item complete
   uint64_t* fin_bar = o_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
@@ -117,12 +122,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       mbar_init(&q_full[i], 1);
       mbar_init(&q_empty[i], 1);
       mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kSoftmaxThreads);
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(p_full, kSoftmaxThreads);
     mbar_init(pv_done, 1);
     mbar_init(o_full, 1);
     mbar_init(fin_bar, 1);
@@ -212,9 +217,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
         return stage;
       };
-      auto issue_S = [&](uint64_t dq) -> bool {  // S(gs) = Q K^T into buffer gs & 1
-        const int stage = wait_tile();
-        if (stage < 0) return false;
+      // S(gs) = Q K^T into buffer gs & 1 from the K tile in ring stage `stage`
+      auto mma_S = [&](uint64_t dq, int stage) {
         const uint64_t kb = dk + (uint64_t)((stage * L::kKVBytes) >> 4);
         const uint32_t d_s = tmem_base + (gs & 1) * 128;
 #pragma unroll
@@ -223,42 +227,60 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t offk = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
           mma_ss(d_s, dq + offq, kb + offk, idS, kk > 0 ? 1u : 0u);
         }
-        mma_commit(&kv_empty[stage]);
-        mma_commit(&s_full[gs & 1]);
-        ++gs;
-        ++seq;
-        return true;
       };
+      // Every wait comes before the MMAs it guards, so each step issues one uninterrupted
+      // group (PV(n) then S(n+2): 2 * D/16 or BS/16 + D/16 MMAs) followed by its commits;
+      // a wait or commit between MMAs would let the tensor pipe drain.
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const int cnt = load_cnt(p, item);
         if (cnt == 0) continue;
         const int qb = items & 1;
         if (!mbar_wait(&q_full[qb], (items >> 1) & 1, abort_flag)) { ok = false; break; }
-        tc_fence_after();
         ++items;
+        const int k0 = wait_tile();
+        ++seq;
+        const int k1 = (k0 >= 0 && cnt >= 2) ? wait_tile() : -1;
+        if (cnt >= 2) ++seq;
+        if (k0 < 0 || (cnt >= 2 && k1 < 0)) { ok = false; break; }
+        tc_fence_after();
         const uint64_t dq = dq0 + (uint64_t)((qb * L::kQBytes) >> 4);
-        ok = issue_S(dq) && (cnt < 2 || issue_S(dq));
+        const int gs0 = gs;
+        mma_S(dq, k0);
+        ++gs;
+        if (cnt >= 2) { mma_S(dq, k1); ++gs; }
+        mma_commit(&s_full[gs0 & 1]);
+        if (cnt >= 2) mma_commit(&s_full[(gs0 + 1) & 1]);
+        mma_commit(&kv_empty[k0]);
+        if (cnt >= 2) mma_commit(&kv_empty[k1]);
         for (int n = 0; n < cnt && ok; ++n) {
+          const int sv = wait_tile();
+          ++seq;
+          const bool more = n + 2 < cnt;
+          const int sk = (sv >= 0 && more) ? wait_tile() : -1;
+          if (more) ++seq;
+          if (sv < 0 || (more && sk < 0)) { ok = false; break; }
           // O += P(n) V(n): A = P from TMEM (buffer gp & 1), B = V (MN-major)
-          if (!mbar_wait(p_full, gp & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&p_full[gp & 1], (gp >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const int stage = wait_tile();
-          if (stage < 0) { ok = false; break; }
-          const uint64_t vb = dv + (uint64_t)((stage * L::kKVBytes) >> 4);
+          const uint64_t vb = dv + (uint64_t)((sv * L::kKVBytes) >> 4);
           const uint32_t a_p = tmem_base + (gp & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < BS / 16; ++kk)
             mma_ts(t_o0, a_p + kk * 8, vb + (uint64_t)((kk * 2048) >> 4), idPV,
                    (n > 0 || kk > 0) ? 1u : 0u);
-          mma_commit(&kv_empty[stage]);
+          if (more) {  // S(n+2) into the buffer P(n) came from (read above, in issue order)
+            mma_S(dq, sk);
+            mma_commit(&s_full[gs & 1]);
+            ++gs;
+          }
           mma_commit(pv_done);
           if (n == cnt - 1) {
             mma_commit(o_full);
             mma_commit(&q_empty[qb]);
           }
+          mma_commit(&kv_empty[sv]);
+          if (more) mma_commit(&kv_empty[sk]);
           ++gp;
-          ++seq;
-          if (n + 2 < cnt) ok = issue_S(dq);
         }
       }
       // all MMAs issued by this thread must finish before TMEM is released
@@ -301,8 +323,25 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         continue;
       }
       float m = -INFINITY, l = 0.f;
+      // Key-block indices are fetched 32 steps at a time (lane e holds step n0+e) together
+      // with a ballot of the steps whose block is partial, so no global load or index
+      // arithmetic sits between a step's S and its P.
+      int jreg = 0;
+      uint32_t partial = 0;
       for (int n = 0; n < cnt; ++n, ++gstep) {
         const int b = gstep & 1;
+        if ((n & 31) == 0) {
+          const int nn = n + lane;
+          bool part = false;
+          if (nn < cnt) {
+            jreg = load_idx(p, item, nn);
+            int vt, vh, vw;
+            if (jreg < g.NBc) block_extent(g, g.Tc, jreg, vt, vh, vw);
+            else block_extent(g, g.T, jreg - g.NBc, vt, vh, vw);
+            part = vt < g.bt || vh < g.bh || vw < g.bw;
+          }
+          partial = __ballot_sync(0xffffffffu, part);
+        }
         bool w_ok = mbar_wait(&s_full[b], (gstep >> 1) & 1, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
         if (!w_ok) { ok = false; break; }
@@ -315,11 +354,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           else tmem_ld8_wait(t_s + cg * KC, sr);
         }
         // pad keys of a partial block get -inf (mask built without divisions per column)
-        const int j = load_idx(p, item, n);
-        int vt, vh, vw;
-        if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
-        else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
-        if (vt < g.bt || vh < g.bh || vw < g.bw) {
+        if ((partial >> (n & 31)) & 1u) {
+          const int j = __shfl_sync(0xffffffffu, jreg, n & 31);
+          int vt, vh, vw;
+          if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
+          else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
           uint32_t vm[BS / 32];
           block_valid_mask<BS>(g, vt, vh, vw, vm);
           uint32_t word = vm[0];
@@ -344,7 +383,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         // exchange the four partial row maxima; the slots alternate with the step parity
         float* xs = xch + b * 512;
         xs[cg * 128 + row] = mx;
-        named_bar_sync(1, kSoftmaxThreads);
+        named_bar_sync(1 + quarter, kSoftmaxThreads / 4);
         mx = fmaxf(fmaxf(xs[row], xs[128 + row]), fmaxf(xs[256 + row], xs[384 + row])) * sl2;
         // lazy rescale: raise the running max only when it grew by more than 8 (log2 units);
         // all four threads of a row take the same decision.  tcgen05.ld/st are warp-collective,
@@ -390,12 +429,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(p_full);
+        mbar_arrive(&p_full[b]);
       }
       if (!ok) break;
       // combine the four partial row sums
       xsum[cg * 128 + row] = l;
-      named_bar_sync(1, kSoftmaxThreads);
+      named_bar_sync(1 + quarter, kSoftmaxThreads / 4);
       l = (xsum[row] + xsum[128 + row]) + (xsum[256 + row] + xsum[384 + row]);
       bool w_ok = mbar_wait(o_full, ocons & 1, abort_flag);
       w_ok = __all_sync(0xffffffffu, w_ok);
