@@ -69,7 +69,8 @@ struct FwdLayout {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kXchOff = kMiscOff + 16;               // float [2 parity][4 groups][128]
   static constexpr int kSumOff = kXchOff + 2 * 4 * 128 * 4;   // float [4 groups][128]
-  static constexpr int kBytes = kSumOff + 4 * 128 * 4;
+  static constexpr int kMaskOff = kSumOff + 4 * 128 * 4;     // u32 [12 shapes][BS / 32]
+  static constexpr int kBytes = kMaskOff + 12 * (BS / 32) * 4;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
@@ -142,6 +143,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+  }
+  // Pad-key masks of the partial key-block shapes, indexed by shape code
+  // (t class * 2 + h partial) * 2 + w partial, t class 0 full / 1 last cache t-block /
+  // 2 last current t-block; bit k of word k / 32 = slot k holds a token.
+  if (tid < 12) {
+    const int tcls = tid >> 2, hp = (tid >> 1) & 1, wp = tid & 1;
+    const int rt = tcls == 1 ? g.Tc % g.bt : g.T % g.bt, rh = g.GH % g.bh, rw = g.GW % g.bw;
+    const int vt = tcls == 0 ? g.bt : rt, vh = hp ? rh : g.bh, vw = wp ? rw : g.bw;
+    uint32_t mw[BS / 32];
+    block_valid_mask<BS>(g, vt, vh, vw, mw);
+    uint32_t* mtab = reinterpret_cast<uint32_t*>(smem + L::kMaskOff);
+#pragma unroll
+    for (int w2 = 0; w2 < BS / 32; ++w2) mtab[tid * (BS / 32) + w2] = mw[w2];
   }
   tc_fence_before();
   __syncthreads();
@@ -231,8 +245,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       // Every wait comes before the MMAs it guards, so each step issues one uninterrupted
       // group (PV(n) then S(n+2): 2 * D/16 or BS/16 + D/16 MMAs) followed by its commits;
       // a wait or commit between MMAs would let the tensor pipe drain.
+      int cnt_next = (int)blockIdx.x < p.n_items ? load_cnt(p, blockIdx.x) : 0;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        const int cnt = load_cnt(p, item);
+        const int cnt = cnt_next;
+        cnt_next = item + (int)gridDim.x < p.n_items ? load_cnt(p, item + gridDim.x) : 0;
         if (cnt == 0) continue;
         const int qb = items & 1;
         if (!mbar_wait(&q_full[qb], (items >> 1) & 1, abort_flag)) { ok = false; break; }
@@ -300,8 +316,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const float sl2 = g.scale * 1.4426950408889634f;
     int gstep = 0, ocons = 0;  // global step (= S buffer use / P / PV index)
     bool ok = true;
+    int cnt_next = (int)blockIdx.x < p.n_items ? load_cnt(p, blockIdx.x) : 0;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-      const int cnt = load_cnt(p, item);
+      const int cnt = cnt_next;  // the next item's count is fetched one item ahead
+      cnt_next = item + (int)gridDim.x < p.n_items ? load_cnt(p, item + gridDim.x) : 0;
       const int i = item % g.NBq;
       // this row's query slot (rows >= BS belong to the tile's padding and are discarded)
       bool qvalid = false;
@@ -323,24 +341,27 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         continue;
       }
       float m = -INFINITY, l = 0.f;
-      // Key-block indices are fetched 32 steps at a time (lane e holds step n0+e) together
-      // with a ballot of the steps whose block is partial, so no global load or index
-      // arithmetic sits between a step's S and its P.
-      int jreg = 0;
+      // Key-block indices come 32 steps at a time (lane e holds step n0 + e), the next chunk's
+      // load in flight while the current one runs; per chunk a ballot marks the steps whose
+      // block is partial and each lane keeps its step's shape code, so no global load or
+      // index arithmetic sits between a step's S and its P.
+      int jnext = lane < cnt ? load_idx(p, item, lane) : 0;
+      int creg = 0;
       uint32_t partial = 0;
       for (int n = 0; n < cnt; ++n, ++gstep) {
         const int b = gstep & 1;
         if ((n & 31) == 0) {
-          const int nn = n + lane;
-          bool part = false;
-          if (nn < cnt) {
-            jreg = load_idx(p, item, nn);
+          const int jcur = jnext;
+          jnext = n + 32 + lane < cnt ? load_idx(p, item, n + 32 + lane) : 0;
+          creg = 0;
+          if (n + lane < cnt) {
             int vt, vh, vw;
-            if (jreg < g.NBc) block_extent(g, g.Tc, jreg, vt, vh, vw);
-            else block_extent(g, g.T, jreg - g.NBc, vt, vh, vw);
-            part = vt < g.bt || vh < g.bh || vw < g.bw;
+            if (jcur < g.NBc) block_extent(g, g.Tc, jcur, vt, vh, vw);
+            else block_extent(g, g.T, jcur - g.NBc, vt, vh, vw);
+            const int tcls = vt < g.bt ? (jcur < g.NBc ? 1 : 2) : 0;
+            creg = (tcls * 2 + (vh < g.bh ? 1 : 0)) * 2 + (vw < g.bw ? 1 : 0);
           }
-          partial = __ballot_sync(0xffffffffu, part);
+          partial = __ballot_sync(0xffffffffu, creg != 0);
         }
         bool w_ok = mbar_wait(&s_full[b], (gstep >> 1) & 1, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
@@ -353,18 +374,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           if constexpr (KC == 32) tmem_ld32_wait(t_s + cg * KC, sr);
           else tmem_ld8_wait(t_s + cg * KC, sr);
         }
-        // pad keys of a partial block get -inf (mask built without divisions per column)
+        // pad keys of a partial block get -inf (mask from the per-shape table)
         if ((partial >> (n & 31)) & 1u) {
-          const int j = __shfl_sync(0xffffffffu, jreg, n & 31);
-          int vt, vh, vw;
-          if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
-          else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
-          uint32_t vm[BS / 32];
-          block_valid_mask<BS>(g, vt, vh, vw, vm);
-          uint32_t word = vm[0];
-#pragma unroll
-          for (int w2 = 1; w2 < BS / 32; ++w2)
-            if (KC == 32 && cg == w2) word = vm[w2];
+          const int code = __shfl_sync(0xffffffffu, creg, n & 31);
+          const uint32_t* mtab = reinterpret_cast<const uint32_t*>(smem + L::kMaskOff);
+          uint32_t word = mtab[code * (BS / 32) + (KC == 32 ? cg : 0)];
           if (KC < 32) word >>= cg * KC;
 #pragma unroll
           for (int c = 0; c < KC; ++c)
