@@ -155,8 +155,11 @@ __global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams
 // warps 0-15 elementwise: warp w reads TMEM lanes 32*(w%4).. and owns the 32-column group
 // w/4 of every tile (S, dP: 4 x 32 columns); warp 16 TMA producer; warp 17 MMA issuer and
 // TMEM owner; warps 18-19 idle.  No row reductions are needed in the backward (P comes from
-// the stored LSE), so the column groups work independently; one named barrier per step
-// orders the loads of all groups before the bf16 stores that overwrite loaded columns.
+// the stored LSE), so the column groups work independently; per step a named barrier of the
+// four warps that share a row quarter's TMEM lanes (w, w+4, w+8, w+12) orders their loads
+// before the bf16 stores that overwrite loaded columns.  The quarters run independently:
+// every arrive-counted mbarrier they signal is consumed before the MMA that lets any thread
+// signal its next phase is issued, so no phase can be overrun.
 constexpr int kBwdThreads = 640;
 constexpr int kBwdProducer = 16, kBwdMma = 17, kBwdElem = 512;
 constexpr int kBwdStages = 2;  // Q_i + dO_i stages of the key-major pass (64 KB each)
@@ -385,7 +388,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             pk[e2] = pack_bf16x2(p0, p1);
             dk[e2] = pack_bf16x2(s0, s1);
           }
-          named_bar_sync(1, kBwdElem);
+          // the bf16 columns overlap other groups' S^T / dP^T columns of the same lanes
+          named_bar_sync(1 + (warp & 3), kBwdElem / 4);
           tmem_st16(t_s + cg * 16, pk);
           tmem_st16(t_dp + cg * 16, dk);
         }
@@ -463,7 +467,8 @@ struct DqLayout {
   // q_full, q_empty, kv_full[5], kv_empty[5], s_full[2], dp_free, ds_full[2], dq_full, fin
   static constexpr int kNumBars = 2 + 2 * kStages + 2 + 1 + 2 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kAlloc = kMiscOff + 16 + 1024;
+  static constexpr int kMaskOff = kMiscOff + 16;  // u32 [12 shapes][BS / 32]
+  static constexpr int kAlloc = kMaskOff + 12 * (BS / 32) * 4 + 1024;
 };
 
 template <int BS, int D>
@@ -504,6 +509,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_fence_init();
   }
   if (warp == kBwdMma) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
+  if (tid < 12) fill_shape_mask<BS>(g, tid, reinterpret_cast<uint32_t*>(smem + L::kMaskOff));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -668,8 +674,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       }
       const float l2 = row < BS ? p.lse2[qrow] : INFINITY;   // +inf: pad row -> P = 0
       const float dl = row < BS ? p.delta[qrow] : 0.f;
+      // key-block indices 32 steps at a time, the next chunk's load in flight; per chunk a
+      // ballot of the partial blocks and each lane's shape code (as in the forward)
+      int jnext = lane < cnt ? item_idx(item, lane) : 0;
+      int creg = 0;
+      uint32_t partial = 0;
       for (int n = 0; n < cnt; ++n) {
         const int b = n & 1;
+        if ((n & 31) == 0) {
+          const int jcur = jnext;
+          jnext = n + 32 + lane < cnt ? item_idx(item, n + 32 + lane) : 0;
+          creg = n + lane < cnt ? key_shape_code(g, jcur) : 0;
+          partial = __ballot_sync(0xffffffffu, creg != 0);
+        }
         bool w_ok = mbar_wait(&s_full[b], sfc[b] & 1, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
         if (!w_ok) { ok = false; break; }
@@ -688,27 +705,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tc_fence_before();
         mbar_arrive(dp_free);
-        // pad keys of a partial key block: P = 0
-        const int j = item_idx(item, n);
-        int vt, vh, vw;
-        if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
-        else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
-        uint32_t vm[BS / 32];
+        // pad keys of a partial key block: S = -inf, so P = 0
+        if ((partial >> (n & 31)) & 1u) {
+          const int code = __shfl_sync(0xffffffffu, creg, n & 31);
+          const uint32_t* mtab = reinterpret_cast<const uint32_t*>(smem + L::kMaskOff);
+          uint32_t word = mtab[code * (BS / 32) + (KC == 32 ? cg : 0)];
+          if (KC < 32) word >>= cg * KC;
 #pragma unroll
-        for (int w2 = 0; w2 < BS / 32; ++w2) vm[w2] = 0xFFFFFFFFu;
-        if (vt < g.bt || vh < g.bh || vw < g.bw) block_valid_mask<BS>(g, vt, vh, vw, vm);
+          for (int c = 0; c < KC; ++c)
+            if (!((word >> c) & 1u)) sr[c] = __float_as_uint(-INFINITY);
+        }
 #pragma unroll
         for (int e2 = 0; e2 < KC / 2; ++e2) {
-          const int k0 = cg * KC + 2 * e2;
-          float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -l2));
-          float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -l2));
-          if (!((vm[k0 >> 5] >> (k0 & 31)) & 1u)) p0 = 0.f;
-          if (!((vm[(k0 + 1) >> 5] >> ((k0 + 1) & 31)) & 1u)) p1 = 0.f;
+          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -l2));
+          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -l2));
           pk[e2] = pack_bf16x2(p0 * (__uint_as_float(dpr[2 * e2]) - dl),
                                p1 * (__uint_as_float(dpr[2 * e2 + 1]) - dl));
         }
-        // dS goes to columns [KC/2 * cg, ..): other groups may still be reading them
-        named_bar_sync(1, kBwdElem);
+        // dS goes to columns [KC/2 * cg, ..) of this row quarter's lanes, which another group
+        // of the quarter may still be reading: a barrier of the quarter's 128 threads
+        named_bar_sync(1 + (warp & 3), kBwdElem / 4);
         if constexpr (KC == 32) tmem_st16(t_s + cg * (KC / 2), pk);
         else tmem_st8(t_s + cg * (KC / 2), pk);
         tmem_wait_st();

@@ -147,16 +147,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   // Pad-key masks of the partial key-block shapes, indexed by shape code
   // (t class * 2 + h partial) * 2 + w partial, t class 0 full / 1 last cache t-block /
   // 2 last current t-block; bit k of word k / 32 = slot k holds a token.
-  if (tid < 12) {
-    const int tcls = tid >> 2, hp = (tid >> 1) & 1, wp = tid & 1;
-    const int rt = tcls == 1 ? g.Tc % g.bt : g.T % g.bt, rh = g.GH % g.bh, rw = g.GW % g.bw;
-    const int vt = tcls == 0 ? g.bt : rt, vh = hp ? rh : g.bh, vw = wp ? rw : g.bw;
-    uint32_t mw[BS / 32];
-    block_valid_mask<BS>(g, vt, vh, vw, mw);
-    uint32_t* mtab = reinterpret_cast<uint32_t*>(smem + L::kMaskOff);
-#pragma unroll
-    for (int w2 = 0; w2 < BS / 32; ++w2) mtab[tid * (BS / 32) + w2] = mw[w2];
-  }
+  if (tid < 12) fill_shape_mask<BS>(g, tid, reinterpret_cast<uint32_t*>(smem + L::kMaskOff));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -353,14 +344,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if ((n & 31) == 0) {
           const int jcur = jnext;
           jnext = n + 32 + lane < cnt ? load_idx(p, item, n + 32 + lane) : 0;
-          creg = 0;
-          if (n + lane < cnt) {
-            int vt, vh, vw;
-            if (jcur < g.NBc) block_extent(g, g.Tc, jcur, vt, vh, vw);
-            else block_extent(g, g.T, jcur - g.NBc, vt, vh, vw);
-            const int tcls = vt < g.bt ? (jcur < g.NBc ? 1 : 2) : 0;
-            creg = (tcls * 2 + (vh < g.bh ? 1 : 0)) * 2 + (vw < g.bw ? 1 : 0);
-          }
+          creg = n + lane < cnt ? key_shape_code(g, jcur) : 0;
           partial = __ballot_sync(0xffffffffu, creg != 0);
         }
         bool w_ok = mbar_wait(&s_full[b], (gstep >> 1) & 1, abort_flag);

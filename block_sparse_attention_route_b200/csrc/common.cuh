@@ -219,6 +219,28 @@ __device__ __forceinline__ void block_valid_mask(const Geo& g, int vt, int vh, i
     }
 }
 
+// Shape code of key block j: (t class * 2 + h partial) * 2 + w partial, where t class is 0
+// for a full t extent, 1 for the last (partial) t-block of the cache grid, 2 for the last
+// (partial) t-block of the current grid.  Code 0 = full block.
+__device__ __forceinline__ int key_shape_code(const Geo& g, int j) {
+  int vt, vh, vw;
+  if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
+  else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
+  const int tcls = vt < g.bt ? (j < g.NBc ? 1 : 2) : 0;
+  return (tcls * 2 + (vh < g.bh ? 1 : 0)) * 2 + (vw < g.bw ? 1 : 0);
+}
+// Valid-slot mask of shape code `code` (see key_shape_code) into tab[code * BS/32 ..].
+template <int BS>
+__device__ __forceinline__ void fill_shape_mask(const Geo& g, int code, uint32_t* tab) {
+  const int tcls = code >> 2, hp = (code >> 1) & 1, wp = code & 1;
+  const int rt = tcls == 1 ? g.Tc % g.bt : g.T % g.bt, rh = g.GH % g.bh, rw = g.GW % g.bw;
+  const int vt = tcls == 0 ? g.bt : rt, vh = hp ? rh : g.bh, vw = wp ? rw : g.bw;
+  uint32_t mw[BS / 32];
+  block_valid_mask<BS>(g, vt, vh, vw, mw);
+#pragma unroll
+  for (int w2 = 0; w2 < BS / 32; ++w2) tab[code * (BS / 32) + w2] = mw[w2];
+}
+
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
                                             uint64_t* bar) {
