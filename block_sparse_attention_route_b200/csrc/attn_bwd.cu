@@ -24,15 +24,15 @@
 namespace bsa {
 
 struct BwdWs {
-  size_t delta, lse2, rev_off, rev_list, total;
+  size_t ndelta, nlse2, rev_off, rev_list, total;
 };
 inline size_t bwd_align(size_t x) { return (x + 255) & ~size_t(255); }
 BwdWs bwd_ws_layout(const Geo& g, int r) {
   BwdWs w;
   const size_t rows = (size_t)g.B * g.H * g.NBq * g.BS;
-  w.delta = 0;
-  w.lse2 = bwd_align(rows * 4);
-  w.rev_off = w.lse2 + bwd_align(rows * 4);
+  w.ndelta = 0;
+  w.nlse2 = bwd_align(rows * 4);
+  w.rev_off = w.nlse2 + bwd_align(rows * 4);
   w.rev_list = w.rev_off + bwd_align((size_t)g.B * g.H * (g.NBk + 1) * 4);
   w.total = w.rev_list + bwd_align((size_t)g.B * g.H * g.NBq * r * 4);
   return w;
@@ -53,21 +53,22 @@ struct BwdParams {
   const int* cnt;
   const int* rev_off;     // [B*H][NBk+1]
   const int* rev_list;    // [B*H][NBq*r]
-  const float* delta;     // [B*H*NBq*BS]
-  const float* lse2;      // [B*H*NBq*BS], +inf for pad rows
+  const float* ndelta;    // [B*H*NBq*BS] -Delta
+  const float* nlse2;     // [B*H*NBq*BS] -LSE * log2(e), -inf for pad rows
   __nv_bfloat16* out0;    // dkdv: dK, dq: dQ
   __nv_bfloat16* out1;    // dkdv: dV
 };
 
 // ------------------------------------------------------------------------------ prep
-// Delta = rowsum(dO * O) and lse2 = LSE * log2(e) (+inf where LSE = -inf: pad rows or empty
-// selections, so exp2(s - lse2) = 0 there).
+// ndelta = -rowsum(dO * O) and nlse2 = -LSE * log2(e) (-inf where LSE = -inf: pad rows or
+// empty selections, so exp2(s + nlse2) = 0 there).  Stored negated so the elementwise passes
+// form exp2(S * scale * log2e - LSE * log2e) and dP - Delta with single fused f32x2 ops.
 template <int D>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __restrict__ o,
                                                        const __nv_bfloat16* __restrict__ dO,
                                                        const float* __restrict__ lse,
-                                                       float* __restrict__ delta,
-                                                       float* __restrict__ lse2, size_t rows) {
+                                                       float* __restrict__ ndelta,
+                                                       float* __restrict__ nlse2, size_t rows) {
   constexpr int LPR = D / 8;  // lanes per row (16-byte vectors)
   const size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t row = t / LPR;
@@ -87,9 +88,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 #pragma unroll
   for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (row < rows && c == 0) {
-    delta[row] = acc;
+    ndelta[row] = -acc;
     const float l = lse[row];
-    lse2[row] = (l == -INFINITY) ? INFINITY : l * 1.4426950408889634f;
+    nlse2[row] = (l == -INFINITY) ? -INFINITY : -l * 1.4426950408889634f;
   }
 }
 
@@ -154,34 +155,43 @@ __global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams
 // ------------------------------------------------------------------------------ common
 // warps 0-15 elementwise: warp w reads TMEM lanes 32*(w%4).. and owns the 32-column group
 // w/4 of every tile (S, dP: 4 x 32 columns); warp 16 TMA producer; warp 17 MMA issuer and
-// TMEM owner; warps 18-19 idle.  No row reductions are needed in the backward (P comes from
+// TMEM owner.  No row reductions are needed in the backward (P comes from
 // the stored LSE), so the column groups work independently; per step a named barrier of the
 // four warps that share a row quarter's TMEM lanes (w, w+4, w+8, w+12) orders their loads
 // before the bf16 stores that overwrite loaded columns.  The quarters run independently:
 // every arrive-counted mbarrier they signal is consumed before the MMA that lets any thread
 // signal its next phase is issued, so no phase can be overrun.
-constexpr int kBwdThreads = 640;
+constexpr int kBwdThreads = 576;
 constexpr int kBwdProducer = 16, kBwdMma = 17, kBwdElem = 512;
 constexpr int kBwdStages = 2;  // Q_i + dO_i stages of the key-major pass (64 KB each)
 constexpr int kTile = 128;
 
 // ------------------------------------------------------------------------------ dK / dV
 // Work item = current key block (b, h, jc), jc in [0, NBq) (global id NBc + jc).  Steps =
-// the query blocks that selected it.  TMEM: S^T [0,128), dP^T [128,256), dV [256,384),
-// dK [384,512); P^T (bf16) overwrites S^T, dS^T (bf16) overwrites dP^T.
+// the query blocks that selected it, numbered globally (g) over the CTA's items.
+// TMEM: R0 [0,128), R1 [128,256), dV [256,384), dK [384,512).  Step g computes S^T into
+// R[g & 1] and dP^T into R[(g & 1) ^ 1]; the elementwise warps write P^T (bf16) over columns
+// [0,64) and dS^T (bf16) over [64,128) of R[g & 1], so R[(g & 1) ^ 1] is free once dP^T(g)
+// has been loaded -- and S^T(g+1) goes there while P^T(g), dS^T(g) are being formed.
+// MMA order: S^T(g) | dK(g-1), dV(g-1), dP^T(g) | S^T(g+1) | ...; dP^T(g) reuses the region
+// that dK(g-1) and dV(g-1) read, after them in issue order.
+// Q_i and dO_i have rings of their own (2 slots each): Q(g) is last read by dK(g), dO(g) by
+// dV(g), so each slot is released as early as its own last MMA allows.
 template <int BS, int D>
 struct DkdvLayout {
   static constexpr int kKVBytes = BS * D * 2;      // K_j or V_j
   static constexpr int kTileBytes = BS * D * 2;    // Q_i or dO_i (BS query rows)
+  static constexpr int kSlots = 2;
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kKVBytes;
-  static constexpr int kRingOff = 2 * kKVBytes;     // stage s: Q at +0, dO at +kTileBytes
-  static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kVecOff = kRingOff + kBwdStages * kStageBytes;  // lse2 / delta per stage
+  static constexpr int kQOff = 2 * kKVBytes;                       // Q slots
+  static constexpr int kDOOff = kQOff + kSlots * kTileBytes;      // dO slots
+  static constexpr int kVecOff = kDOOff + kSlots * kTileBytes;    // -lse2 / -delta per Q slot
   static constexpr int kVecBytes = 2 * BS * 4;
-  static constexpr int kBarOff = kVecOff + kBwdStages * kVecBytes;
-  // kv_full, kv_empty(unused), st_full[S], st_empty[S], s_full, p_full, acc_full, fin
-  static constexpr int kNumBars = 2 + 2 * kBwdStages + 4;
+  static constexpr int kBarOff = kVecOff + kSlots * kVecBytes;
+  // kv_full, kv_empty, q_full[2], q_empty[2], o_full[2], o_empty[2], s_full, loaded, p_full,
+  // acc_full, fin
+  static constexpr int kNumBars = 2 + 4 * kSlots + 5;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kAlloc = kMiscOff + 16 + 1024;
 };
@@ -192,18 +202,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                         const BwdParams p) {
   using L = DkdvLayout<BS, D>;
+  constexpr int NS = L::kSlots;
   static_assert(BS == 128, "the key-major pass maps one key row to one TMEM lane");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* kv_full = bars;           // K_j, V_j landed (one phase per item)
-  uint64_t* kv_empty = bars + 1;      // K_j, V_j no longer needed (one phase per item)
-  uint64_t* st_full = bars + 2;       // [kBwdStages] Q_i, dO_i, lse2_i, delta_i landed
-  uint64_t* st_empty = st_full + kBwdStages;
-  uint64_t* s_full = st_empty + kBwdStages;  // S^T and dP^T in TMEM
-  uint64_t* p_full = s_full + 1;             // P^T and dS^T in TMEM (128 arrivals)
-  uint64_t* acc_full = p_full + 1;           // dV and dK of the item complete
+  uint64_t* kv_full = bars;           // K_j, V_j landed (one phase per non-empty item)
+  uint64_t* kv_empty = bars + 1;      // K_j, V_j no longer needed
+  uint64_t* q_full = bars + 2;        // [NS] Q_i, lse2_i, delta_i landed
+  uint64_t* q_empty = q_full + NS;    // [NS]
+  uint64_t* o_full = q_empty + NS;    // [NS] dO_i landed
+  uint64_t* o_empty = o_full + NS;    // [NS]
+  uint64_t* s_full = o_empty + NS;    // S^T(g) and dP^T(g) in TMEM
+  uint64_t* loaded = s_full + 1;      // S^T(g), dP^T(g) read into registers (kBwdElem)
+  uint64_t* p_full = loaded + 1;      // P^T(g), dS^T(g) in TMEM (kBwdElem arrivals)
+  uint64_t* acc_full = p_full + 1;    // dV and dK of the item complete
   uint64_t* fin_bar = acc_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -213,8 +227,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (tid == 0) {
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
-    for (int s = 0; s < kBwdStages; ++s) { mbar_init(&st_full[s], 1); mbar_init(&st_empty[s], 1); }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&q_empty[s], 1);
+      mbar_init(&o_full[s], 1);
+      mbar_init(&o_empty[s], 1);
+    }
     mbar_init(s_full, 1);
+    mbar_init(loaded, kBwdElem);
     mbar_init(p_full, kBwdElem);
     mbar_init(acc_full, 1);
     mbar_init(fin_bar, 1);
@@ -239,13 +259,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == kBwdProducer) {
     // ====================================================== TMA producer
     if (lane == 0) {
-      int seq = 0, items = 0;
+      int gq = 0, items = 0;        // steps, non-empty items
+      int q_loads = 0, o_loads = 0;  // copies issued per ring (for the drain)
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         int beg, end;
         item_range(item, beg, end);
+        if (end == beg) continue;
         const int bh = item / g.NBq, jc = item % g.NBq;
-        // K_j, V_j for the item (wait until the previous item's MMAs released them)
+        // K_j, V_j for the item (once the previous item's S^T / dP^T MMAs released them)
         if (items > 0 && !mbar_wait(kv_empty, (items - 1) & 1, abort_flag)) { ok = false; break; }
         mbar_expect_tx(kv_full, 2 * L::kKVBytes);
         const int krow = (bh * g.NBq + jc) * BS;
@@ -256,29 +278,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         ++items;
         const int* list = p.rev_list + (size_t)bh * g.NBq * p.r;
-        for (int e = beg; e < end; ++e) {
+        for (int e = beg; e < end; ++e, ++gq) {
           int i = list[e];
           if (i < 0 || i >= g.NBq) { set_status(DEV_BAD_INDEX); i = 0; }
-          const int stage = seq % kBwdStages, round = seq / kBwdStages;
-          if (round > 0 && !mbar_wait(&st_empty[stage], (round - 1) & 1, abort_flag)) { ok = false; break; }
-          unsigned char* dst = smem + L::kRingOff + stage * L::kStageBytes;
-          unsigned char* vec = smem + L::kVecOff + stage * L::kVecBytes;
-          mbar_expect_tx(&st_full[stage], L::kStageBytes + L::kVecBytes);
+          const int slot = gq % NS, round = gq / NS;
           const int qrow = (bh * g.NBq + i) * BS;
+          if (round > 0 && !mbar_wait(&q_empty[slot], (round - 1) & 1, abort_flag)) { ok = false; break; }
+          unsigned char* vec = smem + L::kVecOff + slot * L::kVecBytes;
+          mbar_expect_tx(&q_full[slot], L::kTileBytes + L::kVecBytes);
 #pragma unroll
-          for (int half = 0; half < D / 64; ++half) {
-            tma_load_2d(dst + half * BS * 128, &tmQ, half * 64, qrow, &st_full[stage]);
-            tma_load_2d(dst + L::kTileBytes + half * BS * 128, &tmdO, half * 64, qrow, &st_full[stage]);
-          }
-          bulk_load(vec, p.lse2 + (size_t)qrow, BS * 4, &st_full[stage]);
-          bulk_load(vec + BS * 4, p.delta + (size_t)qrow, BS * 4, &st_full[stage]);
-          ++seq;
+          for (int half = 0; half < D / 64; ++half)
+            tma_load_2d(smem + L::kQOff + slot * L::kTileBytes + half * BS * 128, &tmQ, half * 64,
+                        qrow, &q_full[slot]);
+          bulk_load(vec, p.nlse2 + (size_t)qrow, BS * 4, &q_full[slot]);
+          bulk_load(vec + BS * 4, p.ndelta + (size_t)qrow, BS * 4, &q_full[slot]);
+          ++q_loads;
+          if (round > 0 && !mbar_wait(&o_empty[slot], (round - 1) & 1, abort_flag)) { ok = false; break; }
+          mbar_expect_tx(&o_full[slot], L::kTileBytes);
+#pragma unroll
+          for (int half = 0; half < D / 64; ++half)
+            tma_load_2d(smem + L::kDOOff + slot * L::kTileBytes + half * BS * 128, &tmdO, half * 64,
+                        qrow, &o_full[slot]);
+          ++o_loads;
         }
       }
       // drain every copy still in flight
-      for (int st = 0; st < kBwdStages; ++st) {
-        const int loads = seq / kBwdStages + (st < seq % kBwdStages ? 1 : 0);
-        if (loads > 0) mbar_wait_drain(&st_full[st], (loads - 1) & 1);
+      for (int s = 0; s < NS; ++s) {
+        const int ql = q_loads / NS + (s < q_loads % NS ? 1 : 0);
+        const int ol = o_loads / NS + (s < o_loads % NS ? 1 : 0);
+        if (ql > 0) mbar_wait_drain(&q_full[s], (ql - 1) & 1);
+        if (ol > 0) mbar_wait_drain(&o_full[s], (ol - 1) & 1);
       }
       if (items > 0) mbar_wait_drain(kv_full, (items - 1) & 1);
     }
@@ -289,56 +318,76 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       constexpr uint32_t idTS = idesc_bf16(kTile, D, 0, 1);    // dV, dK: B MN-major
       const uint64_t dK0 = smem_desc_sw128(smem_u32(smem + L::kKOff), 16, 1024);
       const uint64_t dV0 = smem_desc_sw128(smem_u32(smem + L::kVOff), 16, 1024);
-      const uint64_t dR0 = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
-      const uint64_t dRmn = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
-      const uint32_t t_s = tmem_base, t_dp = tmem_base + 128, t_dv = tmem_base + 256,
-                     t_dk = tmem_base + 384;
-      int seq = 0, items = 0, steps = 0;
+      const uint64_t dQk = smem_desc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+      const uint64_t dOk = smem_desc_sw128(smem_u32(smem + L::kDOOff), 16, 1024);
+      const uint64_t dQmn = smem_desc_sw128(smem_u32(smem + L::kQOff), BS * 128, 1024);
+      const uint64_t dOmn = smem_desc_sw128(smem_u32(smem + L::kDOOff), BS * 128, 1024);
+      const uint32_t t_dv = tmem_base + 256, t_dk = tmem_base + 384;
+      int gs = 0, items = 0;      // steps issued, non-empty items started
+      bool have_prev = false, prev_first = false, prev_last = false;
       bool ok = true;
+      // dK(g-1), dV(g-1) from the bf16 halves of R[(g-1) & 1], then the slot releases
+      auto finish_prev = [&]() -> bool {
+        const int gp = gs - 1, slot = gp % NS;
+        if (!mbar_wait(p_full, gp & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t r = tmem_base + (gp & 1) * 128;
+        const uint64_t mq = dQmn + (uint64_t)((slot * L::kTileBytes) >> 4);
+        const uint64_t mdo = dOmn + (uint64_t)((slot * L::kTileBytes) >> 4);
+        const uint32_t acc0 = prev_first ? 0u : 1u;
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_ts(t_dk, r + 64 + kk * 8, mq + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
+        mma_commit(&q_empty[slot]);
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_ts(t_dv, r + kk * 8, mdo + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
+        mma_commit(&o_empty[slot]);
+        if (prev_last) mma_commit(acc_full);
+        have_prev = false;
+        return true;
+      };
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         int beg, end;
         item_range(item, beg, end);
+        if (end == beg) continue;
         if (!mbar_wait(kv_full, items & 1, abort_flag)) { ok = false; break; }
+        ++items;
         tc_fence_after();
         for (int e = beg; e < end; ++e) {
-          const int stage = seq % kBwdStages;
-          if (!mbar_wait(&st_full[stage], (seq / kBwdStages) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t rq = dR0 + (uint64_t)((stage * L::kStageBytes) >> 4);
-          const uint64_t rdo = rq + (uint64_t)(L::kTileBytes >> 4);
-          // S^T = K Q^T, dP^T = V dO^T  (K-dim = D)
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
-            mma_ss(t_s, dK0 + off, rq + off, idSS, kk > 0 ? 1u : 0u);
+          const int slot = gs % NS;
+          // S^T(g) = K Q^T into R[g & 1] (free once dP^T(g-1) was read out)
+          if (gs > 0) {
+            if (!mbar_wait(loaded, (gs - 1) & 1, abort_flag)) { ok = false; break; }
           }
+          if (!mbar_wait(&q_full[slot], (gs / NS) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t rx = tmem_base + (gs & 1) * 128, ry = tmem_base + ((gs & 1) ^ 1) * 128;
+          const uint64_t rq = dQk + (uint64_t)((slot * L::kTileBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
             const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
-            mma_ss(t_dp, dV0 + off, rdo + off, idSS, kk > 0 ? 1u : 0u);
+            mma_ss(rx, dK0 + off, rq + off, idSS, kk > 0 ? 1u : 0u);
+          }
+          if (have_prev && !finish_prev()) { ok = false; break; }
+          // dP^T(g) = V dO^T into R[(g & 1) ^ 1], after dK(g-1) / dV(g-1) read it
+          if (!mbar_wait(&o_full[slot], (gs / NS) & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t rdo = dOk + (uint64_t)((slot * L::kTileBytes) >> 4);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
+            mma_ss(ry, dV0 + off, rdo + off, idSS, kk > 0 ? 1u : 0u);
           }
           mma_commit(s_full);
-          if (!mbar_wait(p_full, steps & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          ++steps;
-          // dV += P^T dO, dK += dS^T Q  (K-dim = the BS query rows; B operands MN-major)
-          const uint64_t mq = dRmn + (uint64_t)((stage * L::kStageBytes) >> 4);
-          const uint64_t mdo = mq + (uint64_t)(L::kTileBytes >> 4);
-          const uint32_t acc0 = (e > beg) ? 1u : 0u;
-#pragma unroll
-          for (int kk = 0; kk < BS / 16; ++kk)
-            mma_ts(t_dv, t_s + kk * 8, mdo + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
-#pragma unroll
-          for (int kk = 0; kk < BS / 16; ++kk)
-            mma_ts(t_dk, t_dp + kk * 8, mq + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
-          mma_commit(&st_empty[stage]);
-          ++seq;
+          if (e == end - 1) mma_commit(kv_empty);  // K_j, V_j: last S^T / dP^T issued
+          have_prev = true;
+          prev_first = e == beg;
+          prev_last = e == end - 1;
+          ++gs;
         }
-        if (!ok) break;
-        mma_commit(kv_empty);
-        if (end > beg) mma_commit(acc_full);
-        ++items;
       }
+      if (ok && have_prev) finish_prev();
       mma_commit(fin_bar);
       mbar_wait_drain(fin_bar, 0);
     }
@@ -347,9 +396,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int row = 32 * (warp % 4) + lane;  // key slot within the block
     const int cg = warp / 4;                 // 32-column group
     const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
-    const uint32_t t_s = tmem_base + t_lane, t_dp = t_s + 128, t_dv = t_s + 256, t_dk = t_s + 384;
+    const uint32_t t_dv = tmem_base + t_lane + 256, t_dk = tmem_base + t_lane + 384;
     const float sl2 = g.scale * 1.4426950408889634f;
-    int seq = 0, steps = 0, items = 0;
+    int gs = 0, items = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       int beg, end;
@@ -359,45 +408,55 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       block_extent(g, g.T, jc, vt, vh, vw);
       const int lt = row / (g.bh * g.bw), lh = (row / g.bw) % g.bh, lw = row % g.bw;
       const bool kvalid = lt < vt && lh < vh && lw < vw;
-      for (int e = beg; e < end; ++e) {
-        const int stage = seq % kBwdStages;
-        bool w_ok = mbar_wait(s_full, steps & 1, abort_flag);
+      for (int e = beg; e < end; ++e, ++gs) {
+        bool w_ok = mbar_wait(s_full, gs & 1, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
         if (!w_ok) { ok = false; break; }
         tc_fence_after();
-        const float* vec = reinterpret_cast<const float*>(smem + L::kVecOff + stage * L::kVecBytes);
-        const float* lse2 = vec;
-        const float* dlt = vec + BS;
+        const uint32_t rx = tmem_base + t_lane + (gs & 1) * 128;
+        const uint32_t ry = tmem_base + t_lane + ((gs & 1) ^ 1) * 128;
+        const float* vec = reinterpret_cast<const float*>(smem + L::kVecOff + (gs % NS) * L::kVecBytes);
+        const float4* nl4 = reinterpret_cast<const float4*>(vec + cg * 32);       // -lse2[q]
+        const float4* nd4 = reinterpret_cast<const float4*>(vec + BS + cg * 32);  // -delta[q]
         // this group's 32 query columns: P^T = exp2(S^T*sl2 - lse2[q]),
-        // dS^T = P^T * (dP^T - delta[q]); bf16 results go to columns [16cg, 16cg+16), which
-        // another group may still be reading until the barrier.
-        {
-          uint32_t sr[32], dr[32], pk[16], dk[16];
-          tmem_ld32_wait(t_s + cg * 32, sr);
-          tmem_ld32_wait(t_dp + cg * 32, dr);
+        // dS^T = P^T * (dP^T - delta[q]), two columns per f32x2 instruction
+        uint32_t sr[32], dr[32], pk[16], dk[16];
+        tmem_ld32_wait(rx + cg * 32, sr);
+        tmem_ld32_wait(ry + cg * 32, dr);
+        tc_fence_before();
+        mbar_arrive(loaded);  // R[(g & 1) ^ 1] may now take S^T(g+1)
+        if (!kvalid) {        // pad key slot: S^T = -inf, so P^T = dS^T = 0
 #pragma unroll
-          for (int e2 = 0; e2 < 16; ++e2) {
-            const int q0 = cg * 32 + 2 * e2;
-            const float2 ld = *reinterpret_cast<const float2*>(lse2 + q0);
-            const float2 dd = *reinterpret_cast<const float2*>(dlt + q0);
-            float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -ld.x));
-            float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -ld.y));
-            if (!kvalid) { p0 = 0.f; p1 = 0.f; }
-            const float s0 = p0 * (__uint_as_float(dr[2 * e2]) - dd.x);
-            const float s1 = p1 * (__uint_as_float(dr[2 * e2 + 1]) - dd.y);
+          for (int c = 0; c < 32; ++c) sr[c] = __float_as_uint(-INFINITY);
+        }
+        const uint64_t sl2x2 = f2pack(sl2, sl2);
+#pragma unroll
+        for (int e4 = 0; e4 < 8; ++e4) {
+          const float4 nl = nl4[e4], nd = nd4[e4];
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int e2 = 2 * e4 + h;
+            const uint64_t x = fma2(f2pack(__uint_as_float(sr[2 * e2]), __uint_as_float(sr[2 * e2 + 1])),
+                                    sl2x2, h ? f2pack(nl.z, nl.w) : f2pack(nl.x, nl.y));
+            float x0, x1;
+            f2unpack(x, x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            const uint64_t dd = add2(f2pack(__uint_as_float(dr[2 * e2]), __uint_as_float(dr[2 * e2 + 1])),
+                                     h ? f2pack(nd.z, nd.w) : f2pack(nd.x, nd.y));
+            float s0, s1;
+            f2unpack(mul2(f2pack(p0, p1), dd), s0, s1);
             pk[e2] = pack_bf16x2(p0, p1);
             dk[e2] = pack_bf16x2(s0, s1);
           }
-          // the bf16 columns overlap other groups' S^T / dP^T columns of the same lanes
-          named_bar_sync(1 + (warp & 3), kBwdElem / 4);
-          tmem_st16(t_s + cg * 16, pk);
-          tmem_st16(t_dp + cg * 16, dk);
         }
+        // P^T -> columns [16cg, 16cg+16), dS^T -> [64+16cg, ..) of R[g & 1]: other groups of
+        // this row quarter may still be reading those columns until the barrier
+        named_bar_sync(1 + (warp & 3), kBwdElem / 4);
+        tmem_st16(rx + cg * 16, pk);
+        tmem_st16(rx + 64 + cg * 16, dk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full);
-        ++steps;
-        ++seq;
       }
       if (!ok) break;
       // epilogue: dV, dK rows of this key block (zeros for pad keys / no selections)
@@ -408,6 +467,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         bool w_ok = mbar_wait(acc_full, items & 1, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
         if (!w_ok) { ok = false; break; }
+        ++items;
         tc_fence_after();
         constexpr int DC = D / 4;  // dV / dK columns of this group
         uint32_t a[DC], bk[DC];
@@ -441,7 +501,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           reinterpret_cast<uint4*>(dk_row + cg * (D / 4))[c] = z;
         }
       }
-      if (end > beg) ++items;
     }
   }
   tc_fence_before();
@@ -672,8 +731,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         continue;
       }
-      const float l2 = row < BS ? p.lse2[qrow] : INFINITY;   // +inf: pad row -> P = 0
-      const float dl = row < BS ? p.delta[qrow] : 0.f;
+      const float nl2 = row < BS ? p.nlse2[qrow] : -INFINITY;  // -inf: pad row -> P = 0
+      const float nd = row < BS ? p.ndelta[qrow] : 0.f;
+      const uint64_t nl2x2 = f2pack(nl2, nl2), ndx2 = f2pack(nd, nd), sl2x2 = f2pack(sl2, sl2);
       // key-block indices 32 steps at a time, the next chunk's load in flight; per chunk a
       // ballot of the partial blocks and each lane's shape code (as in the forward)
       int jnext = lane < cnt ? item_idx(item, lane) : 0;
@@ -716,11 +776,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!((word >> c) & 1u)) sr[c] = __float_as_uint(-INFINITY);
         }
 #pragma unroll
-        for (int e2 = 0; e2 < KC / 2; ++e2) {
-          const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2]), sl2, -l2));
-          const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * e2 + 1]), sl2, -l2));
-          pk[e2] = pack_bf16x2(p0 * (__uint_as_float(dpr[2 * e2]) - dl),
-                               p1 * (__uint_as_float(dpr[2 * e2 + 1]) - dl));
+        for (int e2 = 0; e2 < KC / 2; ++e2) {  // dS = P (dP - delta), two keys per f32x2 op
+          float x0, x1;
+          f2unpack(fma2(f2pack(__uint_as_float(sr[2 * e2]), __uint_as_float(sr[2 * e2 + 1])), sl2x2, nl2x2),
+                   x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          const uint64_t dd = add2(f2pack(__uint_as_float(dpr[2 * e2]), __uint_as_float(dpr[2 * e2 + 1])), ndx2);
+          float s0, s1;
+          f2unpack(mul2(f2pack(p0, p1), dd), s0, s1);
+          pk[e2] = pack_bf16x2(s0, s1);
         }
         // dS goes to columns [KC/2 * cg, ..) of this row quarter's lanes, which another group
         // of the quarter may still be reading: a barrier of the quarter's 128 threads
@@ -747,7 +811,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint32_t* v32 = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
           for (int e2 = 0; e2 < DC / 2; ++e2)
-            v32[e2] = (l2 == INFINITY) ? 0u
+            v32[e2] = (nl2 == -INFINITY) ? 0u
                                        : pack_bf16x2(__uint_as_float(a[2 * e2]) * g.scale,
                                                      __uint_as_float(a[2 * e2 + 1]) * g.scale);
 #pragma unroll
@@ -767,8 +831,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, const CUtensorMap* maps,
                      int n_sm, cudaStream_t s) {
   if (g.BS != 128) return BSA_ERR_UNSUPPORTED;  // the key-major pass needs 128-token blocks
-  float* delta = reinterpret_cast<float*>(P.ws + w.delta);
-  float* lse2 = reinterpret_cast<float*>(P.ws + w.lse2);
+  float* ndelta = reinterpret_cast<float*>(P.ws + w.ndelta);
+  float* nlse2 = reinterpret_cast<float*>(P.ws + w.nlse2);
   int* rev_off = reinterpret_cast<int*>(P.ws + w.rev_off);
   int* rev_list = reinterpret_cast<int*>(P.ws + w.rev_list);
   const size_t rows = (size_t)g.B * g.H * g.NBq * g.BS;
@@ -778,11 +842,11 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
     if (g.D == 128)
       bwd_prep_kernel<128><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(P.o),
                                                   static_cast<const __nv_bfloat16*>(P.dO), P.lse,
-                                                  delta, lse2, rows);
+                                                  ndelta, nlse2, rows);
     else
       bwd_prep_kernel<64><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(P.o),
                                                  static_cast<const __nv_bfloat16*>(P.dO), P.lse,
-                                                 delta, lse2, rows);
+                                                 ndelta, nlse2, rows);
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   BwdParams bp;
@@ -793,8 +857,8 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
   bp.cnt = P.cnt;
   bp.rev_off = rev_off;
   bp.rev_list = rev_list;
-  bp.delta = delta;
-  bp.lse2 = lse2;
+  bp.ndelta = ndelta;
+  bp.nlse2 = nlse2;
   {
     const size_t smem = (size_t)(g.NBk + kRevThreads) * 4;
     if (cudaFuncSetAttribute(bwd_revidx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -10,7 +10,7 @@
 // the K/V tiles of idx[b,h,i,0:cnt].  Persistent CTAs (one per SM), items in head-major
 // order so the CTAs running at once share one head's K/V in L2.
 //
-// Warp roles (576 threads, 112 registers each):
+// Warp roles (576 threads; 18 warps put 5 on two SM sub-partitions, so at most 96 registers):
 //   warps 0-15  softmax + epilogue: warp w reads TMEM lanes 32*(w%4).. (query rows) and owns
 //               the key-column group w/4 (BS/4 keys) of every S tile and the O-column group
 //               w/4 (D/4 columns) of the output
