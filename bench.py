@@ -12,7 +12,9 @@ value    = effective TFLOP/s of the step on selected-block tile FLOPs (4*BS^2*D 
            all ranks / max-over-ranks step time.
 e2e      = the same metric through the public pipeline API with host (pinned) raster
            inputs copied in and the output O copied back inside the timed region.
-roofline = the forward attention kernel against the measured dense bf16 tensor peak.
+roofline = the attention kernel with the longest launches (timed live with CUDA events on its
+           stream through the library's kernel timing) against the measured sustained
+           dense bf16 tensor peak.
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload (the path
 has no exchange step: routing and attention are independent per (batch, head)), so
@@ -37,6 +39,23 @@ from synth import WORKLOADS, make_raster_inputs  # noqa: E402
 
 def tile_flops(bs: int, d: int, n_pairs: int) -> float:
     return 4.0 * bs * bs * d * n_pairs
+
+
+KERNEL_NAMES = {"fwd": "bsa_fwd_kernel", "bwd_dkdv": "bsa_bwd_dkdv_kernel",
+                "bwd_dq": "bsa_bwd_dq_kernel"}
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per unit of work, from one ncu
+# capture of the kernel as it now stands on the 480p workload (profiles/ names the file and
+# the command); a unit is a selected block pair (fwd, dq) or a pair with a current key block
+# (dkdv).  Traffic grows with the pairs a launch processes, so a full launch is scaled from it.
+# None = not captured for the current kernel.
+DRAM_BYTES_PER_PAIR = {"fwd": None, "bwd_dkdv": None, "bwd_dq": None}
+
+
+def traffic_per_launch(kernel, workload, n_pairs, n_pairs_cur):
+    b = DRAM_BYTES_PER_PAIR.get(kernel)
+    if b is None:
+        return None
+    return b * (n_pairs_cur if kernel == "bwd_dkdv" else n_pairs)
 
 
 def load_peaks():
@@ -246,6 +265,9 @@ def main():
         raise SystemExit(f"device status {st} after warm-up")
 
     n_pairs = int(pipe.cnt.sum().item())
+    r_idx = torch.arange(w.top_r, device=dev).view(1, 1, 1, -1)
+    sel = r_idx < pipe.cnt.unsqueeze(-1)
+    n_pairs_cur = int(((pipe.idx >= g.nbc) & sel).sum().item())  # pairs with a current key block
     fl_fwd = tile_flops(g.bs, g.head_dim, n_pairs)
     fl_step = fl_fwd * (3.5 if with_bwd else 1.0)
 
@@ -254,12 +276,15 @@ def main():
     all_marks = []
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    bsa.bsa_kernel_timing(True)  # event pairs around each attention kernel, on its stream
     with ClockSampler(dev.index or 0) as clk:
         t0.record(stream)
         for _ in range(args.steps):
             all_marks.append(step(True))
         t1.record(stream)
         torch.cuda.synchronize()
+    ktimes = bsa.bsa_kernel_times()
+    bsa.bsa_kernel_timing(False)
     barrier()
     ms = t0.elapsed_time(t1) / args.steps
     names = ["prologue", "route", "fwd"] + (["bwd"] if with_bwd else [])
@@ -310,9 +335,22 @@ def main():
     d2h = o_host.numel() * 2
 
     peaks = load_peaks()
-    fwd_ms = parts["fwd"]
-    achieved = fl_fwd / (fwd_ms * 1e-3) / 1e12
     peak = peaks["bf16_tflops_sustained"]
+    # algorithmic tensor FLOPs per launch of each attention kernel (128x128xD GEMM tiles):
+    # forward S and PV per selected pair; dK/dV pass S^T, dP^T, dV, dK per pair with a
+    # current key block; dQ pass S, dP, dQ per selected pair
+    kflops = {"fwd": tile_flops(g.bs, g.head_dim, n_pairs),
+              "bwd_dkdv": 2 * tile_flops(g.bs, g.head_dim, n_pairs_cur),
+              "bwd_dq": 1.5 * tile_flops(g.bs, g.head_dim, n_pairs)}
+    kernels = {}
+    for kname, (nl, tot_ms) in ktimes.items():
+        if nl == 0:
+            continue
+        avg = tot_ms / nl
+        kernels[kname] = {"launches": nl, "ms_per_launch": avg,
+                          "tflops": kflops[kname] / (avg * 1e-3) / 1e12}
+    dom = max(kernels, key=lambda k_: kernels[k_]["ms_per_launch"])
+    achieved = kernels[dom]["tflops"]
     value = world * fl_step / (ms_max * 1e-3) / 1e12
     line = {
         "metric": "BSA fwd(+bwd) effective TFLOP/s at 720p tokens",
@@ -324,11 +362,12 @@ def main():
                    "top_r": w.top_r, "selected_pairs": n_pairs, "with_bwd": with_bwd,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (126 MB)"},
         "ms_per_call": parts,
-        "tflops_fwd": achieved,
-        "roofline": {"bound": "tensor", "kernel": "bsa_fwd_kernel", "achieved": achieved,
+        "kernels": kernels,
+        "roofline": {"bound": "tensor", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                     "peak_source": f"{peaks['source']} bf16 dense, sustained",
-                     "traffic": None},
+                     "peak_source": f"{peaks['source']} bf16 dense, sustained (of measured)"
+                                    if peaks["source"] == "measured" else "fallback",
+                     "traffic": traffic_per_launch(dom, args.workload, n_pairs, n_pairs_cur)},
         "e2e": {"value": world * fl_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": args.steps * (3 + (4 if with_bwd else 0)),

@@ -116,6 +116,8 @@ def lib() -> ctypes.CDLL:
             "bsa_device_status": (I32, [P]),
             "bsa_selftest_bounded_wait": (I32, [I32, P]),
             "bsa_route_noalloc": (I32, [G, I32, P, P, P, P, P, P]),
+            "bsa_kernel_timing": (I32, [I32]),
+            "bsa_kernel_times": (I32, [P, P]),
             "bsa_error_string": (ctypes.c_char_p, [I32]),
             "bsa_last_error_detail": (ctypes.c_char_p, []),
         }
@@ -208,6 +210,23 @@ def bsa_attn_bwd(g: Geometry, top_r: int, q_blk, k_blk, v_blk, k_cache_blk, v_ca
 
 def bsa_selftest_bounded_wait(limit_us: int, stream=None):
     _check(lib().bsa_selftest_bounded_wait(limit_us, _stream(stream)), "bsa_selftest_bounded_wait")
+
+
+TIMED_KERNELS = ("fwd", "bwd_dkdv", "bwd_dq")  # BSA_TIMED_* order
+
+
+def bsa_kernel_timing(on: bool):
+    """Start (True) or stop (False) CUDA-event timing of the attention kernels; either call
+    discards what was recorded."""
+    _check(lib().bsa_kernel_timing(1 if on else 0), "bsa_kernel_timing")
+
+
+def bsa_kernel_times() -> dict:
+    """Per timed kernel: (launches, total ms) since the last call; waits for the events."""
+    n = (ctypes.c_int32 * len(TIMED_KERNELS))()
+    ms = (ctypes.c_float * len(TIMED_KERNELS))()
+    _check(lib().bsa_kernel_times(ctypes.addressof(n), ctypes.addressof(ms)), "bsa_kernel_times")
+    return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(TIMED_KERNELS)}
 
 
 def bsa_device_status(stream=None) -> int:

@@ -156,9 +156,9 @@ __global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams
 // warps 0-15 elementwise: warp w reads TMEM lanes 32*(w%4).. and owns the 32-column group
 // w/4 of every tile (S, dP: 4 x 32 columns); warp 16 TMA producer; warp 17 MMA issuer and
 // TMEM owner.  No row reductions are needed in the backward (P comes from
-// the stored LSE), so the column groups work independently; per step a named barrier of the
-// four warps that share a row quarter's TMEM lanes (w, w+4, w+8, w+12) orders their loads
-// before the bf16 stores that overwrite loaded columns.  The quarters run independently:
+// the stored LSE), so the column groups work independently: each writes its bf16 results
+// back over TMEM columns it read itself, and the MMAs read the slices from where they land.
+// Groups and quarters run independently:
 // every arrive-counted mbarrier they signal is consumed before the MMA that lets any thread
 // signal its next phase is issued, so no phase can be overrun.
 constexpr int kBwdThreads = 576;
@@ -170,9 +170,11 @@ constexpr int kTile = 128;
 // Work item = current key block (b, h, jc), jc in [0, NBq) (global id NBc + jc).  Steps =
 // the query blocks that selected it, numbered globally (g) over the CTA's items.
 // TMEM: R0 [0,128), R1 [128,256), dV [256,384), dK [384,512).  Step g computes S^T into
-// R[g & 1] and dP^T into R[(g & 1) ^ 1]; the elementwise warps write P^T (bf16) over columns
-// [0,64) and dS^T (bf16) over [64,128) of R[g & 1], so R[(g & 1) ^ 1] is free once dP^T(g)
-// has been loaded -- and S^T(g+1) goes there while P^T(g), dS^T(g) are being formed.
+// R[g & 1] and dP^T into R[(g & 1) ^ 1]; the elementwise warps write P^T and dS^T (bf16) back
+// over S^T in R[g & 1] -- each 32-column group over its own columns, as [P^T | dS^T] per 16
+// queries (so the K16 slice kk of P^T sits at column 16kk, of dS^T at 16kk + 8) -- and
+// R[(g & 1) ^ 1] is free once dP^T(g) has been loaded: S^T(g+1) goes there while P^T(g),
+// dS^T(g) are being formed.
 // MMA order: S^T(g) | dK(g-1), dV(g-1), dP^T(g) | S^T(g+1) | ...; dP^T(g) reuses the region
 // that dK(g-1) and dV(g-1) read, after them in issue order.
 // Q_i and dO_i have rings of their own (2 slots each): Q(g) is last read by dK(g), dO(g) by
@@ -326,7 +328,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int gs = 0, items = 0;      // steps issued, non-empty items started
       bool have_prev = false, prev_first = false, prev_last = false;
       bool ok = true;
-      // dK(g-1), dV(g-1) from the bf16 halves of R[(g-1) & 1], then the slot releases
+      // dK(g-1), dV(g-1) from the interleaved bf16 slices in R[(g-1) & 1], then the slot releases
       auto finish_prev = [&]() -> bool {
         const int gp = gs - 1, slot = gp % NS;
         if (!mbar_wait(p_full, gp & 1, abort_flag)) return false;
@@ -336,12 +338,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint64_t mdo = dOmn + (uint64_t)((slot * L::kTileBytes) >> 4);
         const uint32_t acc0 = prev_first ? 0u : 1u;
 #pragma unroll
-        for (int kk = 0; kk < BS / 16; ++kk)
-          mma_ts(t_dk, r + 64 + kk * 8, mq + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
+        for (int kk = 0; kk < BS / 16; ++kk)  // dS^T of queries [16kk, 16kk+16) at columns 16kk + 8
+          mma_ts(t_dk, r + kk * 16 + 8, mq + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
         mma_commit(&q_empty[slot]);
 #pragma unroll
-        for (int kk = 0; kk < BS / 16; ++kk)
-          mma_ts(t_dv, r + kk * 8, mdo + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
+        for (int kk = 0; kk < BS / 16; ++kk)  // P^T of queries [16kk, 16kk+16) at columns 16kk
+          mma_ts(t_dv, r + kk * 16, mdo + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
         mma_commit(&o_empty[slot]);
         if (prev_last) mma_commit(acc_full);
         have_prev = false;
@@ -419,41 +421,47 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float4* nl4 = reinterpret_cast<const float4*>(vec + cg * 32);       // -lse2[q]
         const float4* nd4 = reinterpret_cast<const float4*>(vec + BS + cg * 32);  // -delta[q]
         // this group's 32 query columns: P^T = exp2(S^T*sl2 - lse2[q]),
-        // dS^T = P^T * (dP^T - delta[q]), two columns per f32x2 instruction
-        uint32_t sr[32], dr[32], pk[16], dk[16];
-        tmem_ld32_wait(rx + cg * 32, sr);
+        // dS^T = P^T * (dP^T - delta[q]), two columns per f32x2 instruction.  dP^T is read
+        // whole (its region takes S^T(g+1) next); S^T 16 columns at a time, and each round's
+        // results go back over the S^T columns it just read -- this group's own -- as
+        // [P^T 8 cols | dS^T 8 cols] per 16 queries, so no other group is involved.
+        uint32_t dr[32], sr[16];
         tmem_ld32_wait(ry + cg * 32, dr);
+        tmem_ld16_wait(rx + cg * 32, sr);
         tc_fence_before();
         mbar_arrive(loaded);  // R[(g & 1) ^ 1] may now take S^T(g+1)
-        if (!kvalid) {        // pad key slot: S^T = -inf, so P^T = dS^T = 0
-#pragma unroll
-          for (int c = 0; c < 32; ++c) sr[c] = __float_as_uint(-INFINITY);
-        }
         const uint64_t sl2x2 = f2pack(sl2, sl2);
 #pragma unroll
-        for (int e4 = 0; e4 < 8; ++e4) {
-          const float4 nl = nl4[e4], nd = nd4[e4];
+        for (int round = 0; round < 2; ++round) {
+          if (round == 1) tmem_ld16_wait(rx + cg * 32 + 16, sr);
+          if (!kvalid) {  // pad key slot: S^T = -inf, so P^T = dS^T = 0
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int e2 = 2 * e4 + h;
-            const uint64_t x = fma2(f2pack(__uint_as_float(sr[2 * e2]), __uint_as_float(sr[2 * e2 + 1])),
-                                    sl2x2, h ? f2pack(nl.z, nl.w) : f2pack(nl.x, nl.y));
-            float x0, x1;
-            f2unpack(x, x0, x1);
-            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            const uint64_t dd = add2(f2pack(__uint_as_float(dr[2 * e2]), __uint_as_float(dr[2 * e2 + 1])),
-                                     h ? f2pack(nd.z, nd.w) : f2pack(nd.x, nd.y));
-            float s0, s1;
-            f2unpack(mul2(f2pack(p0, p1), dd), s0, s1);
-            pk[e2] = pack_bf16x2(p0, p1);
-            dk[e2] = pack_bf16x2(s0, s1);
+            for (int c = 0; c < 16; ++c) sr[c] = __float_as_uint(-INFINITY);
           }
+          uint32_t pk[8], dk[8];
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 nl = nl4[round * 4 + e4], nd = nd4[round * 4 + e4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int j = 2 * e4 + h;           // column pair within the round
+              const int e2 = round * 8 + j;       // column pair within the 32
+              const uint64_t x = fma2(f2pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])),
+                                      sl2x2, h ? f2pack(nl.z, nl.w) : f2pack(nl.x, nl.y));
+              float x0, x1;
+              f2unpack(x, x0, x1);
+              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+              const uint64_t dd = add2(f2pack(__uint_as_float(dr[2 * e2]), __uint_as_float(dr[2 * e2 + 1])),
+                                       h ? f2pack(nd.z, nd.w) : f2pack(nd.x, nd.y));
+              float s0, s1;
+              f2unpack(mul2(f2pack(p0, p1), dd), s0, s1);
+              pk[j] = pack_bf16x2(p0, p1);
+              dk[j] = pack_bf16x2(s0, s1);
+            }
+          }
+          tmem_st8(rx + cg * 32 + round * 16, pk);
+          tmem_st8(rx + cg * 32 + round * 16 + 8, dk);
         }
-        // P^T -> columns [16cg, 16cg+16), dS^T -> [64+16cg, ..) of R[g & 1]: other groups of
-        // this row quarter may still be reading those columns until the barrier
-        named_bar_sync(1 + (warp & 3), kBwdElem / 4);
-        tmem_st16(rx + cg * 16, pk);
-        tmem_st16(rx + 64 + cg * 16, dk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(p_full);
@@ -469,29 +477,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (!w_ok) { ok = false; break; }
         ++items;
         tc_fence_after();
-        constexpr int DC = D / 4;  // dV / dK columns of this group
-        uint32_t a[DC], bk[DC];
-        if constexpr (DC == 32) {
-          tmem_ld32_wait(t_dv + cg * DC, a);
-          tmem_ld32_wait(t_dk + cg * DC, bk);
-        } else {
-          tmem_ld16_wait(t_dv + cg * DC, a);
-          tmem_ld16_wait(t_dk + cg * DC, bk);
-        }
-        uint4 va[DC / 8], vb[DC / 8];
-        uint32_t* a32 = reinterpret_cast<uint32_t*>(va);
-        uint32_t* b32 = reinterpret_cast<uint32_t*>(vb);
+        constexpr int DC = D / 4;  // dV / dK columns of this group, 16 at a time
 #pragma unroll
-        for (int e2 = 0; e2 < DC / 2; ++e2) {
-          a32[e2] = kvalid ? pack_bf16x2(__uint_as_float(a[2 * e2]), __uint_as_float(a[2 * e2 + 1])) : 0u;
-          b32[e2] = kvalid ? pack_bf16x2(__uint_as_float(bk[2 * e2]) * g.scale,
-                                         __uint_as_float(bk[2 * e2 + 1]) * g.scale)
-                           : 0u;
-        }
+        for (int c0 = 0; c0 < DC; c0 += 16) {
 #pragma unroll
-        for (int e2 = 0; e2 < DC / 8; ++e2) {
-          reinterpret_cast<uint4*>(dv_row + cg * DC)[e2] = va[e2];
-          reinterpret_cast<uint4*>(dk_row + cg * DC)[e2] = vb[e2];
+          for (int which = 0; which < 2; ++which) {  // dV, then dK (scaled)
+            uint32_t a[16];
+            tmem_ld16_wait((which ? t_dk : t_dv) + cg * DC + c0, a);
+            const float sc = which ? g.scale : 1.0f;
+            uint4 va[2];
+            uint32_t* a32 = reinterpret_cast<uint32_t*>(va);
+#pragma unroll
+            for (int e2 = 0; e2 < 8; ++e2)
+              a32[e2] = kvalid ? pack_bf16x2(__uint_as_float(a[2 * e2]) * sc, __uint_as_float(a[2 * e2 + 1]) * sc)
+                               : 0u;
+            __nv_bfloat16* dst = (which ? dk_row : dv_row) + cg * DC + c0;
+            reinterpret_cast<uint4*>(dst)[0] = va[0];
+            reinterpret_cast<uint4*>(dst)[1] = va[1];
+          }
         }
       } else {
         const uint4 z = make_uint4(0, 0, 0, 0);
@@ -512,7 +515,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ------------------------------------------------------------------------------ dQ
 // Work item = query block (b, h, i); steps = its selected key blocks (cached ones included).
 // TMEM: S0 [0,128), S1 [128,256), dP [256,384), dQ [384,512); dS (bf16) overwrites the S
-// buffer it came from.  MMA order per step n: dP(n) once the previous dP was read out,
+// buffer it came from, each 32-key group's 16 columns over the first half of its own S columns.  MMA order per step n: dP(n) once the previous dP was read out,
 // dQ += dS(n-1) K_{n-1}, S(n+1); so the tensor cores run while dS(n) is formed.
 template <int BS, int D>
 struct DqLayout {
@@ -696,9 +699,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int kseq = seq_base + 2 * n;
           const uint64_t kb = dkmn + (uint64_t)(((kseq % S) * L::kKVBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < BS / 16; ++kk)
-            mma_ts(t_dq, tmem_base + b * 128 + kk * 8, kb + (uint64_t)((kk * 2048) >> 4), idQ,
-                   (n > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < BS / 16; ++kk)  // dS of keys [16kk, 16kk+16): group kk/2's columns
+            mma_ts(t_dq, tmem_base + b * 128 + 32 * (kk >> 1) + 8 * (kk & 1),
+                   kb + (uint64_t)((kk * 2048) >> 4), idQ, (n > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&kv_empty[kseq % S]);  // K_n done
           if (n + 2 < cnt) { ok = issue_S(n + 2); if (!ok) break; }
         }
@@ -786,11 +789,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           f2unpack(mul2(f2pack(p0, p1), dd), s0, s1);
           pk[e2] = pack_bf16x2(s0, s1);
         }
-        // dS goes to columns [KC/2 * cg, ..) of this row quarter's lanes, which another group
-        // of the quarter may still be reading: a barrier of the quarter's 128 threads
-        named_bar_sync(1 + (warp & 3), kBwdElem / 4);
-        if constexpr (KC == 32) tmem_st16(t_s + cg * (KC / 2), pk);
-        else tmem_st8(t_s + cg * (KC / 2), pk);
+        // dS (bf16) goes back over this group's own S columns: keys [KC*cg, KC*cg + KC) at
+        // columns [KC*cg, KC*cg + KC/2), so no other group's S is overwritten
+        static_assert(KC == 32, "the dQ pass runs with 128-key blocks");
+        tmem_st16(t_s + cg * KC, pk);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&ds_full[b]);
@@ -877,7 +879,10 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
     const int s1 = DkdvLayout<128, Dv>::kAlloc;                                                   \
     if (cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, s1) != cudaSuccess) \
       return BSA_ERR_CUDA;                                                                        \
+    cudaEvent_t e1;                                                                               \
+    const int w1 = timed_begin(BSA_TIMED_BWD_DKDV, s, &e1);                                       \
     k1<<<grid, kBwdThreads, s1, s>>>(maps[1], maps[2], maps[0], maps[5], a);                      \
+    timed_end(w1, s, e1);                                                                         \
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;                                   \
     BwdParams c = bp;                                                                             \
     c.out0 = static_cast<__nv_bfloat16*>(P.dq);                                                   \
@@ -886,7 +891,10 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
     const int s2 = DqLayout<128, Dv>::kAlloc;                                                     \
     if (cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, s2) != cudaSuccess) \
       return BSA_ERR_CUDA;                                                                        \
+    cudaEvent_t e2;                                                                               \
+    const int w2 = timed_begin(BSA_TIMED_BWD_DQ, s, &e2);                                         \
     k2<<<grid, kBwdThreads, s2, s>>>(maps[0], maps[5], maps[1], maps[2], maps[3], maps[4], c);   \
+    timed_end(w2, s, e2);                                                                         \
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;                                   \
   } while (0)
   if (g.D == 128) BSA_LAUNCH_BWD(128);

@@ -12,6 +12,7 @@
 #include <string>
 
 #include "common.cuh"
+#include "timing.cuh"
 
 #include "prologue.cu"
 #include "route.cu"
@@ -361,7 +362,10 @@ bsa_status_t bsa_attn_fwd(const bsa_geom_t* gi, int32_t top_r, const void* q_blk
   p.cnt = cnt;
   p.o = static_cast<__nv_bfloat16*>(o_blk);
   p.lse = lse;
+  cudaEvent_t t0;
+  const int tw = timed_begin(BSA_TIMED_FWD, reinterpret_cast<cudaStream_t>(stream), &t0);
   cudaError_t e = launch_fwd(maps, p, n_sm, reinterpret_cast<cudaStream_t>(stream));
+  timed_end(tw, reinterpret_cast<cudaStream_t>(stream), t0);
   if (e != cudaSuccess) return cuda_fail(e, "fwd launch");
   return BSA_OK;
 }
@@ -427,6 +431,46 @@ bsa_status_t bsa_selftest_bounded_wait(int32_t limit_us, bsa_stream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "selftest launch");
   return BSA_OK;
+}
+
+bsa_status_t bsa_kernel_timing(int32_t on) {
+  t_detail.clear();
+  KernelTimer& t = kernel_timer();
+  std::lock_guard<std::mutex> lk(t.mu);
+  for (auto& v : t.pending) {  // drop what was recorded before (events go back to the pool)
+    for (auto& pr : v) {
+      cudaEventSynchronize(pr.second);
+      t.pool.push_back(pr.first);
+      t.pool.push_back(pr.second);
+    }
+    v.clear();
+  }
+  t.on.store(on ? 1 : 0);
+  return BSA_OK;
+}
+
+bsa_status_t bsa_kernel_times(int32_t* launches, float* total_ms) {
+  t_detail.clear();
+  if (!launches || !total_ms) return fail(BSA_ERR_INVALID_ARG, "launches and total_ms are required");
+  KernelTimer& t = kernel_timer();
+  std::lock_guard<std::mutex> lk(t.mu);
+  bsa_status_t st = BSA_OK;
+  for (int k = 0; k < kNumTimed; ++k) {
+    launches[k] = 0;
+    total_ms[k] = 0.f;
+    for (auto& pr : t.pending[k]) {
+      float ms = 0.f;
+      cudaError_t e = cudaEventSynchronize(pr.second);
+      if (e == cudaSuccess) e = cudaEventElapsedTime(&ms, pr.first, pr.second);
+      if (e != cudaSuccess && st == BSA_OK) st = cuda_fail(e, "kernel timing event");
+      ++launches[k];
+      total_ms[k] += ms;
+      t.pool.push_back(pr.first);
+      t.pool.push_back(pr.second);
+    }
+    t.pending[k].clear();
+  }
+  return st;
 }
 
 bsa_status_t bsa_device_status(bsa_stream_t stream) {

@@ -162,6 +162,20 @@ BSA_API bsa_status_t bsa_attn_bwd(const bsa_geom_t* g, int32_t top_r, const void
                           void* dq_blk, void* dk_blk, void* dv_blk, void* ws,
                           size_t ws_bytes, bsa_stream_t stream);
 
+/* Per-kernel timing for benchmarks (not part of the method; no page counterpart).
+ * bsa_kernel_timing(1) starts it, (0) stops it; either call discards what was recorded.
+ * While on, bsa_attn_fwd and bsa_attn_bwd record a CUDA event pair on their own stream
+ * around each attention kernel they launch.  bsa_kernel_times(launches, total_ms) waits for
+ * those events and fills BSA_NUM_TIMED entries (index BSA_TIMED_*): launches timed and their
+ * summed milliseconds since the last call; the caller owns both arrays.  The library keeps
+ * and reuses the events (host-side bookkeeping only; no device memory).  Off by default. */
+#define BSA_TIMED_FWD 0
+#define BSA_TIMED_BWD_DKDV 1
+#define BSA_TIMED_BWD_DQ 2
+#define BSA_NUM_TIMED 3
+BSA_API bsa_status_t bsa_kernel_timing(int32_t on);
+BSA_API bsa_status_t bsa_kernel_times(int32_t* launches, float* total_ms);
+
 /* Waits for `stream`, then reads and clears the current device's status word.
  * Returns BSA_OK, BSA_ERR_TIMEOUT or BSA_ERR_BAD_INDEX (or BSA_ERR_CUDA). */
 BSA_API bsa_status_t bsa_device_status(bsa_stream_t stream);

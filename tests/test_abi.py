@@ -88,3 +88,11 @@ def test_bad_arguments_rejected_on_host():
         bsa.bsa_attn_bwd(g, 8, *([16] * 3), None, None, 16, 16, 16, 16, 16, 16, 16, 16, 16,
                          stream=0)
     assert ei.value.code == 6
+
+
+def test_kernel_timing_bookkeeping_without_launches():
+    # host-side only: nothing recorded, so nothing to wait for and all counts are zero
+    bsa.bsa_kernel_timing(True)
+    assert bsa.bsa_kernel_times() == {k: (0, 0.0) for k in bsa.TIMED_KERNELS}
+    bsa.bsa_kernel_timing(False)
+    assert bsa.bsa_kernel_times() == {k: (0, 0.0) for k in bsa.TIMED_KERNELS}

@@ -99,3 +99,16 @@ def test_backward_unsupported_block_size_is_reported():
                          torch.zeros(bsa.bsa_workspace_size(g, 2, bsa.WS_BWD), dtype=torch.uint8,
                                      device="cuda"))
     assert ei.value.code == 2
+
+
+def test_kernel_timing_counts_each_attention_launch():
+    import block_sparse_attention_route_b200 as bsa
+    w = WORKLOADS["small"]
+    bsa.bsa_kernel_timing(True)
+    try:
+        run_fwd_bwd(w)
+        t = bsa.bsa_kernel_times()
+    finally:
+        bsa.bsa_kernel_timing(False)
+    assert {k: n for k, (n, _) in t.items()} == {"fwd": 1, "bwd_dkdv": 1, "bwd_dq": 1}
+    assert all(ms > 0 for _, ms in t.values())
