@@ -44,11 +44,12 @@ def tile_flops(bs: int, d: int, n_pairs: int) -> float:
 KERNEL_NAMES = {"fwd": "bsa_fwd_kernel", "bwd_dkdv": "bsa_bwd_dkdv_kernel",
                 "bwd_dq": "bsa_bwd_dq_kernel"}
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per unit of work, from one ncu
-# capture of the kernel as it now stands on the 480p workload (profiles/ names the file and
-# the command); a unit is a selected block pair (fwd, dq) or a pair with a current key block
-# (dkdv).  Traffic grows with the pairs a launch processes, so a full launch is scaled from it.
-# None = not captured for the current kernel.
-DRAM_BYTES_PER_PAIR = {"fwd": None, "bwd_dkdv": None, "bwd_dq": None}
+# --set full capture of the kernel as it now stands on the 480p workload (365,568 pairs; the
+# attention-kernel summary under profiles/ holds the figures and the command); a unit is a
+# selected block pair (fwd, dq) or a pair with a current key block (dkdv).  Traffic grows with
+# the pairs a launch processes, so a full launch is scaled from it.  None = not captured for
+# the kernel as it now stands.
+DRAM_BYTES_PER_PAIR = {"fwd": 3855, "bwd_dkdv": None, "bwd_dq": None}
 
 
 def traffic_per_launch(kernel, workload, n_pairs, n_pairs_cur):
