@@ -191,9 +191,9 @@ struct DkdvLayout {
   static constexpr int kVecOff = kDOOff + kSlots * kTileBytes;    // -lse2 / -delta per Q slot
   static constexpr int kVecBytes = 2 * BS * 4;
   static constexpr int kBarOff = kVecOff + kSlots * kVecBytes;
-  // kv_full, kv_empty, q_full[2], q_empty[2], o_full[2], o_empty[2], s_full, loaded, p_full,
-  // acc_full, fin
-  static constexpr int kNumBars = 2 + 4 * kSlots + 5;
+  // kv_full, kv_empty, q_full[2], q_empty[2], o_full[2], o_empty[2], s_full, loaded,
+  // p_full[2], acc_full, fin
+  static constexpr int kNumBars = 2 + 4 * kSlots + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kAlloc = kMiscOff + 16 + 1024;
 };
@@ -218,8 +218,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* o_empty = o_full + NS;    // [NS]
   uint64_t* s_full = o_empty + NS;    // S^T(g) and dP^T(g) in TMEM
   uint64_t* loaded = s_full + 1;      // S^T(g), dP^T(g) read into registers (kBwdElem)
-  uint64_t* p_full = loaded + 1;      // P^T(g), dS^T(g) in TMEM (kBwdElem arrivals)
-  uint64_t* acc_full = p_full + 1;    // dV and dK of the item complete
+  uint64_t* p_full = loaded + 1;      // [2] P^T(g), dS^T(g) of queries 16kk.. with kk even
+                                      // ([0]) / odd ([1]) in TMEM (kBwdElem arrivals each)
+  uint64_t* acc_full = p_full + 2;    // dV and dK of the item complete
   uint64_t* fin_bar = acc_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -237,7 +238,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     mbar_init(s_full, 1);
     mbar_init(loaded, kBwdElem);
-    mbar_init(p_full, kBwdElem);
+    mbar_init(&p_full[0], kBwdElem);
+    mbar_init(&p_full[1], kBwdElem);
     mbar_init(acc_full, 1);
     mbar_init(fin_bar, 1);
     *abort_flag = 0;
@@ -328,22 +330,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int gs = 0, items = 0;      // steps issued, non-empty items started
       bool have_prev = false, prev_first = false, prev_last = false;
       bool ok = true;
-      // dK(g-1), dV(g-1) from the interleaved bf16 slices in R[(g-1) & 1], then the slot releases
+      // dK(g-1), dV(g-1) from the interleaved bf16 slices in R[(g-1) & 1], then the slot
+      // releases.  The K16 slices of even kk (each group's first 16 queries) are formed in the
+      // elementwise warps' first round and go as soon as p_full[0] says so; odd kk follow.
       auto finish_prev = [&]() -> bool {
         const int gp = gs - 1, slot = gp % NS;
-        if (!mbar_wait(p_full, gp & 1, abort_flag)) return false;
-        tc_fence_after();
         const uint32_t r = tmem_base + (gp & 1) * 128;
         const uint64_t mq = dQmn + (uint64_t)((slot * L::kTileBytes) >> 4);
         const uint64_t mdo = dOmn + (uint64_t)((slot * L::kTileBytes) >> 4);
-        const uint32_t acc0 = prev_first ? 0u : 1u;
 #pragma unroll
-        for (int kk = 0; kk < BS / 16; ++kk)  // dS^T of queries [16kk, 16kk+16) at columns 16kk + 8
-          mma_ts(t_dk, r + kk * 16 + 8, mq + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
+        for (int half = 0; half < 2; ++half) {
+          if (!mbar_wait(&p_full[half], gp & 1, abort_flag)) return false;
+          tc_fence_after();
+#pragma unroll
+          for (int k2 = 0; k2 < BS / 32; ++k2) {
+            const int kk = 2 * k2 + half;
+            const uint32_t acc = (prev_first && kk == 0) ? 0u : 1u;
+            // dS^T of queries [16kk, 16kk+16) at columns 16kk + 8, P^T at 16kk
+            mma_ts(t_dk, r + kk * 16 + 8, mq + (uint64_t)((kk * 2048) >> 4), idTS, acc);
+            mma_ts(t_dv, r + kk * 16, mdo + (uint64_t)((kk * 2048) >> 4), idTS, acc);
+          }
+        }
         mma_commit(&q_empty[slot]);
-#pragma unroll
-        for (int kk = 0; kk < BS / 16; ++kk)  // P^T of queries [16kk, 16kk+16) at columns 16kk
-          mma_ts(t_dv, r + kk * 16, mdo + (uint64_t)((kk * 2048) >> 4), idTS, (acc0 | kk) ? 1u : 0u);
         mma_commit(&o_empty[slot]);
         if (prev_last) mma_commit(acc_full);
         have_prev = false;
@@ -461,10 +469,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           }
           tmem_st8(rx + cg * 32 + round * 16, pk);
           tmem_st8(rx + cg * 32 + round * 16 + 8, dk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_full[round]);  // this round's K16 slice of every group is in TMEM
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(p_full);
       }
       if (!ok) break;
       // epilogue: dV, dK rows of this key block (zeros for pad keys / no selections)
