@@ -191,9 +191,9 @@ struct DkdvLayout {
   static constexpr int kVecOff = kDOOff + kSlots * kTileBytes;    // -lse2 / -delta per Q slot
   static constexpr int kVecBytes = 2 * BS * 4;
   static constexpr int kBarOff = kVecOff + kSlots * kVecBytes;
-  // kv_full, kv_empty, q_full[2], q_empty[2], o_full[2], o_empty[2], s_full, loaded,
-  // p_full[2], acc_full, fin
-  static constexpr int kNumBars = 2 + 4 * kSlots + 6;
+  // kv_full, kv_empty, q_full[2], q_empty[2], o_full[2], o_empty[2], s_full, dp_full,
+  // p_ready, dp_loaded, ds_ready, acc_full, fin
+  static constexpr int kNumBars = 2 + 4 * kSlots + 7;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kAlloc = kMiscOff + 16 + 1024;
 };
@@ -216,11 +216,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* q_empty = q_full + NS;    // [NS]
   uint64_t* o_full = q_empty + NS;    // [NS] dO_i landed
   uint64_t* o_empty = o_full + NS;    // [NS]
-  uint64_t* s_full = o_empty + NS;    // S^T(g) and dP^T(g) in TMEM
-  uint64_t* loaded = s_full + 1;      // S^T(g), dP^T(g) read into registers (kBwdElem)
-  uint64_t* p_full = loaded + 1;      // [2] P^T(g), dS^T(g) of queries 16kk.. with kk even
-                                      // ([0]) / odd ([1]) in TMEM (kBwdElem arrivals each)
-  uint64_t* acc_full = p_full + 2;    // dV and dK of the item complete
+  uint64_t* s_full = o_empty + NS;    // S^T(g) in TMEM
+  uint64_t* dp_full = s_full + 1;     // dP^T(g) in TMEM
+  uint64_t* p_ready = dp_full + 1;    // P^T(g) (bf16) in TMEM (kBwdElem arrivals)
+  uint64_t* dp_loaded = p_ready + 1;  // dP^T(g) read into registers (kBwdElem arrivals)
+  uint64_t* ds_ready = dp_loaded + 1; // dS^T(g) (bf16) in TMEM (kBwdElem arrivals)
+  uint64_t* acc_full = ds_ready + 1;  // dV and dK of the item complete
   uint64_t* fin_bar = acc_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -237,9 +238,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(&o_empty[s], 1);
     }
     mbar_init(s_full, 1);
-    mbar_init(loaded, kBwdElem);
-    mbar_init(&p_full[0], kBwdElem);
-    mbar_init(&p_full[1], kBwdElem);
+    mbar_init(dp_full, 1);
+    mbar_init(p_ready, kBwdElem);
+    mbar_init(dp_loaded, kBwdElem);
+    mbar_init(ds_ready, kBwdElem);
     mbar_init(acc_full, 1);
     mbar_init(fin_bar, 1);
     *abort_flag = 0;
@@ -327,77 +329,100 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const uint64_t dQmn = smem_desc_sw128(smem_u32(smem + L::kQOff), BS * 128, 1024);
       const uint64_t dOmn = smem_desc_sw128(smem_u32(smem + L::kDOOff), BS * 128, 1024);
       const uint32_t t_dv = tmem_base + 256, t_dk = tmem_base + 384;
-      int gs = 0, items = 0;      // steps issued, non-empty items started
-      bool have_prev = false, prev_first = false, prev_last = false;
+      static_assert(NS == 2, "slot = step & 1");
+      int kv_items = 0;  // K/V loads waited for
       bool ok = true;
-      // dK(g-1), dV(g-1) from the interleaved bf16 slices in R[(g-1) & 1], then the slot
-      // releases.  The K16 slices of even kk (each group's first 16 queries) are formed in the
-      // elementwise warps' first round and go as soon as p_full[0] says so; odd kk follow.
-      auto finish_prev = [&]() -> bool {
-        const int gp = gs - 1, slot = gp % NS;
-        const uint32_t r = tmem_base + (gp & 1) * 128;
-        const uint64_t mq = dQmn + (uint64_t)((slot * L::kTileBytes) >> 4);
-        const uint64_t mdo = dOmn + (uint64_t)((slot * L::kTileBytes) >> 4);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          if (!mbar_wait(&p_full[half], gp & 1, abort_flag)) return false;
-          tc_fence_after();
-#pragma unroll
-          for (int k2 = 0; k2 < BS / 32; ++k2) {
-            const int kk = 2 * k2 + half;
-            const uint32_t acc = (prev_first && kk == 0) ? 0u : 1u;
-            // dS^T of queries [16kk, 16kk+16) at columns 16kk + 8, P^T at 16kk
-            mma_ts(t_dk, r + kk * 16 + 8, mq + (uint64_t)((kk * 2048) >> 4), idTS, acc);
-            mma_ts(t_dv, r + kk * 16, mdo + (uint64_t)((kk * 2048) >> 4), idTS, acc);
-          }
+      // first non-empty item >= it (p.n_items if none), with its step range
+      auto seek = [&](int it, int& beg, int& end) -> int {
+        for (; it < p.n_items; it += gridDim.x) {
+          item_range(it, beg, end);
+          if (end > beg) return it;
         }
-        mma_commit(&q_empty[slot]);
-        mma_commit(&o_empty[slot]);
-        if (prev_last) mma_commit(acc_full);
-        have_prev = false;
+        return p.n_items;
+      };
+      // S^T(g) = K Q^T into R[g & 1]; the first step of an item waits for the item's K/V
+      auto issue_S = [&](int gg, bool item_first) -> bool {
+        if (item_first) {
+          if (!mbar_wait(kv_full, kv_items & 1, abort_flag)) return false;
+          ++kv_items;
+        }
+        if (!mbar_wait(&q_full[gg & 1], (gg >> 1) & 1, abort_flag)) return false;
+        tc_fence_after();
+        const uint64_t rq = dQk + (uint64_t)(((gg & 1) * L::kTileBytes) >> 4);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
+          mma_ss(tmem_base + (gg & 1) * 128, dK0 + off, rq + off, idSS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(s_full);
         return true;
       };
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        int beg, end;
-        item_range(item, beg, end);
-        if (end == beg) continue;
-        if (!mbar_wait(kv_full, items & 1, abort_flag)) { ok = false; break; }
-        ++items;
+      // dP^T(g) = V dO^T into R[(g & 1) ^ 1]; after an item's last one K_j, V_j are free
+      auto issue_dP = [&](int gg, bool item_last) -> bool {
+        if (!mbar_wait(&o_full[gg & 1], (gg >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
-        for (int e = beg; e < end; ++e) {
-          const int slot = gs % NS;
-          // S^T(g) = K Q^T into R[g & 1] (free once dP^T(g-1) was read out)
-          if (gs > 0) {
-            if (!mbar_wait(loaded, (gs - 1) & 1, abort_flag)) { ok = false; break; }
-          }
-          if (!mbar_wait(&q_full[slot], (gs / NS) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t rx = tmem_base + (gs & 1) * 128, ry = tmem_base + ((gs & 1) ^ 1) * 128;
-          const uint64_t rq = dQk + (uint64_t)((slot * L::kTileBytes) >> 4);
+        const uint64_t rdo = dOk + (uint64_t)(((gg & 1) * L::kTileBytes) >> 4);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
-            mma_ss(rx, dK0 + off, rq + off, idSS, kk > 0 ? 1u : 0u);
-          }
-          if (have_prev && !finish_prev()) { ok = false; break; }
-          // dP^T(g) = V dO^T into R[(g & 1) ^ 1], after dK(g-1) / dV(g-1) read it
-          if (!mbar_wait(&o_full[slot], (gs / NS) & 1, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          const uint64_t rdo = dOk + (uint64_t)((slot * L::kTileBytes) >> 4);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
-            mma_ss(ry, dV0 + off, rdo + off, idSS, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(s_full);
-          if (e == end - 1) mma_commit(kv_empty);  // K_j, V_j: last S^T / dP^T issued
-          have_prev = true;
-          prev_first = e == beg;
-          prev_last = e == end - 1;
-          ++gs;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
+          mma_ss(tmem_base + ((gg & 1) ^ 1) * 128, dV0 + off, rdo + off, idSS, kk > 0 ? 1u : 0u);
         }
+        mma_commit(dp_full);
+        if (item_last) mma_commit(kv_empty);
+        return true;
+      };
+      // dV(g) += P^T(g) dO or dK(g) += dS^T(g) Q; the K16 slice kk of P^T sits at column
+      // 32*(kk/2) + 8*(kk%2) of R[g & 1], of dS^T 16 columns further
+      auto issue_grad = [&](int gg, bool item_first, bool is_dk) {
+        const uint32_t r = tmem_base + (gg & 1) * 128 + (is_dk ? 16 : 0);
+        const uint64_t mb = (is_dk ? dQmn : dOmn) + (uint64_t)(((gg & 1) * L::kTileBytes) >> 4);
+        const uint32_t acc_d = is_dk ? t_dk : t_dv;
+#pragma unroll
+        for (int kk = 0; kk < BS / 16; ++kk)
+          mma_ts(acc_d, r + 32 * (kk >> 1) + 8 * (kk & 1), mb + (uint64_t)((kk * 2048) >> 4), idTS,
+                 (item_first && kk == 0) ? 0u : 1u);
+      };
+      // Per step g: dV(g) | S^T(g+1) (into the region dP^T(g) left) | dK(g) | dP^T(g+1) (into
+      // the region dV(g), dK(g) just read).  The elementwise warps form P^T(g+1) while the
+      // tensor cores run dK(g) and dP^T(g+1).  The first step of an item is issued at the end
+      // of the previous item's last step (its S^T waits for the item's K/V).
+      int beg = 0, end = 0;
+      int item = seek(blockIdx.x, beg, end);
+      int gg = 0;
+      if (item < p.n_items) ok = issue_S(0, true) && issue_dP(0, end - beg == 1);
+      while (item < p.n_items && ok) {
+        int nbeg = 0, nend = 0;
+        const int nitem = seek(item + gridDim.x, nbeg, nend);
+        for (int e = beg; e < end; ++e, ++gg) {
+          const bool first = e == beg, more = e + 1 < end;
+          if (!mbar_wait(p_ready, gg & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_grad(gg, first, false);
+          mma_commit(&o_empty[gg & 1]);
+          if (more) {
+            if (!mbar_wait(dp_loaded, gg & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (!issue_S(gg + 1, false)) { ok = false; break; }
+          }
+          if (!mbar_wait(ds_ready, gg & 1, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          issue_grad(gg, first, true);
+          mma_commit(&q_empty[gg & 1]);
+          if (more) {
+            if (!issue_dP(gg + 1, e + 2 == end)) { ok = false; break; }
+          } else {
+            mma_commit(acc_full);
+            if (nitem < p.n_items) {
+              if (!mbar_wait(dp_loaded, gg & 1, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+              if (!issue_S(gg + 1, true) || !issue_dP(gg + 1, nend - nbeg == 1)) { ok = false; break; }
+            }
+          }
+        }
+        item = nitem;
+        beg = nbeg;
+        end = nend;
       }
-      if (ok && have_prev) finish_prev();
       mma_commit(fin_bar);
       mbar_wait_drain(fin_bar, 0);
     }
@@ -408,6 +433,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
     const uint32_t t_dv = tmem_base + t_lane + 256, t_dk = tmem_base + t_lane + 384;
     const float sl2 = g.scale * 1.4426950408889634f;
+    const uint64_t sl2x2 = f2pack(sl2, sl2);
     int gs = 0, items = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
@@ -419,60 +445,78 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const int lt = row / (g.bh * g.bw), lh = (row / g.bw) % g.bh, lw = row % g.bw;
       const bool kvalid = lt < vt && lh < vh && lw < vw;
       for (int e = beg; e < end; ++e, ++gs) {
-        bool w_ok = mbar_wait(s_full, gs & 1, abort_flag);
-        w_ok = __all_sync(0xffffffffu, w_ok);
-        if (!w_ok) { ok = false; break; }
-        tc_fence_after();
+        // this group's 32 query columns of step g: P^T = exp2(S^T*sl2 - lse2[q]) as soon as
+        // S^T is in, then dS^T = P^T * (dP^T - delta[q]) once dP^T is; both in bf16 back over
+        // the group's own S^T columns as [P^T 16 cols | dS^T 16 cols]
         const uint32_t rx = tmem_base + t_lane + (gs & 1) * 128;
         const uint32_t ry = tmem_base + t_lane + ((gs & 1) ^ 1) * 128;
         const float* vec = reinterpret_cast<const float*>(smem + L::kVecOff + (gs % NS) * L::kVecBytes);
         const float4* nl4 = reinterpret_cast<const float4*>(vec + cg * 32);       // -lse2[q]
         const float4* nd4 = reinterpret_cast<const float4*>(vec + BS + cg * 32);  // -delta[q]
-        // this group's 32 query columns: P^T = exp2(S^T*sl2 - lse2[q]),
-        // dS^T = P^T * (dP^T - delta[q]), two columns per f32x2 instruction.  dP^T is read
-        // whole (its region takes S^T(g+1) next); S^T 16 columns at a time, and each round's
-        // results go back over the S^T columns it just read -- this group's own -- as
-        // [P^T 8 cols | dS^T 8 cols] per 16 queries, so no other group is involved.
-        uint32_t dr[32], sr[16];
-        tmem_ld32_wait(ry + cg * 32, dr);
-        tmem_ld16_wait(rx + cg * 32, sr);
-        tc_fence_before();
-        mbar_arrive(loaded);  // R[(g & 1) ^ 1] may now take S^T(g+1)
-        const uint64_t sl2x2 = f2pack(sl2, sl2);
-#pragma unroll
-        for (int round = 0; round < 2; ++round) {
-          if (round == 1) tmem_ld16_wait(rx + cg * 32 + 16, sr);
+        bool w_ok = mbar_wait(s_full, gs & 1, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) { ok = false; break; }
+        tc_fence_after();
+        float pf[32];
+        {
+          uint32_t* sr = reinterpret_cast<uint32_t*>(pf);
+          tmem_ld32_wait(rx + cg * 32, sr);
           if (!kvalid) {  // pad key slot: S^T = -inf, so P^T = dS^T = 0
 #pragma unroll
-            for (int c = 0; c < 16; ++c) sr[c] = __float_as_uint(-INFINITY);
+            for (int c = 0; c < 32; ++c) pf[c] = -INFINITY;
           }
-          uint32_t pk[8], dk[8];
+          uint32_t pk[16];
 #pragma unroll
-          for (int e4 = 0; e4 < 4; ++e4) {
-            const float4 nl = nl4[round * 4 + e4], nd = nd4[round * 4 + e4];
+          for (int e4 = 0; e4 < 8; ++e4) {
+            const float4 nl = nl4[e4];
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int j = 2 * e4 + h;           // column pair within the round
-              const int e2 = round * 8 + j;       // column pair within the 32
-              const uint64_t x = fma2(f2pack(__uint_as_float(sr[2 * j]), __uint_as_float(sr[2 * j + 1])),
-                                      sl2x2, h ? f2pack(nl.z, nl.w) : f2pack(nl.x, nl.y));
+              const int e2 = 2 * e4 + h;
               float x0, x1;
-              f2unpack(x, x0, x1);
-              const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-              const uint64_t dd = add2(f2pack(__uint_as_float(dr[2 * e2]), __uint_as_float(dr[2 * e2 + 1])),
-                                       h ? f2pack(nd.z, nd.w) : f2pack(nd.x, nd.y));
+              f2unpack(fma2(f2pack(pf[2 * e2], pf[2 * e2 + 1]), sl2x2,
+                            h ? f2pack(nl.z, nl.w) : f2pack(nl.x, nl.y)), x0, x1);
+              pf[2 * e2] = fast_exp2(x0);
+              pf[2 * e2 + 1] = fast_exp2(x1);
+              pk[e2] = pack_bf16x2(pf[2 * e2], pf[2 * e2 + 1]);
+            }
+          }
+          tmem_st16(rx + cg * 32, pk);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(p_ready);  // dV(g) may start
+        }
+        w_ok = mbar_wait(dp_full, gs & 1, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int round = 0; round < 2; ++round) {
+          uint32_t dr[16], dk[8];
+          tmem_ld16_wait(ry + cg * 32 + round * 16, dr);
+          if (round == 1) {
+            tc_fence_before();
+            mbar_arrive(dp_loaded);  // R[(g & 1) ^ 1] may now take S^T(g+1)
+          }
+#pragma unroll
+          for (int e4 = 0; e4 < 4; ++e4) {
+            const float4 nd = nd4[round * 4 + e4];
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int j = 2 * e4 + h;         // column pair within the round
+              const int e2 = round * 8 + j;     // column pair within the 32
               float s0, s1;
-              f2unpack(mul2(f2pack(p0, p1), dd), s0, s1);
-              pk[j] = pack_bf16x2(p0, p1);
+              f2unpack(mul2(f2pack(pf[2 * e2], pf[2 * e2 + 1]),
+                            add2(f2pack(__uint_as_float(dr[2 * j]), __uint_as_float(dr[2 * j + 1])),
+                                 h ? f2pack(nd.z, nd.w) : f2pack(nd.x, nd.y))),
+                       s0, s1);
               dk[j] = pack_bf16x2(s0, s1);
             }
           }
-          tmem_st8(rx + cg * 32 + round * 16, pk);
-          tmem_st8(rx + cg * 32 + round * 16 + 8, dk);
-          tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&p_full[round]);  // this round's K16 slice of every group is in TMEM
+          tmem_st8(rx + cg * 32 + 16 + round * 8, dk);
         }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(ds_ready);  // dK(g) may start
       }
       if (!ok) break;
       // epilogue: dV, dK rows of this key block (zeros for pad keys / no selections)
