@@ -177,8 +177,8 @@ constexpr int kTile = 128;
 // dS^T(g) are being formed.
 // MMA order: S^T(g) | dK(g-1), dV(g-1), dP^T(g) | S^T(g+1) | ...; dP^T(g) reuses the region
 // that dK(g-1) and dV(g-1) read, after them in issue order.
-// Q_i and dO_i have rings of their own (2 slots each): Q(g) is last read by dK(g), dO(g) by
-// dV(g), so each slot is released as early as its own last MMA allows.
+// Q_i and dO_i (with -lse2_i, -delta_i) share a 2-slot ring; a slot is released after dK(g),
+// its last reader.
 template <int BS, int D>
 struct DkdvLayout {
   static constexpr int kKVBytes = BS * D * 2;      // K_j or V_j
@@ -191,9 +191,9 @@ struct DkdvLayout {
   static constexpr int kVecOff = kDOOff + kSlots * kTileBytes;    // -lse2 / -delta per Q slot
   static constexpr int kVecBytes = 2 * BS * 4;
   static constexpr int kBarOff = kVecOff + kSlots * kVecBytes;
-  // kv_full, kv_empty, q_full[2], q_empty[2], o_full[2], o_empty[2], s_full, dp_full,
-  // p_ready, dp_loaded, ds_ready, acc_full, fin
-  static constexpr int kNumBars = 2 + 4 * kSlots + 7;
+  // kv_full, kv_empty, q_full[2], q_empty[2], s_full, dp_full, p_ready, dp_loaded, ds_ready,
+  // acc_full, fin
+  static constexpr int kNumBars = 2 + 2 * kSlots + 7;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kAlloc = kMiscOff + 16 + 1024;
 };
@@ -212,11 +212,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
   uint64_t* kv_full = bars;           // K_j, V_j landed (one phase per non-empty item)
   uint64_t* kv_empty = bars + 1;      // K_j, V_j no longer needed
-  uint64_t* q_full = bars + 2;        // [NS] Q_i, lse2_i, delta_i landed
-  uint64_t* q_empty = q_full + NS;    // [NS]
-  uint64_t* o_full = q_empty + NS;    // [NS] dO_i landed
-  uint64_t* o_empty = o_full + NS;    // [NS]
-  uint64_t* s_full = o_empty + NS;    // S^T(g) in TMEM
+  uint64_t* q_full = bars + 2;        // [NS] Q_i, dO_i, -lse2_i, -delta_i landed in the slot
+  uint64_t* q_empty = q_full + NS;    // [NS] slot free (after dK(g), the slot's last reader)
+  uint64_t* s_full = q_empty + NS;    // S^T(g) in TMEM
   uint64_t* dp_full = s_full + 1;     // dP^T(g) in TMEM
   uint64_t* p_ready = dp_full + 1;    // P^T(g) (bf16) in TMEM (kBwdElem arrivals)
   uint64_t* dp_loaded = p_ready + 1;  // dP^T(g) read into registers (kBwdElem arrivals)
@@ -234,8 +232,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int s = 0; s < NS; ++s) {
       mbar_init(&q_full[s], 1);
       mbar_init(&q_empty[s], 1);
-      mbar_init(&o_full[s], 1);
-      mbar_init(&o_empty[s], 1);
     }
     mbar_init(s_full, 1);
     mbar_init(dp_full, 1);
@@ -266,7 +262,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ====================================================== TMA producer
     if (lane == 0) {
       int gq = 0, items = 0;        // steps, non-empty items
-      int q_loads = 0, o_loads = 0;  // copies issued per ring (for the drain)
+      int q_loads = 0;               // slot loads issued (for the drain)
       bool ok = true;
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         int beg, end;
@@ -291,29 +287,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int qrow = (bh * g.NBq + i) * BS;
           if (round > 0 && !mbar_wait(&q_empty[slot], (round - 1) & 1, abort_flag)) { ok = false; break; }
           unsigned char* vec = smem + L::kVecOff + slot * L::kVecBytes;
-          mbar_expect_tx(&q_full[slot], L::kTileBytes + L::kVecBytes);
+          mbar_expect_tx(&q_full[slot], 2 * L::kTileBytes + L::kVecBytes);
 #pragma unroll
-          for (int half = 0; half < D / 64; ++half)
+          for (int half = 0; half < D / 64; ++half) {
             tma_load_2d(smem + L::kQOff + slot * L::kTileBytes + half * BS * 128, &tmQ, half * 64,
                         qrow, &q_full[slot]);
+            tma_load_2d(smem + L::kDOOff + slot * L::kTileBytes + half * BS * 128, &tmdO, half * 64,
+                        qrow, &q_full[slot]);
+          }
           bulk_load(vec, p.nlse2 + (size_t)qrow, BS * 4, &q_full[slot]);
           bulk_load(vec + BS * 4, p.ndelta + (size_t)qrow, BS * 4, &q_full[slot]);
           ++q_loads;
-          if (round > 0 && !mbar_wait(&o_empty[slot], (round - 1) & 1, abort_flag)) { ok = false; break; }
-          mbar_expect_tx(&o_full[slot], L::kTileBytes);
-#pragma unroll
-          for (int half = 0; half < D / 64; ++half)
-            tma_load_2d(smem + L::kDOOff + slot * L::kTileBytes + half * BS * 128, &tmdO, half * 64,
-                        qrow, &o_full[slot]);
-          ++o_loads;
         }
       }
       // drain every copy still in flight
       for (int s = 0; s < NS; ++s) {
         const int ql = q_loads / NS + (s < q_loads % NS ? 1 : 0);
-        const int ol = o_loads / NS + (s < o_loads % NS ? 1 : 0);
         if (ql > 0) mbar_wait_drain(&q_full[s], (ql - 1) & 1);
-        if (ol > 0) mbar_wait_drain(&o_full[s], (ol - 1) & 1);
       }
       if (items > 0) mbar_wait_drain(kv_full, (items - 1) & 1);
     }
@@ -357,10 +347,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_commit(s_full);
         return true;
       };
-      // dP^T(g) = V dO^T into R[(g & 1) ^ 1]; after an item's last one K_j, V_j are free
+      // dP^T(g) = V dO^T into R[(g & 1) ^ 1] (dO landed with Q: issue_S(g) waited for the
+      // slot); after an item's last one K_j, V_j are free
       auto issue_dP = [&](int gg, bool item_last) -> bool {
-        if (!mbar_wait(&o_full[gg & 1], (gg >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
         const uint64_t rdo = dOk + (uint64_t)(((gg & 1) * L::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -398,7 +387,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           if (!mbar_wait(p_ready, gg & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           issue_grad(gg, first, false);
-          mma_commit(&o_empty[gg & 1]);
           if (more) {
             if (!mbar_wait(dp_loaded, gg & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
