@@ -24,7 +24,7 @@
 namespace bsa {
 
 struct BwdWs {
-  size_t ndelta, nlse2, rev_off, rev_list, total;
+  size_t ndelta, nlse2, rev_off, rev_list, ctr, total;
 };
 inline size_t bwd_align(size_t x) { return (x + 255) & ~size_t(255); }
 BwdWs bwd_ws_layout(const Geo& g, int r) {
@@ -34,7 +34,8 @@ BwdWs bwd_ws_layout(const Geo& g, int r) {
   w.nlse2 = bwd_align(rows * 4);
   w.rev_off = w.nlse2 + bwd_align(rows * 4);
   w.rev_list = w.rev_off + bwd_align((size_t)g.B * g.H * (g.NBk + 1) * 4);
-  w.total = w.rev_list + bwd_align((size_t)g.B * g.H * g.NBq * r * 4);
+  w.ctr = w.rev_list + bwd_align((size_t)g.B * g.H * g.NBq * r * 4);
+  w.total = w.ctr + 256;  // dK/dV work counter (one int, zeroed by the prep pass)
   return w;
 }
 struct BwdPtrs {
@@ -55,6 +56,7 @@ struct BwdParams {
   const int* rev_list;    // [B*H][NBq*r]
   const float* ndelta;    // [B*H*NBq*BS] -Delta
   const float* nlse2;     // [B*H*NBq*BS] -LSE * log2(e), -inf for pad rows
+  int* ctr;               // dkdv: next item to hand out (minus gridDim.x), zeroed by prep
   __nv_bfloat16* out0;    // dkdv: dK, dq: dQ
   __nv_bfloat16* out1;    // dkdv: dV
 };
@@ -68,8 +70,10 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
                                                        const __nv_bfloat16* __restrict__ dO,
                                                        const float* __restrict__ lse,
                                                        float* __restrict__ ndelta,
-                                                       float* __restrict__ nlse2, size_t rows) {
+                                                       float* __restrict__ nlse2, size_t rows,
+                                                       int* __restrict__ ctr) {
   constexpr int LPR = D / 8;  // lanes per row (16-byte vectors)
+  if (blockIdx.x == 0 && threadIdx.x == 0) *ctr = 0;  // the dK/dV pass's work counter
   const size_t t = (size_t)blockIdx.x * blockDim.x + threadIdx.x;
   const size_t row = t / LPR;
   const int c = (int)(t % LPR);
@@ -192,10 +196,12 @@ struct DkdvLayout {
   static constexpr int kVecBytes = 2 * BS * 4;
   static constexpr int kBarOff = kVecOff + kSlots * kVecBytes;
   // kv_full, kv_empty, q_full[2], q_empty[2], s_full, dp_full, p_ready, dp_loaded, ds_ready,
-  // acc_full, fin
-  static constexpr int kNumBars = 2 + 2 * kSlots + 7;
+  // acc_full, fin, iq_full[kQueue], iq_empty[kQueue]
+  static constexpr int kQueue = 4;  // items handed from the producer to the other roles
+  static constexpr int kNumBars = 2 + 2 * kSlots + 7 + 2 * kQueue;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kAlloc = kMiscOff + 16 + 1024;
+  static constexpr int kQueueOff = kMiscOff + 16;  // int [kQueue]
+  static constexpr int kAlloc = kQueueOff + kQueue * 4 + 1024;
 };
 
 template <int BS, int D>
@@ -221,12 +227,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* ds_ready = dp_loaded + 1; // dS^T(g) (bf16) in TMEM (kBwdElem arrivals)
   uint64_t* acc_full = ds_ready + 1;  // dV and dK of the item complete
   uint64_t* fin_bar = acc_full + 1;
+  uint64_t* iq_full = fin_bar + 1;            // [kQueue] queue entry written (producer)
+  uint64_t* iq_empty = iq_full + L::kQueue;   // [kQueue] entry read by the MMA thread and
+                                              // every elementwise thread
+  volatile int* iq = reinterpret_cast<volatile int*>(smem + L::kQueueOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const Geo& g = p.g;
 
   if (tid == 0) {
+    for (int k = 0; k < L::kQueue; ++k) {
+      mbar_init(&iq_full[k], 1);
+      mbar_init(&iq_empty[k], 1 + kBwdElem);
+    }
     mbar_init(kv_full, 1);
     mbar_init(kv_empty, 1);
     for (int s = 0; s < NS; ++s) {
@@ -257,6 +271,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     end = off[1];
     if (beg < 0 || end < beg || end > g.NBq * p.r) { set_status(DEV_BAD_INDEX); beg = end = 0; }
   };
+  // Work distribution: items (key blocks) are handed out dynamically in their natural
+  // head-major order -- the first one per CTA is blockIdx.x, the rest come from a global
+  // counter -- so the CTAs finish together although items differ in steps (a key block is
+  // selected by anything from a few to a few hundred query blocks).  The producer fetches,
+  // zero-fills empty items itself, and passes the non-empty ones (then -1) to the MMA thread
+  // and the elementwise warps through a small queue in shared memory.
+  auto read_item = [&](int k, bool elem) -> int {  // k-th queue entry; -1 = no more
+    const int slot = k % L::kQueue;
+    bool w_ok = mbar_wait(&iq_full[slot], (k / L::kQueue) & 1, abort_flag);
+    if (elem) w_ok = __all_sync(0xffffffffu, w_ok);
+    if (!w_ok) return -1;
+    const int it = iq[slot];
+    mbar_arrive(&iq_empty[slot]);
+    return it;
+  };
 
   if (warp == kBwdProducer) {
     // ====================================================== TMA producer
@@ -264,10 +293,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int gq = 0, items = 0;        // steps, non-empty items
       int q_loads = 0;               // slot loads issued (for the drain)
       bool ok = true;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        int beg, end;
-        item_range(item, beg, end);
-        if (end == beg) continue;
+      for (int k = 0; ok; ++k) {
+        // next non-empty item; empty ones get their zero dK / dV rows here
+        int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.ctr, 1);
+        int beg = 0, end = 0;
+        while (item < p.n_items) {
+          item_range(item, beg, end);
+          if (end > beg) break;
+          const uint4 z = make_uint4(0, 0, 0, 0);
+          uint4* dk4 = reinterpret_cast<uint4*>(p.out0 + (size_t)item * BS * D);
+          uint4* dv4 = reinterpret_cast<uint4*>(p.out1 + (size_t)item * BS * D);
+          for (int c = 0; c < BS * D / 8; ++c) { dk4[c] = z; dv4[c] = z; }
+          item = (int)gridDim.x + atomicAdd(p.ctr, 1);
+        }
+        const int slot = k % L::kQueue;
+        if (k >= L::kQueue && !mbar_wait(&iq_empty[slot], ((k / L::kQueue) - 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        iq[slot] = item < p.n_items ? item : -1;
+        mbar_arrive(&iq_full[slot]);
+        if (item >= p.n_items) break;
         const int bh = item / g.NBq, jc = item % g.NBq;
         // K_j, V_j for the item (once the previous item's S^T / dP^T MMAs released them)
         if (items > 0 && !mbar_wait(kv_empty, (items - 1) & 1, abort_flag)) { ok = false; break; }
@@ -322,14 +368,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       static_assert(NS == 2, "slot = step & 1");
       int kv_items = 0;  // K/V loads waited for
       bool ok = true;
-      // first non-empty item >= it (p.n_items if none), with its step range
-      auto seek = [&](int it, int& beg, int& end) -> int {
-        for (; it < p.n_items; it += gridDim.x) {
-          item_range(it, beg, end);
-          if (end > beg) return it;
-        }
-        return p.n_items;
-      };
       // S^T(g) = K Q^T into R[g & 1]; the first step of an item waits for the item's K/V
       auto issue_S = [&](int gg, bool item_first) -> bool {
         if (item_first) {
@@ -375,13 +413,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // the region dV(g), dK(g) just read).  The elementwise warps form P^T(g+1) while the
       // tensor cores run dK(g) and dP^T(g+1).  The first step of an item is issued at the end
       // of the previous item's last step (its S^T waits for the item's K/V).
-      int beg = 0, end = 0;
-      int item = seek(blockIdx.x, beg, end);
+      int beg = 0, end = 0, kq = 0;
+      int item = read_item(kq++, false);
       int gg = 0;
-      if (item < p.n_items) ok = issue_S(0, true) && issue_dP(0, end - beg == 1);
-      while (item < p.n_items && ok) {
-        int nbeg = 0, nend = 0;
-        const int nitem = seek(item + gridDim.x, nbeg, nend);
+      if (item >= 0) {
+        item_range(item, beg, end);
+        ok = issue_S(0, true) && issue_dP(0, end - beg == 1);
+      }
+      while (item >= 0 && ok) {
+        int nitem = -1, nbeg = 0, nend = 0;
         for (int e = beg; e < end; ++e, ++gg) {
           const bool first = e == beg, more = e + 1 < end;
           if (!mbar_wait(p_ready, gg & 1, abort_flag)) { ok = false; break; }
@@ -400,7 +440,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!issue_dP(gg + 1, e + 2 == end)) { ok = false; break; }
           } else {
             mma_commit(acc_full);
-            if (nitem < p.n_items) {
+            nitem = read_item(kq++, false);  // the next item, looked up at this item's end
+            if (nitem >= 0) {
+              item_range(nitem, nbeg, nend);
               if (!mbar_wait(dp_loaded, gg & 1, abort_flag)) { ok = false; break; }
               tc_fence_after();
               if (!issue_S(gg + 1, true) || !issue_dP(gg + 1, nend - nbeg == 1)) { ok = false; break; }
@@ -424,7 +466,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint64_t sl2x2 = f2pack(sl2, sl2);
     int gs = 0, items = 0;
     bool ok = true;
-    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
+    for (int k = 0; ok; ++k) {
+      const int item = read_item(k, true);
+      if (item < 0) break;
       int beg, end;
       item_range(item, beg, end);
       const int jc = item % g.NBq;
@@ -507,41 +551,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_arrive(ds_ready);  // dK(g) may start
       }
       if (!ok) break;
-      // epilogue: dV, dK rows of this key block (zeros for pad keys / no selections)
+      // epilogue: dV, dK rows of this key block (zeros for pad keys)
       const size_t orow = (size_t)item * BS + row;
       __nv_bfloat16* dv_row = p.out1 + orow * D;
       __nv_bfloat16* dk_row = p.out0 + orow * D;
-      if (end > beg) {
-        bool w_ok = mbar_wait(acc_full, items & 1, abort_flag);
-        w_ok = __all_sync(0xffffffffu, w_ok);
-        if (!w_ok) { ok = false; break; }
-        ++items;
-        tc_fence_after();
-        constexpr int DC = D / 4;  // dV / dK columns of this group, 16 at a time
+      bool w_ok = mbar_wait(acc_full, items & 1, abort_flag);
+      w_ok = __all_sync(0xffffffffu, w_ok);
+      if (!w_ok) { ok = false; break; }
+      ++items;
+      tc_fence_after();
+      constexpr int DC = D / 4;  // dV / dK columns of this group, 16 at a time
 #pragma unroll
-        for (int c0 = 0; c0 < DC; c0 += 16) {
+      for (int c0 = 0; c0 < DC; c0 += 16) {
 #pragma unroll
-          for (int which = 0; which < 2; ++which) {  // dV, then dK (scaled)
-            uint32_t a[16];
-            tmem_ld16_wait((which ? t_dk : t_dv) + cg * DC + c0, a);
-            const float sc = which ? g.scale : 1.0f;
-            uint4 va[2];
-            uint32_t* a32 = reinterpret_cast<uint32_t*>(va);
+        for (int which = 0; which < 2; ++which) {  // dV, then dK (scaled)
+          uint32_t a[16];
+          tmem_ld16_wait((which ? t_dk : t_dv) + cg * DC + c0, a);
+          const float sc = which ? g.scale : 1.0f;
+          uint4 va[2];
+          uint32_t* a32 = reinterpret_cast<uint32_t*>(va);
 #pragma unroll
-            for (int e2 = 0; e2 < 8; ++e2)
-              a32[e2] = kvalid ? pack_bf16x2(__uint_as_float(a[2 * e2]) * sc, __uint_as_float(a[2 * e2 + 1]) * sc)
-                               : 0u;
-            __nv_bfloat16* dst = (which ? dk_row : dv_row) + cg * DC + c0;
-            reinterpret_cast<uint4*>(dst)[0] = va[0];
-            reinterpret_cast<uint4*>(dst)[1] = va[1];
-          }
-        }
-      } else {
-        const uint4 z = make_uint4(0, 0, 0, 0);
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-          reinterpret_cast<uint4*>(dv_row + cg * (D / 4))[c] = z;
-          reinterpret_cast<uint4*>(dk_row + cg * (D / 4))[c] = z;
+          for (int e2 = 0; e2 < 8; ++e2)
+            a32[e2] = kvalid ? pack_bf16x2(__uint_as_float(a[2 * e2]) * sc, __uint_as_float(a[2 * e2 + 1]) * sc)
+                             : 0u;
+          __nv_bfloat16* dst = (which ? dk_row : dv_row) + cg * DC + c0;
+          reinterpret_cast<uint4*>(dst)[0] = va[0];
+          reinterpret_cast<uint4*>(dst)[1] = va[1];
         }
       }
     }
@@ -555,8 +590,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 // ------------------------------------------------------------------------------ dQ
 // Work item = query block (b, h, i); steps = its selected key blocks (cached ones included).
 // TMEM: S0 [0,128), S1 [128,256), dP [256,384), dQ [384,512); dS (bf16) overwrites the S
-// buffer it came from, each 32-key group's 16 columns over the first half of its own S columns.  MMA order per step n: dP(n) once the previous dP was read out,
-// dQ += dS(n-1) K_{n-1}, S(n+1); so the tensor cores run while dS(n) is formed.
+// buffer it came from, each 32-key group's 16 columns over the first half of its own S
+// columns.  MMA order per step n: dP(n+1) once dP(n) was read out, dQ += dS(n) K_n, S(n+2);
+// so the tensor cores run while dS(n+1) is formed.
 template <int BS, int D>
 struct DqLayout {
   static constexpr int kTileBytes = kTile * D * 2;  // Q_i / dO_i (128-row tiles)
@@ -877,6 +913,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
   float* nlse2 = reinterpret_cast<float*>(P.ws + w.nlse2);
   int* rev_off = reinterpret_cast<int*>(P.ws + w.rev_off);
   int* rev_list = reinterpret_cast<int*>(P.ws + w.rev_list);
+  int* ctr = reinterpret_cast<int*>(P.ws + w.ctr);
   const size_t rows = (size_t)g.B * g.H * g.NBq * g.BS;
   {
     const size_t threads = rows * (g.D / 8);
@@ -884,11 +921,11 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
     if (g.D == 128)
       bwd_prep_kernel<128><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(P.o),
                                                   static_cast<const __nv_bfloat16*>(P.dO), P.lse,
-                                                  ndelta, nlse2, rows);
+                                                  ndelta, nlse2, rows, ctr);
     else
       bwd_prep_kernel<64><<<blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(P.o),
                                                  static_cast<const __nv_bfloat16*>(P.dO), P.lse,
-                                                 ndelta, nlse2, rows);
+                                                 ndelta, nlse2, rows, ctr);
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   BwdParams bp;
@@ -901,6 +938,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
   bp.rev_list = rev_list;
   bp.ndelta = ndelta;
   bp.nlse2 = nlse2;
+  bp.ctr = ctr;
   {
     const size_t smem = (size_t)(g.NBk + kRevThreads) * 4;
     if (cudaFuncSetAttribute(bwd_revidx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

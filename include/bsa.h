@@ -94,7 +94,8 @@ BSA_API int32_t bsa_abi_version(void);
 
 /* Bytes of workspace `which` (BSA_WS_*) needs for this geometry; 0 on invalid arguments.
  * Workspace must be 256-byte aligned.  ROUTE: pooled q/k means.  FWD: none (returns 0).
- * BWD: fp32 dQ accumulator, row sums of dO*O and the key-block -> query-block index. */
+ * BWD: per query row -Delta (Delta = rowsum(dO*O)) and -LSE*log2(e), the key-block ->
+ * query-block index and a work counter of the dK/dV pass. */
 BSA_API size_t bsa_workspace_size(const bsa_geom_t* g, int32_t top_r, int32_t which);
 
 /* Fused QK-RMSNorm + 3D RoPE prologue and raster -> blocked relayout.

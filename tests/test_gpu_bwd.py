@@ -82,6 +82,16 @@ def test_backward_all_blocks_selected():
     check_bwd(w, pipe, x, [0, 1])
 
 
+def test_backward_top1_leaves_key_blocks_unselected():
+    """r = 1: most key blocks are selected by no query block; their dK / dV rows must be exactly
+    zero, and the work distribution of the dK/dV pass must skip them without stalling."""
+    w = WORKLOADS["small"]
+    pipe, x = run_fwd_bwd(w, top_r=1)
+    idx = pipe.idx.cpu().numpy()
+    assert np.unique(idx[idx >= 0]).size < pipe.g.nbq  # some blocks really are unselected
+    check_bwd(w, pipe, x, list(range(w.heads)))
+
+
 def test_backward_480p_sampled_heads():
     w = WORKLOADS["480p_bwd"]
     pipe, x = run_fwd_bwd(w)
