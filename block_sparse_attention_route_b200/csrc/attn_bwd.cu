@@ -99,39 +99,56 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 }
 
 // ------------------------------------------------------------------------------ reverse index
-// One CTA per (b, h).  Counts how often each key block is selected, scans the counts into
-// offsets, then fills each key block's list with the query blocks that selected it, in
-// increasing query-block order (rows are visited in order; a row never repeats a block).
-constexpr int kRevThreads = 256;
+// One CTA per (b, h) with kRevChunks warps; warp w owns a contiguous chunk of query blocks.
+// (1) each warp counts, per key block, the selections in its chunk; (2) per key block the
+// chunk counts are scanned, then the totals over key blocks, giving the CSR offsets and each
+// chunk's first position in each list; (3) each warp fills its chunk's entries in increasing
+// query-block order.  Lists come out ordered by i, deterministically and without atomics:
+// the entries of one row are distinct blocks, so the lanes handling a row touch distinct
+// counters.
+constexpr int kRevChunks = 8;
+constexpr int kRevThreads = 32 * kRevChunks;
 __global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams p, int* rev_off,
                                                                 int* rev_list) {
-  extern __shared__ int rsm[];  // cnt/cursor [NBk], scan scratch [kRevThreads]
+  // counts / cursors [kRevChunks][NBk], totals [NBk], scan scratch [kRevThreads]
+  extern __shared__ int rsm[];
   const Geo& g = p.g;
   const int bh = blockIdx.x;
-  int* cntk = rsm;
-  int* part = rsm + g.NBk;
-  const int tid = threadIdx.x;
-  for (int j = tid; j < g.NBk; j += kRevThreads) cntk[j] = 0;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  int* tot = rsm + kRevChunks * g.NBk;
+  int* part = tot + g.NBk;
+  for (int e = tid; e < kRevChunks * g.NBk; e += kRevThreads) rsm[e] = 0;
   __syncthreads();
   const int* idx = p.idx + (size_t)bh * g.NBq * p.r;
   const int* cnt = p.cnt + (size_t)bh * g.NBq;
-  for (int e = tid; e < g.NBq * p.r; e += kRevThreads) {
-    const int i = e / p.r, n = e % p.r;
+  const int per_chunk = (g.NBq + kRevChunks - 1) / kRevChunks;
+  const int i0 = warp * per_chunk, i1 = min(g.NBq, i0 + per_chunk);
+  int* ck = rsm + warp * g.NBk;
+  for (int i = i0; i < i1; ++i) {
     int c = cnt[i];
     if (c < 0 || c > p.r) { set_status(DEV_BAD_INDEX); c = min(max(c, 0), p.r); }
-    if (n < c) {
-      const int j = idx[e];
-      if (j >= 0 && j < g.NBk) atomicAdd(&cntk[j], 1);
+    for (int n = lane; n < c; n += 32) {
+      const int j = idx[(size_t)i * p.r + n];
+      if (j >= 0 && j < g.NBk) ck[j] += 1;
       else set_status(DEV_BAD_INDEX);
     }
+    __syncwarp();
   }
   __syncthreads();
-  // exclusive scan: each thread scans a contiguous chunk, then the chunk totals
   const int per = (g.NBk + kRevThreads - 1) / kRevThreads;
-  const int j0 = tid * per, j1 = min(g.NBk, j0 + per);
-  int s = 0;
-  for (int j = j0; j < j1; ++j) s += cntk[j];
-  part[tid] = s;
+  const int j0 = min(g.NBk, tid * per), j1 = min(g.NBk, j0 + per);
+  int s_sum = 0;
+  for (int j = j0; j < j1; ++j) {  // exclusive scan over the chunks of key block j
+    int run = 0;
+    for (int w = 0; w < kRevChunks; ++w) {
+      const int v = rsm[w * g.NBk + j];
+      rsm[w * g.NBk + j] = run;
+      run += v;
+    }
+    tot[j] = run;
+    s_sum += run;
+  }
+  part[tid] = s_sum;
   __syncthreads();
   if (tid == 0) {
     int run = 0;
@@ -140,19 +157,25 @@ __global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams
   __syncthreads();
   int run = part[tid];
   int* off = rev_off + (size_t)bh * (g.NBk + 1);
-  for (int j = j0; j < j1; ++j) { const int v = cntk[j]; off[j] = run; cntk[j] = run; run += v; }
-  if (tid == kRevThreads - 1) off[g.NBk] = run;
+  for (int j = j0; j < j1; ++j) {  // list start of key block j; each chunk's first position
+    off[j] = run;
+    for (int w = 0; w < kRevChunks; ++w) rsm[w * g.NBk + j] += run;
+    run += tot[j];
+  }
+  if (tid == kRevThreads - 1) off[g.NBk] = run;  // the last range ends at NBk: run = total
   __syncthreads();
-  if (tid < 32) {  // one warp fills rows in order; entries of a row have distinct blocks
-    int* list = rev_list + (size_t)bh * g.NBq * p.r;
-    for (int i = 0; i < g.NBq; ++i) {
-      const int c = min(max(cnt[i], 0), p.r);
-      for (int n = tid; n < c; n += 32) {
-        const int j = idx[(size_t)i * p.r + n];
-        if (j >= 0 && j < g.NBk) list[cntk[j]++] = i;
+  int* list = rev_list + (size_t)bh * g.NBq * p.r;
+  const int cap = g.NBq * p.r;
+  for (int i = i0; i < i1; ++i) {
+    const int c = min(max(cnt[i], 0), p.r);
+    for (int n = lane; n < c; n += 32) {
+      const int j = idx[(size_t)i * p.r + n];
+      if (j >= 0 && j < g.NBk) {
+        const int pos = ck[j]++;
+        if (pos < cap) list[pos] = i;
       }
-      __syncwarp();
     }
+    __syncwarp();
   }
 }
 
@@ -940,7 +963,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
   bp.nlse2 = nlse2;
   bp.ctr = ctr;
   {
-    const size_t smem = (size_t)(g.NBk + kRevThreads) * 4;
+    const size_t smem = (size_t)((kRevChunks + 1) * g.NBk + kRevThreads) * 4;
     if (cudaFuncSetAttribute(bwd_revidx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return BSA_ERR_CUDA;
