@@ -50,7 +50,7 @@ KERNEL_NAMES = {"fwd": "bsa_fwd_kernel", "bwd_dkdv": "bsa_bwd_dkdv_kernel",
 # selected block pair (fwd, dq) or a pair with a current key block (dkdv).  Traffic grows with
 # the pairs a launch processes, so a full launch is scaled from it.  None = not captured for
 # the kernel as it now stands.
-DRAM_BYTES_PER_PAIR = {"fwd": 3855, "bwd_dkdv": None, "bwd_dq": None}
+DRAM_BYTES_PER_PAIR = {"fwd": 3854, "bwd_dkdv": 5764, "bwd_dq": 4838}
 
 
 def traffic_per_launch(kernel, workload, n_pairs, n_pairs_cur):
