@@ -612,21 +612,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
 // ------------------------------------------------------------------------------ dQ
 // Work item = query block (b, h, i); steps = its selected key blocks (cached ones included).
-// TMEM: S0 [0,128), S1 [128,256), dP [256,384), dQ [384,512); dS (bf16) overwrites the S
-// buffer it came from, each 32-key group's 16 columns over the first half of its own S
-// columns.  MMA order per step n: dP(n+1) once dP(n) was read out, dQ += dS(n) K_n, S(n+2);
-// so the tensor cores run while dS(n+1) is formed.
+// TMEM: Q [0,64) and dO [64,128) as bf16 pairs (A operands, copied in by the elementwise warps
+// from the TMA-staged tiles once per item), S [128,256), dP [256,384), dQ [384,512).  dS (bf16)
+// goes back over dP, each 32-key group's 16 columns over the first half of its own dP columns,
+// and feeds dQ += dS K_n from TMEM.  All three MMAs read one operand from TMEM, so per pair
+// shared memory serves only the K / V tiles.  MMA order per step n: S(n+1) (once S(n) was read
+// out) | dQ(n), dP(n+1) (once dS(n) is in): the exponentials of step n+1 run while the tensor
+// cores do dQ(n) and dP(n+1).
 template <int BS, int D>
 struct DqLayout {
-  static constexpr int kTileBytes = kTile * D * 2;  // Q_i / dO_i (128-row tiles)
+  static constexpr int kTileBytes = kTile * D * 2;  // Q_i / dO_i staging (128-row tiles)
   static constexpr int kKVBytes = BS * D * 2;
   static constexpr int kQOff = 0;
   static constexpr int kDOOff = kTileBytes;
   static constexpr int kRingOff = 2 * kTileBytes;
   static constexpr int kStages = 5;
   static constexpr int kBarOff = kRingOff + kStages * kKVBytes;
-  // q_full, q_empty, kv_full[5], kv_empty[5], s_full[2], dp_free, ds_full[2], dq_full, fin
-  static constexpr int kNumBars = 2 + 2 * kStages + 2 + 1 + 2 + 2;
+  // q_full, q_empty, kv_full[5], kv_empty[5], s_full, s_loaded, dp_full, ds_full, dq_full, fin
+  static constexpr int kNumBars = 2 + 2 * kStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kMaskOff = kMiscOff + 16;  // u32 [12 shapes][BS / 32]
   static constexpr int kAlloc = kMaskOff + 12 * (BS / 32) * 4 + 1024;
@@ -640,18 +643,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                       const BwdParams p) {
   using L = DqLayout<BS, D>;
   constexpr int S = L::kStages;
+  static_assert(BS == 128, "dS of one row fills the 32-key groups of a 128-key block");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars;
-  uint64_t* q_empty = bars + 1;
+  uint64_t* q_full = bars;            // Q_i, dO_i staged in shared memory
+  uint64_t* q_empty = bars + 1;       // ... and copied into TMEM (kBwdElem arrivals); the MMA
+                                      // thread waits on it too before the item's first S
   uint64_t* kv_full = bars + 2;
   uint64_t* kv_empty = kv_full + S;
-  uint64_t* s_full = kv_empty + S;   // [2] S(n) and dP(n) complete (committed after dP)
-  uint64_t* dp_free = s_full + 2;    // dP read out (128 arrivals)
-  uint64_t* ds_full = dp_free + 1;   // [2] dS(n) in TMEM (128 arrivals)
-  uint64_t* dq_full = ds_full + 2;
+  uint64_t* s_full = kv_empty + S;    // S(n) in TMEM
+  uint64_t* s_loaded = s_full + 1;    // S(n) read out (kBwdElem arrivals)
+  uint64_t* dp_full = s_loaded + 1;   // dP(n) in TMEM
+  uint64_t* ds_full = dp_full + 1;    // dS(n) in TMEM (kBwdElem arrivals)
+  uint64_t* dq_full = ds_full + 1;    // dQ of the item complete
   uint64_t* fin_bar = dq_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
@@ -660,10 +666,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(q_empty, 1);
+    mbar_init(q_empty, kBwdElem);
     for (int s = 0; s < S; ++s) { mbar_init(&kv_full[s], 1); mbar_init(&kv_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&s_full[b], 1); mbar_init(&ds_full[b], kBwdElem); }
-    mbar_init(dp_free, kBwdElem);
+    mbar_init(s_full, 1);
+    mbar_init(s_loaded, kBwdElem);
+    mbar_init(dp_full, 1);
+    mbar_init(ds_full, kBwdElem);
     mbar_init(dq_full, 1);
     mbar_init(fin_bar, 1);
     *abort_flag = 0;
@@ -675,6 +683,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+  constexpr uint32_t kTq = 0, kTdo = 64, kTs = 128, kTdp = 256, kTdq = 384;  // TMEM columns
 
   auto item_cnt = [&](int item) {
     int c = __ldg(p.cnt + item);
@@ -731,14 +740,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdMma) {
     // ====================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(kTile, BS, 0, 0);
-      constexpr uint32_t idQ = idesc_bf16(kTile, D, 0, 1);
-      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
-      const uint64_t ddo = smem_desc_sw128(smem_u32(smem + L::kDOOff), 16, 1024);
+      constexpr uint32_t idS = idesc_bf16(kTile, BS, 0, 0);   // S, dP: B (K or V tile) K-major
+      constexpr uint32_t idQ = idesc_bf16(kTile, D, 0, 1);    // dQ: B (K tile) MN-major
       const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
       const uint64_t dkmn = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
-      const uint32_t t_dp = tmem_base + 256, t_dq = tmem_base + 384;
-      int qcons = 0, dp_issued = 0, dsw0 = 0, dsw1 = 0;
+      int items = 0, gn = 0;  // non-empty items, global step
       bool ok = true;
       // the ring holds K_n at seq_base + 2n and V_n at seq_base + 2n + 1
       int seq_base = 0;
@@ -747,65 +753,62 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         return true;
       };
-      auto issue_S = [&](int n) -> bool {  // S(n) = Q K_n^T into buffer n & 1
-        const int seq = seq_base + 2 * n;
-        if (!wait_tile(seq)) return false;
-        const uint64_t kb = dk + (uint64_t)(((seq % S) * L::kKVBytes) >> 4);
+      auto mma_S = [&](int n) {  // S(n) = Q K_n^T (A = Q from TMEM)
+        const uint64_t kb = dk + (uint64_t)((((seq_base + 2 * n) % S) * L::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t offq = ((kk / 4) * (kTile * 128) + (kk % 4) * 32) >> 4;
           const uint32_t offk = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
-          mma_ss(tmem_base + (n & 1) * 128, dq0 + offq, kb + offk, idS, kk > 0 ? 1u : 0u);
+          mma_ts(tmem_base + kTs, tmem_base + kTq + kk * 8, kb + offk, idS, kk > 0 ? 1u : 0u);
         }
-        return true;
+        mma_commit(s_full);
       };
-      // dP(n) = dO V_n^T once the previous dP has been read out; then signal S(n) + dP(n)
-      auto issue_dP = [&](int n) -> bool {
+      auto mma_dP = [&](int n) {  // dP(n) = dO V_n^T (A = dO from TMEM); then V_n is done
         const int seq = seq_base + 2 * n + 1;
-        if (dp_issued > 0) {
-          if (!mbar_wait(dp_free, (dp_issued - 1) & 1, abort_flag)) return false;
-          tc_fence_after();
-        }
-        if (!wait_tile(seq)) return false;
         const uint64_t vb = dk + (uint64_t)(((seq % S) * L::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t offq = ((kk / 4) * (kTile * 128) + (kk % 4) * 32) >> 4;
           const uint32_t offk = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
-          mma_ss(t_dp, ddo + offq, vb + offk, idS, kk > 0 ? 1u : 0u);
+          mma_ts(tmem_base + kTdp, tmem_base + kTdo + kk * 8, vb + offk, idS, kk > 0 ? 1u : 0u);
         }
-        ++dp_issued;
-        mma_commit(&kv_empty[seq % S]);  // V_n done
-        mma_commit(&s_full[n & 1]);
-        return true;
+        mma_commit(&kv_empty[seq % S]);
+        mma_commit(dp_full);
       };
       for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
         const int cnt = item_cnt(item);
         if (cnt == 0) continue;
-        if (!mbar_wait(q_full, qcons & 1, abort_flag)) { ok = false; break; }
-        ++qcons;
+        // Q, dO of the item in TMEM (the previous item's S / dP MMAs were issued before, and
+        // the elementwise warps copy them only after reading that item's last S / dP)
+        if (!mbar_wait(q_empty, items & 1, abort_flag)) { ok = false; break; }
+        ++items;
+        // S(0) into S once the previous step's S was read out; dP(0) into dP after the previous
+        // dQ (issue order)
+        if (gn > 0 && !mbar_wait(s_loaded, (gn - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        ok = issue_S(0) && issue_dP(0);
-        if (ok && cnt > 1) ok = issue_S(1);
-        for (int n = 0; n < cnt && ok; ++n) {
-          if (n + 1 < cnt) { ok = issue_dP(n + 1); if (!ok) break; }
-          // dQ += dS(n) K_n  (dS(n) sits in S buffer n & 1)
-          const int b = n & 1;
-          int& dsw = b ? dsw1 : dsw0;
-          if (!mbar_wait(&ds_full[b], dsw & 1, abort_flag)) { ok = false; break; }
-          ++dsw;
+        if (!wait_tile(seq_base) || !wait_tile(seq_base + 1)) { ok = false; break; }
+        mma_S(0);
+        mma_dP(0);
+        for (int n = 0; n < cnt && ok; ++n, ++gn) {
+          const bool more = n + 1 < cnt;
+          if (more) {  // S(n+1) once S(n) was read out
+            if (!mbar_wait(s_loaded, gn & 1, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            if (!wait_tile(seq_base + 2 * (n + 1))) { ok = false; break; }
+            mma_S(n + 1);
+            if (!wait_tile(seq_base + 2 * (n + 1) + 1)) { ok = false; break; }  // V_{n+1}, early
+          }
+          // dQ += dS(n) K_n (A = dS over the dP columns), then dP(n+1) into those columns
+          if (!mbar_wait(ds_full, gn & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const int kseq = seq_base + 2 * n;
           const uint64_t kb = dkmn + (uint64_t)(((kseq % S) * L::kKVBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BS / 16; ++kk)  // dS of keys [16kk, 16kk+16): group kk/2's columns
-            mma_ts(t_dq, tmem_base + b * 128 + 32 * (kk >> 1) + 8 * (kk & 1),
+            mma_ts(tmem_base + kTdq, tmem_base + kTdp + 32 * (kk >> 1) + 8 * (kk & 1),
                    kb + (uint64_t)((kk * 2048) >> 4), idQ, (n > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&kv_empty[kseq % S]);  // K_n done
-          if (n + 2 < cnt) { ok = issue_S(n + 2); if (!ok) break; }
+          if (more) mma_dP(n + 1);
         }
         if (!ok) break;
-        mma_commit(q_empty);
         mma_commit(dq_full);
         seq_base += 2 * cnt;
       }
@@ -814,12 +817,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
   } else if (warp < kBwdElem / 32) {
     // ====================================================== elementwise + epilogue
-    const int row = 32 * (warp % 4) + lane;  // query row of the 128-row tile
-    const int cg = warp / 4;                 // 32-column group (BS / 4 keys)
-    const uint32_t t_lane = (uint32_t)(32 * (warp % 4)) << 16;
-    const uint32_t t_dp = tmem_base + t_lane + 256, t_dq = tmem_base + t_lane + 384;
+    const int quarter = warp % 4;
+    const int row = 32 * quarter + lane;     // query row of the 128-row tile
+    const int cg = warp / 4;                 // 32-column group (BS / 4 keys, D / 4 dims)
+    const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
+    const uint32_t t_s = tmem_base + t_lane + kTs, t_dp = tmem_base + t_lane + kTdp;
+    const uint32_t t_dq = tmem_base + t_lane + kTdq;
     const float sl2 = g.scale * 1.4426950408889634f;
-    int sfc[2] = {0, 0}, dqc = 0;
+    constexpr int KC = BS / 4;
+    int qc = 0, gn = 0, dqc = 0;
     bool ok = true;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const int cnt = item_cnt(item);
@@ -833,6 +839,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         continue;
       }
+      // Q and dO rows of this thread (dims [D/4*cg, D/4*(cg+1))) from the 128-byte-swizzled
+      // staging tiles into TMEM as bf16 pairs: the A operands of S and dP
+      {
+        bool w_ok = mbar_wait(q_full, qc & 1, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) { ok = false; break; }
+        ++qc;
+        constexpr int DC = D / 4;         // dims of this group: DC / 8 chunks of 16 bytes
+        const int d0 = cg * DC, half = d0 / 64, c0 = (d0 % 64) / 8;
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          const unsigned char* tile = smem + (t ? L::kDOOff : L::kQOff) + half * (kTile * 128) + row * 128;
+          uint32_t w[DC / 2];
+#pragma unroll
+          for (int c = 0; c < DC / 8; ++c) {
+            const uint4 v = *reinterpret_cast<const uint4*>(tile + (((c0 + c) ^ (row & 7)) << 4));
+            w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+          }
+          const uint32_t dst = tmem_base + t_lane + (t ? kTdo : kTq) + cg * (DC / 2);
+          if constexpr (DC == 32) tmem_st16(dst, w);
+          else tmem_st8(dst, w);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(q_empty);  // staging free; Q, dO in TMEM
+      }
       const float nl2 = row < BS ? p.nlse2[qrow] : -INFINITY;  // -inf: pad row -> P = 0
       const float nd = row < BS ? p.ndelta[qrow] : 0.f;
       const uint64_t nl2x2 = f2pack(nl2, nl2), ndx2 = f2pack(nd, nd), sl2x2 = f2pack(sl2, sl2);
@@ -841,60 +873,60 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int jnext = lane < cnt ? item_idx(item, lane) : 0;
       int creg = 0;
       uint32_t partial = 0;
-      for (int n = 0; n < cnt; ++n) {
-        const int b = n & 1;
+      for (int n = 0; n < cnt; ++n, ++gn) {
         if ((n & 31) == 0) {
           const int jcur = jnext;
           jnext = n + 32 + lane < cnt ? item_idx(item, n + 32 + lane) : 0;
           creg = n + lane < cnt ? key_shape_code(g, jcur) : 0;
           partial = __ballot_sync(0xffffffffu, creg != 0);
         }
-        bool w_ok = mbar_wait(&s_full[b], sfc[b] & 1, abort_flag);
+        // P = exp2(S*sl2 - lse2) for this group's KC keys as soon as S(n) is in
+        bool w_ok = mbar_wait(s_full, gn & 1, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
         if (!w_ok) { ok = false; break; }
-        ++sfc[b];
         tc_fence_after();
-        // this group's BS/4 key columns of dP and S; release dP for dP(n+1) once read
-        constexpr int KC = BS / 4;
-        uint32_t dpr[KC], sr[KC], pk[KC / 2];
-        const uint32_t t_s = tmem_base + t_lane + b * 128;
-        if constexpr (KC == 32) {
-          tmem_ld32_wait(t_dp + cg * KC, dpr);
-          tmem_ld32_wait(t_s + cg * KC, sr);
-        } else {
-          tmem_ld16_wait(t_dp + cg * KC, dpr);
-          tmem_ld16_wait(t_s + cg * KC, sr);
-        }
+        float pf[KC];
+        tmem_ld32_wait(t_s + cg * KC, reinterpret_cast<uint32_t*>(pf));
         tc_fence_before();
-        mbar_arrive(dp_free);
-        // pad keys of a partial key block: S = -inf, so P = 0
-        if ((partial >> (n & 31)) & 1u) {
+        mbar_arrive(s_loaded);  // S may take S(n+1)
+        if ((partial >> (n & 31)) & 1u) {  // pad keys of a partial key block: P = 0
           const int code = __shfl_sync(0xffffffffu, creg, n & 31);
-          const uint32_t* mtab = reinterpret_cast<const uint32_t*>(smem + L::kMaskOff);
-          uint32_t word = mtab[code * (BS / 32) + (KC == 32 ? cg : 0)];
-          if (KC < 32) word >>= cg * KC;
+          const uint32_t word = reinterpret_cast<const uint32_t*>(smem + L::kMaskOff)[code * (BS / 32) + cg];
 #pragma unroll
           for (int c = 0; c < KC; ++c)
-            if (!((word >> c) & 1u)) sr[c] = __float_as_uint(-INFINITY);
+            if (!((word >> c) & 1u)) pf[c] = -INFINITY;
         }
 #pragma unroll
-        for (int e2 = 0; e2 < KC / 2; ++e2) {  // dS = P (dP - delta), two keys per f32x2 op
+        for (int e2 = 0; e2 < KC / 2; ++e2) {
           float x0, x1;
-          f2unpack(fma2(f2pack(__uint_as_float(sr[2 * e2]), __uint_as_float(sr[2 * e2 + 1])), sl2x2, nl2x2),
-                   x0, x1);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          const uint64_t dd = add2(f2pack(__uint_as_float(dpr[2 * e2]), __uint_as_float(dpr[2 * e2 + 1])), ndx2);
-          float s0, s1;
-          f2unpack(mul2(f2pack(p0, p1), dd), s0, s1);
-          pk[e2] = pack_bf16x2(s0, s1);
+          f2unpack(fma2(f2pack(pf[2 * e2], pf[2 * e2 + 1]), sl2x2, nl2x2), x0, x1);
+          pf[2 * e2] = fast_exp2(x0);
+          pf[2 * e2 + 1] = fast_exp2(x1);
         }
-        // dS (bf16) goes back over this group's own S columns: keys [KC*cg, KC*cg + KC) at
-        // columns [KC*cg, KC*cg + KC/2), so no other group's S is overwritten
-        static_assert(KC == 32, "the dQ pass runs with 128-key blocks");
-        tmem_st16(t_s + cg * KC, pk);
+        // dS = P (dP - delta) once dP(n) is in, back over this group's own dP columns as
+        // bf16 pairs (keys [KC*cg, KC*cg + KC) at columns [KC*cg, KC*cg + KC/2)), 16 at a time
+        w_ok = mbar_wait(dp_full, gn & 1, abort_flag);
+        w_ok = __all_sync(0xffffffffu, w_ok);
+        if (!w_ok) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int round = 0; round < 2; ++round) {
+          uint32_t dr[16], pk[8];
+          tmem_ld16_wait(t_dp + cg * KC + round * 16, dr);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int e2 = round * 8 + j;
+            float s0, s1;
+            f2unpack(mul2(f2pack(pf[2 * e2], pf[2 * e2 + 1]),
+                          add2(f2pack(__uint_as_float(dr[2 * j]), __uint_as_float(dr[2 * j + 1])), ndx2)),
+                     s0, s1);
+            pk[j] = pack_bf16x2(s0, s1);
+          }
+          tmem_st8(t_dp + cg * KC + round * 8, pk);
+        }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&ds_full[b]);
+        mbar_arrive(ds_full);  // dQ(n) may start
       }
       if (!ok) break;
       bool w_ok = mbar_wait(dq_full, dqc & 1, abort_flag);
@@ -913,8 +945,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
           for (int e2 = 0; e2 < DC / 2; ++e2)
             v32[e2] = (nl2 == -INFINITY) ? 0u
-                                       : pack_bf16x2(__uint_as_float(a[2 * e2]) * g.scale,
-                                                     __uint_as_float(a[2 * e2 + 1]) * g.scale);
+                                         : pack_bf16x2(__uint_as_float(a[2 * e2]) * g.scale,
+                                                       __uint_as_float(a[2 * e2 + 1]) * g.scale);
 #pragma unroll
           for (int e2 = 0; e2 < DC / 8; ++e2) reinterpret_cast<uint4*>(dq_row + cg * DC)[e2] = v[e2];
         }
