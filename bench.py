@@ -50,7 +50,7 @@ KERNEL_NAMES = {"fwd": "bsa_fwd_kernel", "bwd_dkdv": "bsa_bwd_dkdv_kernel",
 # selected block pair (fwd, dq) or a pair with a current key block (dkdv).  Traffic grows with
 # the pairs a launch processes, so a full launch is scaled from it.  None = not captured for
 # the kernel as it now stands.
-DRAM_BYTES_PER_PAIR = {"fwd": 3854, "bwd_dkdv": 5764, "bwd_dq": 4838}
+DRAM_BYTES_PER_PAIR = {"fwd": 3854, "bwd_dkdv": 5764, "bwd_dq": None}
 
 
 def traffic_per_launch(kernel, workload, n_pairs, n_pairs_cur):
@@ -308,7 +308,7 @@ def main():
     # compute (two device input sets; events order every reuse).
     pin = {k_: torch.from_numpy(x[k_].view(np.int16)).pin_memory() for k_ in ("q", "k", "v")}
     o_host = torch.empty(pipe.o.shape, dtype=torch.bfloat16).pin_memory()
-    e_steps = max(3, min(args.steps, 6))
+    e_steps = max(3, args.steps)  # as many as the timed steps; the first upload is pipeline fill
     sets = [{k_: torch.empty_like(q_d) for k_ in ("q", "k", "v")} for _ in range(2)]
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
