@@ -9,7 +9,9 @@ What it computes, with the page passages each step follows:
 * 3D RoPE and RMSNorm + QK-Norm -- "美团LongCat-Video揭秘：13.6B参数长视频生成模型如何终结画面漂移？"
   (xugj520.cn), section 三 "模型架构" (3D RoPE position encoding; RMSNorm + QKNorm); also
   "LongCat-Video : Generate 1 minute long AI videos with this model", section "How it
-  handles long videos" (3D attention with RoPE).
+  handles long videos" (3D attention with RoPE).  Their backward (gradients to the raster
+  q, k and the gains) follows from the same definitions; the talk's section 2.2 says the
+  module is used for training.
 * 3D blocks ("small 3D cubes"), block scores "by similarity", top-r selection --
   "LongCat-Video : Generate 1 minute long AI videos with this model", section "Sparse
   attention"; "LongCat-Video视频生成模型发布 迈出世界模型探索第一步" (youleyou.com), section
@@ -210,6 +212,58 @@ def prologue(x: np.ndarray, frames: int, grid_h: int, grid_w: int, *,
         t, h, w = grid_positions(frames, grid_h, grid_w, t_offset)
         y = rope3d(y, t, h, w, theta)
     return y
+
+
+def rope3d_transpose(dz: np.ndarray, t_pos: np.ndarray, h_pos: np.ndarray, w_pos: np.ndarray,
+                     theta: float) -> np.ndarray:
+    """Gradient of rope3d with respect to its input: each pair was turned by R(a), so the
+    upstream gradient is turned back by R(a)^T (pair (e, o): e' = e cos a + o sin a,
+    o' = -e sin a + o cos a), with the same angles as the forward."""
+    dz = np.asarray(dz, dtype=np.float64)
+    d = dz.shape[-1]
+    dt, dh, dw = rope_split(d)
+    ang = np.concatenate([rope_angles(t_pos, dt, theta), rope_angles(h_pos, dh, theta),
+                          rope_angles(w_pos, dw, theta)], axis=1)
+    c = np.cos(ang)[:, None, :]
+    s = np.sin(ang)[:, None, :]
+    ze, zo = dz[..., 0::2], dz[..., 1::2]
+    dy = np.empty_like(dz)
+    dy[..., 0::2] = ze * c + zo * s
+    dy[..., 1::2] = -ze * s + zo * c
+    return dy
+
+
+def rms_norm_bwd(dy: np.ndarray, x: np.ndarray, gamma: np.ndarray, eps: float):
+    """Gradients of y = x / r * gamma, r = sqrt(mean(x^2) + eps), over the last axis.
+
+    With xh = x / r: d gamma = sum over every leading index of dy * xh; d xh = dy * gamma;
+    dx = (d xh - xh * mean(d xh * xh)) / r (r depends on x through mean(x^2)).
+    Returns (dx, dgamma)."""
+    x = np.asarray(x, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    gamma = np.asarray(gamma, dtype=np.float64)
+    r = np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    xh = x / r
+    dgamma = np.sum((dy * xh).reshape(-1, x.shape[-1]), axis=0)
+    dxh = dy * gamma
+    dx = (dxh - xh * np.mean(dxh * xh, axis=-1, keepdims=True)) / r
+    return dx, dgamma
+
+
+def prologue_bwd(dz: np.ndarray, x: np.ndarray, frames: int, grid_h: int, grid_w: int, *,
+                 gamma: Optional[np.ndarray], eps: float = 1e-6, theta: float = 0.0,
+                 t_offset: int = 0):
+    """Backward of ``prologue``: dz is the gradient of its output (raster [B, N, H, D]), x its
+    raster input.  The steps of the forward are undone in reverse order: RoPE (turn back by
+    the transposed rotation), then RMSNorm.  Returns (dx, dgamma); dgamma is None when the
+    forward had no gain."""
+    dy = np.asarray(dz, dtype=np.float64)
+    if theta:
+        t, h, w = grid_positions(frames, grid_h, grid_w, t_offset)
+        dy = rope3d_transpose(dy, t, h, w, theta)
+    if gamma is None:
+        return dy, None
+    return rms_norm_bwd(dy, x, gamma, eps)
 
 
 # ----------------------------------------------------------------------------------------

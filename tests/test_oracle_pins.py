@@ -451,3 +451,57 @@ def test_bwd_continuation_grads_only_reach_current_keys():
     np.testing.assert_allclose(dq, tq.grad.numpy().transpose(0, 2, 1, 3)[:, nc:], atol=1e-11)
     np.testing.assert_allclose(dk, tk.grad.numpy().transpose(0, 2, 1, 3)[:, nc:], atol=1e-11)
     np.testing.assert_allclose(dv, tv.grad.numpy().transpose(0, 2, 1, 3)[:, nc:], atol=1e-11)
+
+
+# ------------------------------------------------------------------ prologue backward
+def _prologue_case(seed=5, frames=2, gh=3, gw=5, heads=2, d=12):
+    rng = np.random.default_rng(seed)
+    x = rng.standard_normal((1, frames * gh * gw, heads, d))
+    gamma = 1.0 + 0.5 * rng.standard_normal(d)
+    dz = rng.standard_normal(x.shape)
+    return rng, x, gamma, dz
+
+
+def test_prologue_bwd_finite_differences():
+    """dx and dgamma against central differences of sum(dz * prologue(x; gamma))."""
+    rng, x, gamma, dz = _prologue_case()
+    kw = dict(eps=1e-6, theta=10.0, t_offset=3)
+    dx, dgamma = oracle.prologue_bwd(dz, x, 2, 3, 5, gamma=gamma, **kw)
+
+    def loss(xx, gg):
+        return float(np.sum(dz * oracle.prologue(xx, 2, 3, 5, gamma=gg, **kw)))
+    h = 1e-6
+    for _ in range(16):
+        pos = tuple(int(rng.integers(0, s)) for s in x.shape)
+        xp, xm = x.copy(), x.copy()
+        xp[pos] += h
+        xm[pos] -= h
+        assert dx[pos] == pytest.approx((loss(xp, gamma) - loss(xm, gamma)) / (2 * h), rel=1e-6, abs=1e-8)
+    for dd in range(x.shape[-1]):
+        gp, gm = gamma.copy(), gamma.copy()
+        gp[dd] += h
+        gm[dd] -= h
+        assert dgamma[dd] == pytest.approx((loss(x, gp) - loss(x, gm)) / (2 * h), rel=1e-6, abs=1e-8)
+
+
+def test_rope_transpose_undoes_the_rotation():
+    """RoPE turns each pair by an angle, so its transpose is its inverse: rotating the
+    transposed gradient forward gives it back, and pair norms are kept."""
+    _, _, _, dz = _prologue_case(seed=8)
+    t, h, w = oracle.grid_positions(2, 3, 5, t_offset=1)
+    dy = oracle.rope3d_transpose(dz, t, h, w, 10000.0)
+    np.testing.assert_allclose(oracle.rope3d(dy, t, h, w, 10000.0), dz, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dy[..., 0::2] ** 2 + dy[..., 1::2] ** 2,
+                               dz[..., 0::2] ** 2 + dz[..., 1::2] ** 2, rtol=1e-12, atol=1e-12)
+
+
+def test_rmsnorm_bwd_is_orthogonal_to_the_input_without_eps():
+    """With eps = 0 the normalised output does not change when x is scaled, so the gradient
+    of any loss through it is orthogonal to x, row by row."""
+    _, x, gamma, dz = _prologue_case(seed=9)
+    dx, _ = oracle.rms_norm_bwd(dz, x, gamma, 0.0)
+    np.testing.assert_allclose(np.sum(dx * x, axis=-1), 0.0, atol=1e-12)
+    # and without a gain and without RoPE the prologue backward is the plain identity
+    dx2, dg2 = oracle.prologue_bwd(dz, x, 2, 3, 5, gamma=None, theta=0.0)
+    assert dg2 is None
+    np.testing.assert_array_equal(dx2, dz)
