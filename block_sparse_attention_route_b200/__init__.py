@@ -18,13 +18,14 @@ from typing import Optional
 __all__ = [
     "Geometry", "BsaError", "lib", "bsa_workspace_size", "rope3d_qknorm_prologue", "bsa_route",
     "bsa_attn_fwd", "bsa_attn_bwd", "bsa_device_status", "bsa_error_string", "blocked_shape",
-    "bsa_selftest_bounded_wait", "bsa_route_noalloc",
-    "WS_ROUTE", "WS_FWD", "WS_BWD",
+    "bsa_selftest_bounded_wait", "bsa_route_noalloc", "rope3d_qknorm_prologue_bwd",
+    "bsa_kernel_timing", "bsa_kernel_times",
+    "WS_ROUTE", "WS_FWD", "WS_BWD", "WS_PROLOGUE_BWD",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbsa.so")
-WS_ROUTE, WS_FWD, WS_BWD = 1, 2, 3
+WS_ROUTE, WS_FWD, WS_BWD, WS_PROLOGUE_BWD = 1, 2, 3, 4
 STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_CUDA",
           4: "BSA_ERR_TIMEOUT", 5: "BSA_ERR_BAD_INDEX", 6: "BSA_ERR_WORKSPACE"}
 
@@ -110,6 +111,8 @@ def lib() -> ctypes.CDLL:
             "bsa_abi_version": (I32, []),
             "bsa_workspace_size": (S, [G, I32, I32]),
             "rope3d_qknorm_prologue": (I32, [G, I32, I32, P, P, P, P, P, F, F, P, P, P, P, P, P]),
+            "rope3d_qknorm_prologue_bwd": (I32, [G, I32, I32, P, P, P, P, F, F, P, P, P, P, P, P,
+                                                 P, P, P, S, P]),
             "bsa_route": (I32, [G, I32, P, P, P, P, P, P, P, P, S, P]),
             "bsa_attn_fwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P]),
             "bsa_attn_bwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
@@ -173,6 +176,16 @@ def rope3d_qknorm_prologue(g: Geometry, frames: int, t_offset: int, q, k, v, gam
         ctypes.byref(g.c()), frames, t_offset, _ptr(q), _ptr(k), _ptr(v), _ptr(gamma_q),
         _ptr(gamma_k), eps, rope_theta, _ptr(q_blk), _ptr(k_blk), _ptr(v_blk), _ptr(q_pool),
         _ptr(k_pool), _stream(stream)), "rope3d_qknorm_prologue")
+
+
+def rope3d_qknorm_prologue_bwd(g: Geometry, frames: int, t_offset: int, q, k, gamma_q, gamma_k,
+                               eps: float, rope_theta: float, dq_blk, dk_blk, dv_blk, dq, dk, dv,
+                               dgamma_q=None, dgamma_k=None, ws=None, stream=None):
+    _check(lib().rope3d_qknorm_prologue_bwd(
+        ctypes.byref(g.c()), frames, t_offset, _ptr(q), _ptr(k), _ptr(gamma_q), _ptr(gamma_k),
+        eps, rope_theta, _ptr(dq_blk), _ptr(dk_blk), _ptr(dv_blk), _ptr(dq), _ptr(dk), _ptr(dv),
+        _ptr(dgamma_q), _ptr(dgamma_k), _ptr(ws), _nbytes(ws) if ws is not None else 0,
+        _stream(stream)), "rope3d_qknorm_prologue_bwd")
 
 
 def bsa_route(g: Geometry, top_r: int, q_blk, k_blk, q_pool, k_pool, kpool_cache, idx, cnt,

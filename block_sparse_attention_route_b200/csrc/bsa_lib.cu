@@ -214,6 +214,8 @@ size_t bsa_workspace_size(const bsa_geom_t* gi, int32_t top_r, int32_t which) {
   if (which == BSA_WS_ROUTE) return route_ws(g).total;
   if (which == BSA_WS_FWD) return 0;
   if (which == BSA_WS_BWD) return bwd_ws_layout(g, top_r).total;
+  if (which == BSA_WS_PROLOGUE_BWD)
+    return 2 * align256((size_t)prologue_bwd_ctas(g, (g.T + g.bt - 1) / g.bt) * g.D * sizeof(float));
   return 0;
 }
 
@@ -270,6 +272,82 @@ bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* gi, int32_t frames, int32_
   a.dt = g.D - 2 * a.dh;
   cudaError_t e = launch_prologue(a, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "prologue launch");
+  return BSA_OK;
+}
+
+bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
+                                        const void* q_raster, const void* k_raster,
+                                        const float* gamma_q, const float* gamma_k, float eps,
+                                        float rope_theta, const void* dq_blk, const void* dk_blk,
+                                        const void* dv_blk, void* dq, void* dk, void* dv,
+                                        float* dgamma_q, float* dgamma_k, void* ws, size_t ws_bytes,
+                                        bsa_stream_t stream) {
+  t_detail.clear();
+  Geo g;
+  bsa_status_t st = make_geo(gi, &g);
+  if (st != BSA_OK) return st;
+  if (frames < 1) return fail(BSA_ERR_INVALID_ARG, "frames must be >= 1");
+  if (t_offset < 0) return fail(BSA_ERR_INVALID_ARG, "t_offset must be >= 0");
+  if (!(eps >= 0.f) || !(rope_theta >= 0.f) || std::isinf(rope_theta))
+    return fail(BSA_ERR_INVALID_ARG, "eps and rope_theta must be finite and >= 0");
+  const void* dz[3] = {dq_blk, dk_blk, dv_blk};
+  void* dxs[3] = {dq, dk, dv};
+  const void* xs[2] = {q_raster, k_raster};
+  const float* gams[2] = {gamma_q, gamma_k};
+  float* dgs[2] = {dgamma_q, dgamma_k};
+  bool any = false, any_gain = false;
+  for (int i = 0; i < 3; ++i) {
+    if ((dz[i] == nullptr) != (dxs[i] == nullptr))
+      return fail(BSA_ERR_INVALID_ARG, "gradient %d and its output must both be given or both NULL", i);
+    if (dz[i] && (!aligned(dz[i], 16) || !aligned(dxs[i], 16)))
+      return fail(BSA_ERR_INVALID_ARG, "tensor %d not 16-byte aligned", i);
+    any |= dz[i] != nullptr;
+  }
+  if (!any) return fail(BSA_ERR_INVALID_ARG, "no tensor to process");
+  for (int i = 0; i < 2; ++i) {
+    if (dz[i] && gams[i]) {
+      if (!xs[i] || !dgs[i])
+        return fail(BSA_ERR_INVALID_ARG, "with a gain, tensor %d needs its raster input and a dgamma output", i);
+      if (!aligned(xs[i], 16)) return fail(BSA_ERR_INVALID_ARG, "raster input %d not 16-byte aligned", i);
+      any_gain = true;
+    }
+  }
+  if (((long)frames * g.GH * g.GW) * (long)g.B * g.H * g.D >= (1L << 40))
+    return fail(BSA_ERR_UNSUPPORTED, "tensor too large");
+  const int nbt = (frames + g.bt - 1) / g.bt;
+  const size_t part_bytes = align256((size_t)prologue_bwd_ctas(g, nbt) * g.D * sizeof(float));
+  if (any_gain && (ws == nullptr || ws_bytes < 2 * part_bytes || !aligned(ws, 256)))
+    return fail(BSA_ERR_WORKSPACE, "prologue backward needs %zu workspace bytes (256-byte aligned)",
+                2 * part_bytes);
+  st = check_device(nullptr);
+  if (st != BSA_OK) return st;
+  PrologueBwdArgs a;
+  PrologueArgs& f = a.f;
+  f.g = g;
+  f.frames = frames;
+  f.t_offset = t_offset;
+  f.nbt = nbt;
+  for (int i = 0; i < 3; ++i) { f.x[i] = nullptr; f.y[i] = nullptr; }
+  f.gamma[0] = dq_blk ? gamma_q : nullptr;
+  f.gamma[1] = dk_blk ? gamma_k : nullptr;
+  f.pool[0] = f.pool[1] = nullptr;
+  f.eps = eps;
+  f.theta = rope_theta;
+  f.dh = 2 * (g.D / 6);
+  f.dw = f.dh;
+  f.dt = g.D - 2 * f.dh;
+  for (int i = 0; i < 3; ++i) {
+    a.dz[i] = static_cast<const __nv_bfloat16*>(dz[i]);
+    a.dx[i] = static_cast<__nv_bfloat16*>(dxs[i]);
+  }
+  for (int i = 0; i < 2; ++i) {
+    a.x[i] = static_cast<const __nv_bfloat16*>(xs[i]);
+    a.part[i] = (dz[i] && gams[i]) ? reinterpret_cast<float*>(static_cast<char*>(ws) + i * part_bytes)
+                                   : nullptr;
+    if (!(dz[i] && gams[i])) dgs[i] = nullptr;
+  }
+  cudaError_t e = launch_prologue_bwd(a, dgs, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "prologue backward launch");
   return BSA_OK;
 }
 

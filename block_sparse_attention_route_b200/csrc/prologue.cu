@@ -29,6 +29,28 @@ struct PrologueArgs {
 constexpr int kPrologueThreads = 256;
 constexpr int kHeadsPerCta = 8;
 
+// cos/sin of every RoPE angle a block needs, in fp64 then rounded: axis t rows [0, bt), h
+// rows after, w rows last; each row holds that axis' pairs (pos * theta^(-2i/width)).
+__device__ void build_rope_table(const PrologueArgs& a, int ibt, int ibh, int ibw, float2* tab) {
+  const Geo& g = a.g;
+  const int pt = a.dt / 2, ph = a.dh / 2, pw = a.dw / 2;
+  const int off_h = g.bt * pt, off_w = off_h + g.bh * ph, ntab = off_w + g.bw * pw;
+  for (int e = threadIdx.x; e < ntab; e += blockDim.x) {
+    int pos, i, width;
+    if (e < off_h) {
+      pos = a.t_offset + ibt * g.bt + e / pt; i = e % pt; width = a.dt;
+    } else if (e < off_w) {
+      int r = e - off_h; pos = ibh * g.bh + r / ph; i = r % ph; width = a.dh;
+    } else {
+      int r = e - off_w; pos = ibw * g.bw + r / pw; i = r % pw; width = a.dw;
+    }
+    double ang = (double)pos * pow((double)a.theta, -2.0 * (double)i / (double)width);
+    double s, c;
+    sincos(ang, &s, &c);
+    tab[e] = make_float2((float)c, (float)s);
+  }
+}
+
 template <int D>
 __global__ void __launch_bounds__(kPrologueThreads)
     prologue_kernel(const PrologueArgs a) {
@@ -51,23 +73,8 @@ __global__ void __launch_bounds__(kPrologueThreads)
   // ---- cos/sin table: axis t rows [0,bt), h rows [bt, bt+bh), w rows after; each row
   //      holds that axis' pairs.
   const int pt = a.dt / 2, ph = a.dh / 2, pw = a.dw / 2;
-  const int off_h = g.bt * pt, off_w = off_h + g.bh * ph, ntab = off_w + g.bw * pw;
-  if (rope) {
-    for (int e = tid; e < ntab; e += kPrologueThreads) {
-      int pos, i, width;
-      if (e < off_h) {
-        pos = a.t_offset + ibt * g.bt + e / pt; i = e % pt; width = a.dt;
-      } else if (e < off_w) {
-        int r = e - off_h; pos = ibh * g.bh + r / ph; i = r % ph; width = a.dh;
-      } else {
-        int r = e - off_w; pos = ibw * g.bw + r / pw; i = r % pw; width = a.dw;
-      }
-      double ang = (double)pos * pow((double)a.theta, -2.0 * (double)i / (double)width);
-      double s, c;
-      sincos(ang, &s, &c);
-      tab[e] = make_float2((float)c, (float)s);
-    }
-  }
+  const int off_h = g.bt * pt, off_w = off_h + g.bh * ph;
+  if (rope) build_rope_table(a, ibt, ibh, ibw, tab);
   for (int e = tid; e < 2 * kHeadsPerCta * D; e += kPrologueThreads) pool_s[e] = 0.f;
   __syncthreads();
 
@@ -212,6 +219,196 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s) {
     prologue_kernel<64><<<grid, kPrologueThreads, smem, s>>>(a);
   }
   return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------------------ backward
+// Gradients of the prologue: dz (blocked, bf16) -> dx (raster, bf16) and, for q and k with a
+// gain, dgamma.  Per (token, head) row, undoing the forward in reverse order:
+//   RoPE:    dy = R(a)^T dz per pair (turned back by the forward angle);
+//   RMSNorm: xh = x / r, r = sqrt(mean(x^2) + eps); dgamma += dy * xh;
+//            dxh = dy * gamma; dx = (dxh - xh * mean(dxh * xh)) / r.
+// v (and q / k without a gain and RoPE) is the inverse relayout.  Same tiling as the forward
+// (one CTA per block of the padded grid and 8 heads); each thread keeps the dgamma partials
+// of its 8 columns over its rows, the CTA sums them in shared memory and writes one partial
+// row per CTA, and prologue_dgamma_kernel adds the partial rows in a fixed order, so dgamma
+// is deterministic.
+struct PrologueBwdArgs {
+  PrologueArgs f;                 // geometry, RoPE widths, frames, t_offset, gamma, eps, theta
+  const __nv_bfloat16* dz[3];     // blocked gradients of the outputs (NULL = skip)
+  const __nv_bfloat16* x[2];      // raster forward inputs q, k (needed with a gain)
+  __nv_bfloat16* dx[3];           // raster gradients of the inputs
+  float* part[2];                 // [n_cta][D] dgamma partials of q, k
+};
+
+template <int D>
+__global__ void __launch_bounds__(kPrologueThreads)
+    prologue_bwd_kernel(const PrologueBwdArgs a) {
+  constexpr int LPR = D / 8;                     // lanes per row
+  constexpr int RPP = kPrologueThreads / LPR;    // rows per pass
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  float* gsum = reinterpret_cast<float*>(smem_raw);            // [2][D]
+  float2* tab = reinterpret_cast<float2*>(gsum + 2 * D);
+
+  const PrologueArgs& f = a.f;
+  const Geo& g = f.g;
+  const int blk = blockIdx.x, hg = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x;
+  const int per_t = g.nbh * g.nbw;
+  const int ibt = blk / per_t, ibh = (blk % per_t) / g.nbw, ibw = blk % g.nbw;
+  int vt, vh, vw;
+  block_extent(g, f.frames, blk, vt, vh, vw);
+  const bool rope = f.theta > 0.f;
+  const int pt = f.dt / 2, ph = f.dh / 2;
+  const int off_h = g.bt * pt, off_w = off_h + g.bh * ph;
+  if (rope) build_rope_table(f, ibt, ibh, ibw, tab);
+  for (int e = tid; e < 2 * D; e += kPrologueThreads) gsum[e] = 0.f;
+  __syncthreads();
+
+  const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
+  const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
+  const int rows = kHeadsPerCta * g.BS;
+  const size_t n_raster = (size_t)f.frames * g.GH * g.GW;
+  int ax[4], pi[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int pp = c0 / 2 + q;
+    if (2 * pp < f.dt) { ax[q] = 0; pi[q] = pp; }
+    else if (2 * pp < f.dt + f.dh) { ax[q] = 1; pi[q] = pp - pt; }
+    else { ax[q] = 2; pi[q] = pp - pt - ph; }
+  }
+  for (int which = 0; which < 3; ++which) {
+    const __nv_bfloat16* __restrict__ dz = a.dz[which];
+    __nv_bfloat16* __restrict__ dx = a.dx[which];
+    if (dz == nullptr) continue;
+    const bool qk = which < 2;
+    const float* gam = qk ? f.gamma[which] : nullptr;
+    const __nv_bfloat16* __restrict__ xin = qk ? a.x[which] : nullptr;
+    const bool do_rope = qk && rope;
+    float gv[8], gacc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { gv[e] = gam ? gam[c0 + e] : 1.f; gacc[e] = 0.f; }
+    for (int base = 0; base < rows; base += RPP) {
+      const int row = base + rid;
+      const int hl = row % kHeadsPerCta, slot = row / kHeadsPerCta;
+      const int h = hg * kHeadsPerCta + hl;
+      const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
+      const bool valid = row < rows && hl < heads_here && lt < vt && lh < vh && lw < vw;
+      float v[8], xv[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { v[e] = 0.f; xv[e] = 0.f; }
+      size_t xoff = 0;
+      if (valid) {
+        const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
+        const size_t n = ((size_t)t * g.GH + hh) * g.GW + ww;
+        xoff = (((size_t)b * n_raster + n) * g.H + h) * D + c0;
+        const uint4 rz = __ldg(reinterpret_cast<const uint4*>(
+            dz + ((((size_t)b * g.H + h) * (size_t)(f.nbt * per_t) + blk) * g.BS + slot) * D + c0));
+        const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rz);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 ff = __bfloat1622float2(p2[e]);
+          v[2 * e] = ff.x; v[2 * e + 1] = ff.y;
+        }
+        if (gam) {
+          const uint4 rx = __ldg(reinterpret_cast<const uint4*>(xin + xoff));
+          const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&rx);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 ff = __bfloat1622float2(x2[e]);
+            xv[2 * e] = ff.x; xv[2 * e + 1] = ff.y;
+          }
+        }
+      }
+      if (do_rope && valid) {  // dy = R(a)^T dz
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float2 cs;
+          if (ax[q] == 0) cs = tab[lt * pt + pi[q]];
+          else if (ax[q] == 1) cs = tab[off_h + lh * ph + pi[q]];
+          else cs = tab[off_w + lw * (f.dw / 2) + pi[q]];
+          const float z0 = v[2 * q], z1 = v[2 * q + 1];
+          v[2 * q] = z0 * cs.x + z1 * cs.y;
+          v[2 * q + 1] = -z0 * cs.y + z1 * cs.x;
+        }
+      }
+      if (gam) {  // RMSNorm backward; every lane takes part in the shuffles
+        float ss = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(xv[e], xv[e], ss);
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+        const float rs = rsqrtf(ss * (1.0f / D) + f.eps);  // 1 / r
+        float dot = 0.f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float xh = xv[e] * rs;
+          gacc[e] = fmaf(v[e], xh, gacc[e]);   // dgamma (pad rows add 0)
+          v[e] *= gv[e];                        // d xh
+          dot = fmaf(v[e], xh, dot);
+        }
+#pragma unroll
+        for (int o = LPR / 2; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        const float mdot = dot * (1.0f / D);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = (v[e] - xv[e] * rs * mdot) * rs;
+      }
+      if (valid) {
+        uint4 outv;
+        uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) o32[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
+        *reinterpret_cast<uint4*>(dx + xoff) = outv;
+      }
+    }
+    if (gam && a.part[which] != nullptr) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) atomicAdd(&gsum[which * D + c0 + e], gacc[e]);
+    }
+  }
+  __syncthreads();
+  const size_t cta = ((size_t)b * gridDim.y + hg) * gridDim.x + blk;
+  for (int which = 0; which < 2; ++which) {
+    if (a.part[which] == nullptr || a.dz[which] == nullptr || f.gamma[which] == nullptr) continue;
+    for (int e = tid; e < D; e += kPrologueThreads) a.part[which][cta * D + e] = gsum[which * D + e];
+  }
+}
+
+// dgamma[d] = sum over the CTAs' partial rows, in CTA order (deterministic).
+__global__ void __launch_bounds__(256) prologue_dgamma_kernel(const float* __restrict__ part,
+                                                              int n_cta, int d, float* __restrict__ out) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= d) return;
+  float s = 0.f;
+  for (int c = 0; c < n_cta; ++c) s += part[(size_t)c * d + e];
+  out[e] = s;
+}
+
+int prologue_bwd_ctas(const Geo& g, int nbt) {
+  return nbt * g.nbh * g.nbw * ((g.H + kHeadsPerCta - 1) / kHeadsPerCta) * g.B;
+}
+
+cudaError_t launch_prologue_bwd(const PrologueBwdArgs& a, float* dgamma[2], cudaStream_t s) {
+  const Geo& g = a.f.g;
+  dim3 grid(a.f.nbt * g.nbh * g.nbw, (g.H + kHeadsPerCta - 1) / kHeadsPerCta, g.B);
+  const size_t smem = (size_t)2 * g.D * sizeof(float) +
+                      (size_t)(g.bt * (a.f.dt / 2) + g.bh * (a.f.dh / 2) + g.bw * (a.f.dw / 2)) * sizeof(float2);
+  if (g.D == 128) {
+    cudaFuncSetAttribute(prologue_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    prologue_bwd_kernel<128><<<grid, kPrologueThreads, smem, s>>>(a);
+  } else {
+    cudaFuncSetAttribute(prologue_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    prologue_bwd_kernel<64><<<grid, kPrologueThreads, smem, s>>>(a);
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const int n_cta = (int)(grid.x * grid.y * grid.z);
+  for (int w = 0; w < 2; ++w) {
+    if (dgamma[w] == nullptr || a.part[w] == nullptr) continue;
+    prologue_dgamma_kernel<<<(g.D + 255) / 256, 256, 0, s>>>(a.part[w], n_cta, g.D, dgamma[w]);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace bsa

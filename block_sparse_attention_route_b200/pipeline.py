@@ -9,8 +9,9 @@ from typing import Dict, Optional
 
 import torch
 
-from . import (WS_BWD, WS_ROUTE, Geometry, blocked_shape, bsa_attn_bwd, bsa_attn_fwd,
-               bsa_route, bsa_workspace_size, rope3d_qknorm_prologue)
+from . import (WS_BWD, WS_PROLOGUE_BWD, WS_ROUTE, Geometry, blocked_shape, bsa_attn_bwd,
+               bsa_attn_fwd, bsa_route, bsa_workspace_size, rope3d_qknorm_prologue,
+               rope3d_qknorm_prologue_bwd)
 
 
 class BsaPipeline:
@@ -46,6 +47,7 @@ class BsaPipeline:
             self.vc = torch.empty(cshp, **bf)
             self.kc_pool = torch.empty(cshp[:3] + (g.head_dim,), dtype=torch.float32, device=dev)
         self.gamma_q = self.gamma_k = None
+        self.ws_pro_bwd = None
         if with_bwd:
             self.do = torch.empty(shp, **bf)
             self.dq = torch.empty(shp, **bf)
@@ -98,3 +100,19 @@ class BsaPipeline:
                      self.lse, self.do, self.idx, self.cnt, self.dq, self.dk, self.dv,
                      self.ws_bwd, stream=stream)
         return {"dq": self.dq, "dk": self.dk, "dv": self.dv}
+
+    def prologue_backward(self, q_raster, k_raster, dq_raster, dk_raster, dv_raster,
+                          dgamma_q=None, dgamma_k=None, stream=None):
+        """Gradients of the raster q, k, v (and of the gains) from the blocked dq, dk, dv of
+        backward(); q_raster / k_raster are the inputs the forward prologue was given."""
+        g = self.g
+        if self.ws_pro_bwd is None:
+            self.ws_pro_bwd = torch.empty(max(bsa_workspace_size(g, 1, WS_PROLOGUE_BWD), 256),
+                                          dtype=torch.uint8, device=self.dq.device)
+        gq = self.gamma_q if self.qknorm else None
+        gk = self.gamma_k if self.qknorm else None
+        rope3d_qknorm_prologue_bwd(g, g.t_frames, g.cached_t, q_raster, k_raster, gq, gk,
+                                   self.eps, self.theta, self.dq, self.dk, self.dv, dq_raster,
+                                   dk_raster, dv_raster, dgamma_q if gq is not None else None,
+                                   dgamma_k if gk is not None else None, self.ws_pro_bwd,
+                                   stream=stream)

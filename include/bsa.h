@@ -87,7 +87,7 @@ typedef struct bsa_geom {
   float softmax_scale;    /* logits = q.k * scale; 0 selects 1/sqrt(head_dim) */
 } bsa_geom_t;
 
-enum { BSA_WS_ROUTE = 1, BSA_WS_FWD = 2, BSA_WS_BWD = 3 };
+enum { BSA_WS_ROUTE = 1, BSA_WS_FWD = 2, BSA_WS_BWD = 3, BSA_WS_PROLOGUE_BWD = 4 };
 
 /* ABI version of the loaded library (BSA_ABI_VERSION). */
 BSA_API int32_t bsa_abi_version(void);
@@ -95,7 +95,9 @@ BSA_API int32_t bsa_abi_version(void);
 /* Bytes of workspace `which` (BSA_WS_*) needs for this geometry; 0 on invalid arguments.
  * Workspace must be 256-byte aligned.  ROUTE: pooled q/k means.  FWD: none (returns 0).
  * BWD: per query row -Delta (Delta = rowsum(dO*O)) and -LSE*log2(e), the key-block ->
- * query-block index and a work counter of the dK/dV pass. */
+ * query-block index and a work counter of the dK/dV pass.  PROLOGUE_BWD: fp32 partial sums of
+ * d gamma_q and d gamma_k, one D-row per CTA of the prologue backward over g->t_frames frames
+ * (top_r is ignored). */
 BSA_API size_t bsa_workspace_size(const bsa_geom_t* g, int32_t top_r, int32_t which);
 
 /* Fused QK-RMSNorm + 3D RoPE prologue and raster -> blocked relayout.
@@ -118,6 +120,28 @@ BSA_API bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* g, int32_t frames,
                                     const float* gamma_k, float eps, float rope_theta,
                                     void* q_blk, void* k_blk, void* v_blk, float* q_pool,
                                     float* k_pool, bsa_stream_t stream);
+
+/* Backward of rope3d_qknorm_prologue over the same `frames`, t_offset, gamma, eps and
+ * rope_theta.  Same source; the talk "LongCat-Video 高效長視頻生成探索世界模型的第壹步",
+ * section 2.2, has the sparse-attention module trained, which needs these gradients.
+ * Given dq_blk / dk_blk / dv_blk, the gradients of the blocked outputs (bf16, pad slots
+ * ignored), writes the gradients of the raster inputs dq / dk / dv (bf16 [B, frames*gh*gw,
+ * H, D]) and, for q / k processed with a gain, dgamma_q / dgamma_k (fp32 [D], overwritten).
+ * Per (token, head): dy = RoPE^T(dz) (each pair turned back by its forward angle); with a
+ * gain, xh = x / r, r = sqrt(mean_d(x^2) + eps), dgamma += dy * xh (summed over tokens and
+ * heads), dx = (dy*gamma - xh * mean_d(dy*gamma*xh)) / r; without one dx = dy.  v: inverse
+ * relayout.  q / k (the forward's raster inputs) are needed where a gain is given.  Each of
+ * dq_blk / dk_blk / dv_blk may be NULL (then its output must be NULL too).  ws: 256-byte
+ * aligned, bsa_workspace_size(g, 1, BSA_WS_PROLOGUE_BWD) bytes when a gain is given, else
+ * may be NULL.  dgamma is reduced in a fixed order (deterministic). */
+BSA_API bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* g, int32_t frames, int32_t t_offset,
+                                                const void* q_raster, const void* k_raster,
+                                                const float* gamma_q, const float* gamma_k,
+                                                float eps, float rope_theta, const void* dq_blk,
+                                                const void* dk_blk, const void* dv_blk, void* dq,
+                                                void* dk, void* dv, float* dgamma_q,
+                                                float* dgamma_k, void* ws, size_t ws_bytes,
+                                                bsa_stream_t stream);
 
 /* Block-pooled top-r routing.
  * Sources: "LongCat-Video : Generate 1 minute long AI videos with this model", section

@@ -96,3 +96,20 @@ def test_kernel_timing_bookkeeping_without_launches():
     assert bsa.bsa_kernel_times() == {k: (0, 0.0) for k in bsa.TIMED_KERNELS}
     bsa.bsa_kernel_timing(False)
     assert bsa.bsa_kernel_times() == {k: (0, 0.0) for k in bsa.TIMED_KERNELS}
+
+
+def test_prologue_bwd_host_validation():
+    g = _g()
+    assert bsa.bsa_workspace_size(g, 1, bsa.WS_PROLOGUE_BWD) == 2 * (-(-(720 * 4 * 128 * 4) // 256) * 256)
+    with pytest.raises(bsa.BsaError) as ei:  # nothing to process
+        bsa.rope3d_qknorm_prologue_bwd(g, 24, 0, None, None, None, None, 1e-6, 1e4,
+                                       None, None, None, None, None, None, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # a gradient without its output
+        bsa.rope3d_qknorm_prologue_bwd(g, 24, 0, None, None, None, None, 1e-6, 1e4,
+                                       16, None, None, None, None, None, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # a gain needs the raster input and a dgamma output
+        bsa.rope3d_qknorm_prologue_bwd(g, 24, 0, None, None, 16, None, 1e-6, 1e4,
+                                       16, None, None, 16, None, None, stream=0)
+    assert ei.value.code == 1
