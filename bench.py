@@ -360,6 +360,30 @@ def main():
     h2d = sum(pin[k_].numel() * 2 for k_ in pin)
     d2h = o_host.numel() * 2
 
+    # ---------------- the next row of the path, timed on its own (not part of the step):
+    # the prologue backward, raster q, k, v gradients and the gains' gradients from the
+    # attention backward's blocked dq, dk, dv
+    next_rows = {}
+    if with_bwd:
+        pb = [torch.empty_like(q_d) for _ in range(3)]
+        dgq = torch.empty(w.head_dim, device=dev)
+        dgk = torch.empty(w.head_dim, device=dev)
+        for _ in range(2):
+            pipe.prologue_backward(q_d, k_d, pb[0], pb[1], pb[2], dgq, dgk, stream)
+        torch.cuda.synchronize()
+        p0 = torch.cuda.Event(enable_timing=True)
+        p1 = torch.cuda.Event(enable_timing=True)
+        p0.record(stream)
+        for _ in range(args.steps):
+            pipe.prologue_backward(q_d, k_d, pb[0], pb[1], pb[2], dgq, dgk, stream)
+        p1.record(stream)
+        torch.cuda.synchronize()
+        p_ms = p0.elapsed_time(p1) / args.steps
+        # read blocked dq, dk, dv and raster q, k; write raster dq, dk, dv
+        p_bytes = 3 * pipe.dq.numel() * 2 + 5 * q_d.numel() * 2
+        next_rows["prologue_bwd"] = {"ms_per_call": p_ms, "bytes": p_bytes,
+                                     "gbs": p_bytes / (p_ms * 1e-3) / 1e9}
+
     peaks = load_peaks()
     peak = peaks["bf16_tflops_sustained"]
     # algorithmic tensor FLOPs per launch of each attention kernel (128x128xD GEMM tiles):
@@ -396,6 +420,7 @@ def main():
                      "traffic": traffic_per_launch(dom, args.workload, n_pairs, n_pairs_cur)},
         "e2e": {"value": world * fl_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "next_rows": next_rows,
         "gpu_launches": args.steps * (3 + (4 if with_bwd else 0)),
         "clocks": clk.summary(),
     }
