@@ -24,6 +24,7 @@ scaling is weak; ranks meet only at the timing barriers.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import subprocess
@@ -383,6 +384,33 @@ def main():
         p_bytes = 3 * pipe.dq.numel() * 2 + 5 * q_d.numel() * 2
         next_rows["prologue_bwd"] = {"ms_per_call": p_ms, "bytes": p_bytes,
                                      "gbs": p_bytes / (p_ms * 1e-3) / 1e9}
+
+    # the continuation cache for the next round: this geometry's blocked K, V and key-block
+    # means appended to a cache of as many frames (the same tensors stand in for it)
+    if w.t_frames % w.blk[0] == 0:
+        gc = dataclasses.replace(g, cached_t=w.t_frames)
+        cshape = (g.batch, g.heads, 2 * g.nbq, g.bs, g.head_dim)
+        kc_n = torch.empty(cshape, dtype=torch.bfloat16, device=dev)
+        vc_n = torch.empty_like(kc_n)
+        kp_n = torch.empty(cshape[:3] + (g.head_dim,), dtype=torch.float32, device=dev)
+        ca = lambda: bsa.bsa_cache_append(gc, pipe.k, pipe.v, pipe.k_pool, pipe.k, pipe.v,  # noqa: E731
+                                          pipe.k_pool, kc_n, vc_n, kp_n, stream=stream)
+        for _ in range(2):
+            ca()
+        torch.cuda.synchronize()
+        c0 = torch.cuda.Event(enable_timing=True)
+        c1 = torch.cuda.Event(enable_timing=True)
+        c0.record(stream)
+        for _ in range(args.steps):
+            ca()
+        c1.record(stream)
+        torch.cuda.synchronize()
+        c_ms = c0.elapsed_time(c1) / args.steps
+        c_bytes = 2 * (kc_n.numel() * 2 * 2 + kp_n.numel() * 4)  # read + write K, V, means
+        next_rows["cache_append"] = {"ms_per_call": c_ms, "bytes": c_bytes,
+                                     "gbs": c_bytes / (c_ms * 1e-3) / 1e9,
+                                     "cached_t": gc.cached_t}
+        del kc_n, vc_n, kp_n
 
     peaks = load_peaks()
     peak = peaks["bf16_tflops_sustained"]

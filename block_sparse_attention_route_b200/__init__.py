@@ -19,6 +19,7 @@ __all__ = [
     "Geometry", "BsaError", "lib", "bsa_workspace_size", "rope3d_qknorm_prologue", "bsa_route",
     "bsa_attn_fwd", "bsa_attn_bwd", "bsa_device_status", "bsa_error_string", "blocked_shape",
     "bsa_selftest_bounded_wait", "bsa_route_noalloc", "rope3d_qknorm_prologue_bwd",
+    "bsa_cache_append",
     "bsa_kernel_timing", "bsa_kernel_times",
     "WS_ROUTE", "WS_FWD", "WS_BWD", "WS_PROLOGUE_BWD",
 ]
@@ -120,6 +121,7 @@ def lib() -> ctypes.CDLL:
             "bsa_selftest_bounded_wait": (I32, [I32, P]),
             "bsa_route_noalloc": (I32, [G, I32, P, P, P, P, P, P]),
             "bsa_kernel_timing": (I32, [I32]),
+            "bsa_cache_append": (I32, [G, P, P, P, P, P, P, P, P, P, P]),
             "bsa_kernel_times": (I32, [P, P]),
             "bsa_error_string": (ctypes.c_char_p, [I32]),
             "bsa_last_error_detail": (ctypes.c_char_p, []),
@@ -186,6 +188,14 @@ def rope3d_qknorm_prologue_bwd(g: Geometry, frames: int, t_offset: int, q, k, ga
         eps, rope_theta, _ptr(dq_blk), _ptr(dk_blk), _ptr(dv_blk), _ptr(dq), _ptr(dk), _ptr(dv),
         _ptr(dgamma_q), _ptr(dgamma_k), _ptr(ws), _nbytes(ws) if ws is not None else 0,
         _stream(stream)), "rope3d_qknorm_prologue_bwd")
+
+
+def bsa_cache_append(g: Geometry, kc_blk, vc_blk, kc_pool, k_blk, v_blk, k_pool, kc_new, vc_new,
+                     kc_pool_new=None, stream=None):
+    _check(lib().bsa_cache_append(
+        ctypes.byref(g.c()), _ptr(kc_blk), _ptr(vc_blk), _ptr(kc_pool), _ptr(k_blk), _ptr(v_blk),
+        _ptr(k_pool), _ptr(kc_new), _ptr(vc_new), _ptr(kc_pool_new), _stream(stream)),
+        "bsa_cache_append")
 
 
 def bsa_route(g: Geometry, top_r: int, q_blk, k_blk, q_pool, k_pool, kpool_cache, idx, cnt,

@@ -18,6 +18,7 @@
 #include "route.cu"
 #include "attn_fwd.cu"
 #include "attn_bwd.cu"
+#include "cache_append.cu"
 
 namespace bsa {
 
@@ -348,6 +349,39 @@ bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* gi, int32_t frames, in
   }
   cudaError_t e = launch_prologue_bwd(a, dgs, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "prologue backward launch");
+  return BSA_OK;
+}
+
+bsa_status_t bsa_cache_append(const bsa_geom_t* gi, const void* kc_blk, const void* vc_blk,
+                              const float* kc_pool, const void* k_blk, const void* v_blk,
+                              const float* k_pool, void* kc_new, void* vc_new, float* kc_pool_new,
+                              bsa_stream_t stream) {
+  t_detail.clear();
+  Geo g;
+  bsa_status_t st = make_geo(gi, &g);
+  if (st != BSA_OK) return st;
+  if (g.T % g.bt)
+    return fail(BSA_ERR_UNSUPPORTED, "t_frames %d must be a multiple of blk_t to extend a cache", g.T);
+  if (!k_blk || !v_blk || !kc_new || !vc_new)
+    return fail(BSA_ERR_INVALID_ARG, "k_blk, v_blk, kc_new and vc_new are required");
+  if (g.NBc > 0 && (!kc_blk || !vc_blk))
+    return fail(BSA_ERR_INVALID_ARG, "kc_blk and vc_blk are required when cached_t > 0");
+  if ((kc_pool_new != nullptr) != (k_pool != nullptr) || (kc_pool_new && g.NBc > 0 && !kc_pool))
+    return fail(BSA_ERR_INVALID_ARG, "block means: give k_pool and kc_pool_new (and kc_pool when cached_t > 0) or none");
+  const void* ptrs[9] = {kc_blk, vc_blk, kc_pool, k_blk, v_blk, k_pool, kc_new, vc_new, kc_pool_new};
+  for (const void* p : ptrs)
+    if (p && !aligned(p, 16)) return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int n_sm = 0;
+  st = check_device(&n_sm);
+  if (st != BSA_OK) return st;
+  const int bh = g.B * g.H;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t tile = (size_t)g.BS * g.D * 2;
+  cudaError_t e = launch_cache_append(kc_blk, k_blk, kc_new, bh, g.NBc, g.NBq, tile, n_sm, s);
+  if (e == cudaSuccess) e = launch_cache_append(vc_blk, v_blk, vc_new, bh, g.NBc, g.NBq, tile, n_sm, s);
+  if (e == cudaSuccess && kc_pool_new)
+    e = launch_cache_append(kc_pool, k_pool, kc_pool_new, bh, g.NBc, g.NBq, (size_t)g.D * 4, n_sm, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cache append launch");
   return BSA_OK;
 }
 

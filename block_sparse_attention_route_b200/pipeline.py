@@ -10,8 +10,8 @@ from typing import Dict, Optional
 import torch
 
 from . import (WS_BWD, WS_PROLOGUE_BWD, WS_ROUTE, Geometry, blocked_shape, bsa_attn_bwd,
-               bsa_attn_fwd, bsa_route, bsa_workspace_size, rope3d_qknorm_prologue,
-               rope3d_qknorm_prologue_bwd)
+               bsa_attn_fwd, bsa_cache_append, bsa_route, bsa_workspace_size,
+               rope3d_qknorm_prologue, rope3d_qknorm_prologue_bwd)
 
 
 class BsaPipeline:
@@ -66,6 +66,27 @@ class BsaPipeline:
                                self.gamma_k if self.qknorm else None, self.eps,
                                self.theta, None, self.kc, self.vc, None, self.kc_pool,
                                stream=stream)
+
+    def set_cache(self, kc_blk: torch.Tensor, vc_blk: torch.Tensor, kc_pool: torch.Tensor):
+        """Use blocked cache tensors made earlier (e.g. by next_round_cache of the previous
+        round) instead of running the prologue on raster cache frames."""
+        assert self.kc is not None and kc_blk.shape == self.kc.shape and vc_blk.shape == self.vc.shape
+        assert kc_pool.shape == self.kc_pool.shape
+        self.kc, self.vc, self.kc_pool = kc_blk, vc_blk, kc_pool
+
+    def next_round_cache(self, stream=None):
+        """The cache for the next continuation round: this round's cached blocks followed by
+        its current blocks (K, V and the key-block means), as new tensors."""
+        g = self.g
+        nb = g.nbc + g.nbq
+        kc = torch.empty((g.batch, g.heads, nb, g.bs, g.head_dim), dtype=self.k.dtype,
+                         device=self.k.device)
+        vc = torch.empty_like(kc)
+        kp = torch.empty((g.batch, g.heads, nb, g.head_dim), dtype=torch.float32,
+                         device=self.k.device)
+        bsa_cache_append(g, self.kc, self.vc, self.kc_pool, self.k, self.v, self.k_pool, kc, vc,
+                         kp, stream=stream)
+        return kc, vc, kp
 
     def prologue(self, q_raster, k_raster, v_raster, stream=None):
         g = self.g

@@ -121,6 +121,22 @@ BSA_API bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* g, int32_t frames,
                                     void* q_blk, void* k_blk, void* v_blk, float* q_pool,
                                     float* k_pool, bsa_stream_t stream);
 
+/* Continuation: the cache for the next round.  Source: "LongCat-Video 高效長視頻生成探索世界
+ * 模型的第壹步", section 2.1 (Block-Causal attention makes produced frames cacheable), and
+ * "LongCat-Video : Generate 1 minute long AI videos with this model", section "The core idea".
+ * For geometry g of the round just run (cached_t cached frames, t_frames current frames,
+ * t_frames a multiple of blk_t), writes per (b, h) the old cache's NBc blocks followed by the
+ * current NBq blocks: kc_new / vc_new bf16 [B, H, NBc + NBq, BS, D] from kc_blk / vc_blk
+ * (NULL when cached_t == 0) and the current k_blk / v_blk; kc_pool_new fp32 [B, H, NBc + NBq, D]
+ * likewise from kc_pool and k_pool (all three NULL to skip the means).  The result is the
+ * cache of a geometry with cached_t + t_frames cached frames.  Keys carry absolute-frame RoPE,
+ * so nothing is recomputed.  The caller owns every buffer; the outputs must not overlap the
+ * inputs. */
+BSA_API bsa_status_t bsa_cache_append(const bsa_geom_t* g, const void* kc_blk, const void* vc_blk,
+                                      const float* kc_pool, const void* k_blk, const void* v_blk,
+                                      const float* k_pool, void* kc_new, void* vc_new,
+                                      float* kc_pool_new, bsa_stream_t stream);
+
 /* Backward of rope3d_qknorm_prologue over the same `frames`, t_offset, gamma, eps and
  * rope_theta.  Same source; the talk "LongCat-Video 高效長視頻生成探索世界模型的第壹步",
  * section 2.2, has the sparse-attention module trained, which needs these gradients.

@@ -113,3 +113,19 @@ def test_prologue_bwd_host_validation():
         bsa.rope3d_qknorm_prologue_bwd(g, 24, 0, None, None, 16, None, 1e-6, 1e4,
                                        16, None, None, 16, None, None, stream=0)
     assert ei.value.code == 1
+
+
+def test_cache_append_host_validation():
+    g = _g(cached_t=8)
+    with pytest.raises(bsa.BsaError) as ei:  # a ragged last block-frame cannot extend a cache
+        bsa.bsa_cache_append(_g(t_frames=23), 16, 16, 16, 16, 16, 16, 16, 16, 16, stream=0)
+    assert ei.value.code == 2
+    with pytest.raises(bsa.BsaError) as ei:  # cached blocks to copy but no cache given
+        bsa.bsa_cache_append(g, None, None, None, 16, 16, 16, 16, 16, 16, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # new block means without the current ones
+        bsa.bsa_cache_append(g, 16, 16, 16, 16, 16, None, 16, 16, 16, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # misaligned output
+        bsa.bsa_cache_append(g, 16, 16, 16, 16, 16, 16, 24, 16, 16, stream=0)
+    assert ei.value.code == 1
