@@ -24,7 +24,7 @@ What it computes, with the page passages each step follows:
   minute long AI videos with this model", section "The core idea" (KV caching of the fixed
   conditioning frames).
 
-Where the pages are silent, this file takes the readings listed in the design doc: mean pooling
+Where the pages are silent, this file takes these readings: mean pooling
 over valid tokens, unscaled block scores, routing per (batch, head) on post-prologue q/k,
 ties broken by lower key-block index, selected lists in ascending block order, RoPE split
 (d_t, d_h, d_w) = (D - 4*floor(D/6), 2*floor(D/6), 2*floor(D/6)) with interleaved adjacent
@@ -271,11 +271,29 @@ def prologue_bwd(dz: np.ndarray, x: np.ndarray, frames: int, grid_h: int, grid_w
 # ----------------------------------------------------------------------------------------
 def block_means(x: np.ndarray, members: List[List[int]]) -> np.ndarray:
     """Mean over the valid tokens of each block: x raster [B, N, H, D] -> [B, H, NB, D]."""
+    return block_pool(x, members, "mean")
+
+
+def block_pool(x: np.ndarray, members: List[List[int]], mode: str = "mean") -> np.ndarray:
+    """One vector per block from its valid tokens: x raster [B, N, H, D] -> [B, H, NB, D].
+
+    ``mean`` is the routing's default reading of "blocks chosen by similarity"; ``sum`` and
+    ``max`` (channel-wise maximum) are the pooling variants the pages leave open.
+    """
     b_, _, h_, d_ = x.shape
     out = np.zeros((b_, h_, len(members), d_), dtype=np.float64)
     for j, idx in enumerate(members):
-        if idx:
-            out[:, :, j, :] = np.asarray(x[:, idx], dtype=np.float64).mean(axis=1)
+        if not idx:
+            continue
+        tok = np.asarray(x[:, idx], dtype=np.float64)  # [B, n_j, H, D]
+        if mode == "mean":
+            out[:, :, j, :] = tok.mean(axis=1)
+        elif mode == "sum":
+            out[:, :, j, :] = tok.sum(axis=1)
+        elif mode == "max":
+            out[:, :, j, :] = tok.max(axis=1)
+        else:
+            raise ValueError(mode)
     return out
 
 
@@ -317,19 +335,54 @@ def select_top_r(s: np.ndarray, r: int) -> Tuple[np.ndarray, np.ndarray]:
     return idx.reshape(lead + (r,)), cnt.reshape(lead)
 
 
+def select_with_self(s: np.ndarray, r: int, nbc: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Forced self-block variant: query block i always keeps its own key block nbc + i,
+    and the other r - 1 places go to the best of the remaining blocks (the top-r rule with
+    ties to the lower index).  s is [..., NBq, NBk]; same outputs as ``select_top_r``."""
+    nbq, nb = s.shape[-2], s.shape[-1]
+    idx = -np.ones(s.shape[:-1] + (r,), dtype=np.int32)
+    cnt = np.zeros(s.shape[:-1], dtype=np.int32)
+    for lead in np.ndindex(s.shape[:-2]):
+        for i in range(nbq):
+            own = nbc + i
+            rest = s[lead + (i,)].copy()
+            rest[own] = NEG_INF
+            others, n_o = select_top_r(rest[None], r - 1) if r > 1 else (np.zeros((1, 0), np.int32), [0])
+            chosen = np.sort(np.concatenate([[own], others[0, :n_o[0]]]))
+            idx[lead + (i,)][:len(chosen)] = chosen
+            cnt[lead + (i,)] = len(chosen)
+    return idx, cnt
+
+
 def route(q: np.ndarray, k: np.ndarray, grid: Grid, r: int,
-          k_cache: Optional[np.ndarray] = None):
-    """Block-pooled q.k routing: returns (idx [B,H,NBq,r], cnt [B,H,NBq], scores)."""
+          k_cache: Optional[np.ndarray] = None, *, pool: str = "mean",
+          force_self: bool = False, shared_heads: bool = False):
+    """Block-pooled q.k routing: returns (idx [B,H,NBq,r], cnt [B,H,NBq], scores).
+
+    Variants: ``pool`` = mean | sum | max block pooling; ``force_self`` always keeps a query
+    block's own key block; ``shared_heads`` ranks key blocks by the score summed over the
+    heads, s_ij = sum_h qbar_hi . kbar_hj, and gives every head that one selection (the
+    returned scores are then [B, 1, NBq, NBk]).
+    """
     qm = grid.block_members(grid.t_frames)
-    qbar = block_means(q, qm)
-    kbar = block_means(k, qm)
+    qbar = block_pool(q, qm, pool)
+    kbar = block_pool(k, qm, pool)
     counts = [len(m) for m in qm]
     if grid.nbc:
         cm = grid.block_members(grid.cached_t)
-        kbar = np.concatenate([block_means(k_cache, cm), kbar], axis=2)
+        kbar = np.concatenate([block_pool(k_cache, cm, pool), kbar], axis=2)
         counts = [len(m) for m in cm] + counts
     s = block_scores(qbar, kbar, grid, counts)
-    idx, cnt = select_top_r(s, r)
+    if shared_heads:
+        s = s.sum(axis=1, keepdims=True)
+    if force_self:
+        idx, cnt = select_with_self(s, r, grid.nbc)
+    else:
+        idx, cnt = select_top_r(s, r)
+    if shared_heads:
+        h_ = q.shape[2]
+        idx = np.repeat(idx, h_, axis=1)
+        cnt = np.repeat(cnt, h_, axis=1)
     return idx, cnt, s
 
 

@@ -5,6 +5,7 @@ routine (torch CPU scaled_dot_product_attention and autograd in fp64), a pure-Py
 force on tiny grids, closed forms of the rotary embedding, invariants of softmax and RoPE,
 or numerical derivatives.  None of these needs a GPU.
 """
+import itertools
 import math
 
 import numpy as np
@@ -505,3 +506,137 @@ def test_rmsnorm_bwd_is_orthogonal_to_the_input_without_eps():
     dx2, dg2 = oracle.prologue_bwd(dz, x, 2, 3, 5, gamma=None, theta=0.0)
     assert dg2 is None
     np.testing.assert_array_equal(dx2, dz)
+
+
+# ------------------------------------------------------------------ routing variants
+def _brute_variant(q, k, grid, r, pool, force_self, shared):
+    """Scalar loops: per-head block pooling (mean / sum / channel max), scores, optional sum
+    over heads, then the best-scoring set by exhaustive search over combinations (inputs are
+    continuous random values, so the best set is unique), holding the own block when forced.
+    Grids here have no cache, so query block i's own key block is block i."""
+    B, N, H, D = q.shape
+    mem = grid.block_members(grid.t_frames)
+
+    def pooled(arr, b, h, toks):
+        out = []
+        for d in range(D):
+            vals = [float(arr[b, t, h, d]) for t in toks]
+            out.append(max(vals) if pool == "max" else sum(vals) / (len(vals) if pool == "mean" else 1))
+        return out
+
+    res = {}
+    for b in range(B):
+        per_head = []
+        for h in range(H):
+            qp = [pooled(q, b, h, t) for t in mem]
+            kp = [pooled(k, b, h, t) for t in mem]
+            per_head.append([[sum(qp[i][d] * kp[j][d] for d in range(D)) for j in range(grid.nbk)]
+                             for i in range(grid.nbq)])
+        if shared:
+            per_head = [[[sum(per_head[h][i][j] for h in range(H)) for j in range(grid.nbk)]
+                         for i in range(grid.nbq)]]
+        for hh, sc in enumerate(per_head):
+            for i in range(grid.nbq):
+                allowed = [j for j in range(grid.nbk)
+                           if not (grid.chunk_t and grid.key_block_chunk(j) > grid.query_block_chunk(i))]
+                must = [i] if force_self else []
+                rest = [j for j in allowed if j not in must]
+                m = min(r, len(allowed)) - len(must)
+                best = max(itertools.combinations(rest, m), key=lambda c: sum(sc[i][j] for j in c))
+                res[(b, hh, i)] = sorted(must + list(best))
+    return res
+
+
+@pytest.mark.parametrize("gridspec", [(4, 8, 8, 0), (3, 7, 6, 0), (8, 4, 4, 4)])
+@pytest.mark.parametrize("pool,force_self,shared", [
+    ("mean", True, False), ("mean", False, True), ("mean", True, True),
+    ("sum", False, False), ("max", False, False), ("max", True, True)])
+def test_route_variants_brute_force(gridspec, pool, force_self, shared):
+    t, gh, gw, chunk = gridspec
+    g = Grid(t, gh, gw, (2, 4, 4), chunk_t=chunk)
+    rng = np.random.default_rng(17)
+    q = rng.standard_normal((1, t * gh * gw, 2, 8))
+    k = rng.standard_normal((1, t * gh * gw, 2, 8))
+    r = 3
+    idx, cnt, s = oracle.route(q, k, g, r, pool=pool, force_self=force_self, shared_heads=shared)
+    ref = _brute_variant(q, k, g, r, pool, force_self, shared)
+    for h in range(2):
+        for i in range(g.nbq):
+            sel = ref[(0, 0 if shared else h, i)]
+            assert cnt[0, h, i] == len(sel)
+            assert list(idx[0, h, i, :len(sel)]) == sel and all(idx[0, h, i, len(sel):] == -1)
+            if force_self:
+                assert i in sel
+    if shared:
+        assert s.shape[1] == 1 and np.array_equal(idx[:, 0], idx[:, 1])
+
+
+def test_force_self_with_r1_keeps_only_the_own_block():
+    w, x = _inputs("small_cont")
+    g = _grid(w)
+    idx, cnt, _ = oracle.route(x["q"], x["k"], g, 1, k_cache=x["kc"], force_self=True)
+    assert np.all(cnt == 1)
+    assert np.array_equal(idx[0, 0, :, 0], g.nbc + np.arange(g.nbq))
+
+
+def test_force_self_changes_nothing_where_the_own_block_already_wins():
+    w, x = _inputs("small")
+    g = _grid(w)
+    plain, _, _ = oracle.route(x["q"], x["k"], g, w.top_r)
+    forced, _, _ = oracle.route(x["q"], x["k"], g, w.top_r, force_self=True)
+    has_own = np.array([[[i in plain[b, h, i] for i in range(g.nbq)] for h in range(w.heads)]
+                        for b in range(w.batch)])
+    assert has_own.any() and (~has_own).any()
+    assert np.array_equal(plain[has_own], forced[has_own])
+    assert not np.array_equal(plain[~has_own], forced[~has_own])
+
+
+def test_shared_heads_with_identical_heads_is_the_per_head_route():
+    w, x = _inputs("small_b2")
+    g = _grid(w)
+    q = np.repeat(x["q"][:, :, :1], w.heads, axis=2)
+    k = np.repeat(x["k"][:, :, :1], w.heads, axis=2)
+    per, _, s1 = oracle.route(q, k, g, w.top_r)
+    sh, _, s = oracle.route(q, k, g, w.top_r, shared_heads=True)
+    assert np.array_equal(per, sh)
+    np.testing.assert_allclose(s[:, 0], w.heads * s1[:, 0], rtol=1e-12)
+
+
+def test_pooling_modes_closed_forms():
+    g = Grid(3, 7, 6, (2, 4, 4))  # ragged in t, h and w
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((1, 3 * 7 * 6, 2, 8))
+    mem = g.block_members(3)
+    mean, tot, mx = (oracle.block_pool(x, mem, m) for m in ("mean", "sum", "max"))
+    counts = np.array([len(m) for m in mem], dtype=np.float64)
+    np.testing.assert_allclose(tot, mean * counts[None, None, :, None], rtol=1e-12)
+    assert np.all(mx >= mean - 1e-15)
+    # a block whose tokens all hold one vector pools to that vector in every mode
+    x[0, mem[4]] = x[0, mem[4][0]]
+    for m in ("mean", "max"):
+        np.testing.assert_allclose(oracle.block_pool(x, mem, m)[0, :, 4], x[0, mem[4][0]], rtol=1e-15)
+    # channel max commutes with adding a constant and with a token permutation
+    perm = rng.permutation(x.shape[1])
+    inv = np.argsort(perm)
+    mem_p = [[int(inv[t]) for t in m] for m in mem]
+    np.testing.assert_array_equal(oracle.block_pool(x[:, perm], mem_p, "max"), oracle.block_pool(x, mem, "max"))
+    np.testing.assert_allclose(oracle.block_pool(x + 3.0, mem, "max"), oracle.block_pool(x, mem, "max") + 3.0)
+
+
+def test_sum_pooling_ranks_like_mean_on_whole_blocks_and_penalises_partial_ones():
+    w, x = _inputs("small")  # 10 x 20 grid: ragged blocks on h and w
+    g = _grid(w)
+    mem = g.block_members(w.t_frames)
+    whole = [j for j, m in enumerate(mem) if len(m) == g.bs]
+    part = [j for j, m in enumerate(mem) if len(m) < g.bs]
+    assert whole and part
+    _, _, sm = oracle.route(x["q"], x["k"], g, w.top_r)
+    _, _, ss = oracle.route(x["q"], x["k"], g, w.top_r, pool="sum")
+    counts = np.array([len(m) for m in mem], dtype=np.float64)
+    np.testing.assert_allclose(ss, sm * counts[None, None, :, None] * counts[None, None, None, :],
+                               rtol=1e-9, atol=1e-12)
+    # among whole key blocks the order of scores is the same
+    for i in range(g.nbq):
+        a = np.argsort(-sm[0, 0, i, whole], kind="stable")
+        b = np.argsort(-ss[0, 0, i, whole], kind="stable")
+        assert np.array_equal(a, b)
