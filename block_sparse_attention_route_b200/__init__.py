@@ -19,7 +19,8 @@ __all__ = [
     "Geometry", "BsaError", "lib", "bsa_workspace_size", "rope3d_qknorm_prologue", "bsa_route",
     "bsa_attn_fwd", "bsa_attn_bwd", "bsa_device_status", "bsa_error_string", "blocked_shape",
     "bsa_selftest_bounded_wait", "bsa_route_noalloc", "rope3d_qknorm_prologue_bwd",
-    "bsa_cache_append",
+    "bsa_cache_append", "bsa_route_ex", "bsa_block_pool", "ROUTE_FORCE_SELF",
+    "ROUTE_SHARED_HEADS", "ROUTE_POOL_SUM", "ROUTE_POOL_MAX", "POOL_MEAN", "POOL_SUM", "POOL_MAX",
     "bsa_kernel_timing", "bsa_kernel_times",
     "WS_ROUTE", "WS_FWD", "WS_BWD", "WS_PROLOGUE_BWD",
 ]
@@ -27,6 +28,8 @@ __all__ = [
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libbsa.so")
 WS_ROUTE, WS_FWD, WS_BWD, WS_PROLOGUE_BWD = 1, 2, 3, 4
+ROUTE_FORCE_SELF, ROUTE_SHARED_HEADS, ROUTE_POOL_SUM, ROUTE_POOL_MAX = 1, 2, 4, 8
+POOL_MEAN, POOL_SUM, POOL_MAX = 0, 1, 2
 STATUS = {0: "BSA_OK", 1: "BSA_ERR_INVALID_ARG", 2: "BSA_ERR_UNSUPPORTED", 3: "BSA_ERR_CUDA",
           4: "BSA_ERR_TIMEOUT", 5: "BSA_ERR_BAD_INDEX", 6: "BSA_ERR_WORKSPACE"}
 
@@ -115,6 +118,8 @@ def lib() -> ctypes.CDLL:
             "rope3d_qknorm_prologue_bwd": (I32, [G, I32, I32, P, P, P, P, F, F, P, P, P, P, P, P,
                                                  P, P, P, S, P]),
             "bsa_route": (I32, [G, I32, P, P, P, P, P, P, P, P, S, P]),
+            "bsa_route_ex": (I32, [G, I32, ctypes.c_uint32, P, P, P, P, P, P, P, P, S, P]),
+            "bsa_block_pool": (I32, [G, I32, I32, P, P, P]),
             "bsa_attn_fwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P]),
             "bsa_attn_bwd": (I32, [G, I32, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
             "bsa_device_status": (I32, [P]),
@@ -204,6 +209,20 @@ def bsa_route(g: Geometry, top_r: int, q_blk, k_blk, q_pool, k_pool, kpool_cache
     _check(lib().bsa_route(
         ctypes.byref(g.c()), top_r, _ptr(q_blk), _ptr(k_blk), _ptr(q_pool), _ptr(k_pool),
         _ptr(kpool_cache), _ptr(idx), _ptr(cnt), _ptr(ws), nbytes, _stream(stream)), "bsa_route")
+
+
+def bsa_route_ex(g: Geometry, top_r: int, flags: int, q_blk, k_blk, q_pool, k_pool, kpool_cache,
+                 idx, cnt, ws=None, stream=None):
+    nbytes = _nbytes(ws)
+    _check(lib().bsa_route_ex(
+        ctypes.byref(g.c()), top_r, flags, _ptr(q_blk), _ptr(k_blk), _ptr(q_pool), _ptr(k_pool),
+        _ptr(kpool_cache), _ptr(idx), _ptr(cnt), _ptr(ws), nbytes, _stream(stream)),
+        "bsa_route_ex")
+
+
+def bsa_block_pool(g: Geometry, frames: int, mode: int, x_blk, out, stream=None):
+    _check(lib().bsa_block_pool(ctypes.byref(g.c()), frames, mode, _ptr(x_blk), _ptr(out),
+                                _stream(stream)), "bsa_block_pool")
 
 
 def bsa_route_noalloc(g: Geometry, top_r: int, q_blk, k_blk, kpool_cache, idx, cnt, stream=None):

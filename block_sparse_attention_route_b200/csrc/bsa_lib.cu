@@ -389,11 +389,27 @@ bsa_status_t bsa_route(const bsa_geom_t* gi, int32_t top_r, const void* q_blk,
                        const void* k_blk, const float* q_pool, const float* k_pool,
                        const float* kpool_cache, int32_t* idx, int32_t* cnt, void* ws,
                        size_t ws_bytes, bsa_stream_t stream) {
+  return bsa_route_ex(gi, top_r, 0u, q_blk, k_blk, q_pool, k_pool, kpool_cache, idx, cnt, ws,
+                      ws_bytes, stream);
+}
+
+bsa_status_t bsa_route_ex(const bsa_geom_t* gi, int32_t top_r, uint32_t flags, const void* q_blk,
+                          const void* k_blk, const float* q_pool, const float* k_pool,
+                          const float* kpool_cache, int32_t* idx, int32_t* cnt, void* ws,
+                          size_t ws_bytes, bsa_stream_t stream) {
   t_detail.clear();
   Geo g;
   bsa_status_t st = make_geo(gi, &g);
   if (st != BSA_OK) return st;
   if (top_r < 1) return fail(BSA_ERR_INVALID_ARG, "top_r must be >= 1");
+  const uint32_t known = BSA_ROUTE_FORCE_SELF | BSA_ROUTE_SHARED_HEADS | BSA_ROUTE_POOL_SUM |
+                         BSA_ROUTE_POOL_MAX;
+  if (flags & ~known) return fail(BSA_ERR_INVALID_ARG, "unknown route flags 0x%x", flags & ~known);
+  const bool pool_sum = flags & BSA_ROUTE_POOL_SUM, pool_max = flags & BSA_ROUTE_POOL_MAX;
+  if (pool_sum && pool_max) return fail(BSA_ERR_INVALID_ARG, "choose one pooling mode");
+  const int pool_mode = pool_sum ? kPoolSum : pool_max ? kPoolMax : kPoolMean;
+  if (pool_mode != kPoolMean && (q_pool || k_pool))
+    return fail(BSA_ERR_INVALID_ARG, "a pooling flag pools q_blk / k_blk here: pass no q_pool / k_pool");
   if (!idx || !cnt) return fail(BSA_ERR_INVALID_ARG, "idx and cnt are required");
   if ((!q_pool && !q_blk) || (!k_pool && !k_blk))
     return fail(BSA_ERR_INVALID_ARG, "need q_blk or q_pool, and k_blk or k_pool");
@@ -405,6 +421,11 @@ bsa_status_t bsa_route(const bsa_geom_t* gi, int32_t top_r, const void* q_blk,
   const RouteWs w = route_ws(g);
   if ((!q_pool || !k_pool) && (ws == nullptr || ws_bytes < w.total || !aligned(ws, 256)))
     return fail(BSA_ERR_WORKSPACE, "route needs %zu workspace bytes (256-byte aligned)", w.total);
+  // one CTA covers all heads of its query rows when they share a selection: fewer rows per
+  // CTA keep more SMs busy
+  const int qt = (flags & BSA_ROUTE_SHARED_HEADS) ? std::min(select_rows_per_cta(g), 8)
+                                                  : select_rows_per_cta(g);
+  if (qt == 0) return fail(BSA_ERR_UNSUPPORTED, "%d key blocks do not fit the select kernel", g.NBk);
   int n_sm = 0;
   st = check_device(&n_sm);
   if (st != BSA_OK) return st;
@@ -412,26 +433,51 @@ bsa_status_t bsa_route(const bsa_geom_t* gi, int32_t top_r, const void* q_blk,
   cudaError_t e;
   if (!q_pool) {
     float* out = reinterpret_cast<float*>(static_cast<char*>(ws) + w.qpool);
-    if ((e = launch_pool(static_cast<const __nv_bfloat16*>(q_blk), g.T, g.NBq, g, out, s)) != cudaSuccess)
+    if ((e = launch_pool(static_cast<const __nv_bfloat16*>(q_blk), g.T, g.NBq, g, out, s, pool_mode)) != cudaSuccess)
       return cuda_fail(e, "pool launch");
     q_pool = out;
   }
   if (!k_pool) {
     float* out = reinterpret_cast<float*>(static_cast<char*>(ws) + w.kpool);
-    if ((e = launch_pool(static_cast<const __nv_bfloat16*>(k_blk), g.T, g.NBq, g, out, s)) != cudaSuccess)
+    if ((e = launch_pool(static_cast<const __nv_bfloat16*>(k_blk), g.T, g.NBq, g, out, s, pool_mode)) != cudaSuccess)
       return cuda_fail(e, "pool launch");
     k_pool = out;
   }
   SelectArgs a;
   a.g = g;
   a.r = top_r;
-  a.qt = select_rows_per_cta(g);
+  a.flags = (flags & BSA_ROUTE_FORCE_SELF ? kRouteForceSelf : 0u) |
+            (flags & BSA_ROUTE_SHARED_HEADS ? kRouteSharedHeads : 0u);
+  a.qt = qt;
   a.qpool = q_pool;
   a.kpool = k_pool;
   a.kpool_cache = kpool_cache;
   a.idx = idx;
   a.cnt = cnt;
   if ((e = launch_select(a, s)) != cudaSuccess) return cuda_fail(e, "select launch");
+  return BSA_OK;
+}
+
+bsa_status_t bsa_block_pool(const bsa_geom_t* gi, int32_t frames, int32_t mode,
+                            const void* x_blk, float* out, bsa_stream_t stream) {
+  t_detail.clear();
+  Geo g;
+  bsa_status_t st = make_geo(gi, &g);
+  if (st != BSA_OK) return st;
+  if (frames < 1) return fail(BSA_ERR_INVALID_ARG, "frames must be >= 1");
+  if (mode != BSA_POOL_MEAN && mode != BSA_POOL_SUM && mode != BSA_POOL_MAX)
+    return fail(BSA_ERR_INVALID_ARG, "unknown pooling mode %d", mode);
+  if (!x_blk || !out) return fail(BSA_ERR_INVALID_ARG, "x_blk and out are required");
+  if (!aligned(x_blk, 16) || !aligned(out, 16))
+    return fail(BSA_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  int n_sm = 0;
+  st = check_device(&n_sm);
+  if (st != BSA_OK) return st;
+  const int nb = ((frames + g.bt - 1) / g.bt) * g.nbh * g.nbw;
+  const int m = mode == BSA_POOL_SUM ? kPoolSum : mode == BSA_POOL_MAX ? kPoolMax : kPoolMean;
+  cudaError_t e = launch_pool(static_cast<const __nv_bfloat16*>(x_blk), frames, nb, g, out,
+                              reinterpret_cast<cudaStream_t>(stream), m);
+  if (e != cudaSuccess) return cuda_fail(e, "pool launch");
   return BSA_OK;
 }
 

@@ -5,30 +5,40 @@
 // most relevant ones, chosen by similarity); "LongCat-Video视频生成模型发布 迈出世界模型探索
 // 第一步", section 块稀疏注意力（BSA） (only the top-r key blocks are computed).
 //
-// pool_kernel      : qbar/kbar = mean over the valid tokens of each block (fp32).
+// pool_kernel      : qbar/kbar = mean over the valid tokens of each block (fp32); the sum and
+//                    channel-wise max are the pooling variants.
 // score_select     : s_ij = qbar_i . kbar_j in fp32 on CUDA cores (ranking needs fp32, the
 //                    work is ~NBq*NBk*D FMAs per head, tiny next to the attention), masked
 //                    to -inf by the block-causal rule, then an exact warp-level radix select
 //                    of the top r per row on order-preserving 32-bit keys, ties resolved to
 //                    the lower block index, emitted in ascending block order.
+// Variants (the pages leave the routing rule open): the own key block NBc + i forced into
+// every query block's selection (its score is taken as +inf, so it always ranks first), and
+// one selection per (b, query block) shared by all heads, ranked by the score summed over
+// the heads, s_ij = sum_h qbar_hi . kbar_hj.
 #include "common.cuh"
 
 namespace bsa {
 
 constexpr int kPoolThreads = 256;
+constexpr int kPoolMean = 0, kPoolSum = 1, kPoolMax = 2;
+constexpr unsigned kRouteForceSelf = 1u, kRouteSharedHeads = 2u;
 
-template <int D>
+template <int D, int MODE>  // MODE: kPoolMean, kPoolSum, kPoolMax
 __global__ void __launch_bounds__(kPoolThreads)
     pool_kernel(const __nv_bfloat16* __restrict__ x, int frames, int nb, Geo g,
                 float* __restrict__ out) {
   constexpr int CPR = D / 8, RG = kPoolThreads / CPR;
+  constexpr float kInit = MODE == kPoolMax ? -INFINITY : 0.f;
   __shared__ float red[RG][D];
   const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, cc = tid % CPR, rg = tid / CPR;
   int vt, vh, vw;
   block_extent(g, frames, blk, vt, vh, vw);
   const __nv_bfloat16* base = x + (((size_t)b * g.H + h) * nb + blk) * (size_t)g.BS * D;
-  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  float acc[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) acc[e] = kInit;
   for (int slot = rg; slot < g.BS; slot += RG) {
     const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
     if (lt < vt && lh < vh && lw < vw) {
@@ -37,7 +47,11 @@ __global__ void __launch_bounds__(kPoolThreads)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         float2 f = __bfloat1622float2(p2[e]);
-        acc[2 * e] += f.x; acc[2 * e + 1] += f.y;
+        if (MODE == kPoolMax) {
+          acc[2 * e] = fmaxf(acc[2 * e], f.x); acc[2 * e + 1] = fmaxf(acc[2 * e + 1], f.y);
+        } else {
+          acc[2 * e] += f.x; acc[2 * e + 1] += f.y;
+        }
       }
     }
   }
@@ -46,9 +60,11 @@ __global__ void __launch_bounds__(kPoolThreads)
   __syncthreads();
   const int nvalid = max(vt, 0) * max(vh, 0) * max(vw, 0);
   for (int d = tid; d < D; d += kPoolThreads) {
-    float s = 0.f;
-    for (int r = 0; r < RG; ++r) s += red[r][d];
-    out[(((size_t)b * g.H + h) * nb + blk) * D + d] = nvalid ? s / (float)nvalid : 0.f;
+    float s = kInit;
+    for (int r = 0; r < RG; ++r) s = MODE == kPoolMax ? fmaxf(s, red[r][d]) : s + red[r][d];
+    float v = 0.f;
+    if (nvalid) v = MODE == kPoolMean ? s / (float)nvalid : s;
+    out[(((size_t)b * g.H + h) * nb + blk) * D + d] = v;
   }
 }
 
@@ -64,6 +80,7 @@ __device__ __forceinline__ uint32_t ordered_key(float f) {
 struct SelectArgs {
   Geo g;
   int r, qt;                  // top-r, query blocks per CTA
+  unsigned flags = 0;         // kRouteForceSelf | kRouteSharedHeads
   const float* qpool;         // [B,H,NBq,D]
   const float* kpool;         // [B,H,NBq,D] current key blocks
   const float* kpool_cache;   // [B,H,NBc,D] or null
@@ -84,50 +101,57 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(const SelectA
   const Geo& g = a.g;
   const int i0 = blockIdx.x * QT, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const size_t bh = (size_t)b * g.H + h;
+  const bool shared_heads = (a.flags & kRouteSharedHeads) != 0;
+  const bool force_self = (a.flags & kRouteForceSelf) != 0;
+  // heads whose scores are summed: this CTA's head, or all of them (then gridDim.y == 1)
+  const int h_lo = shared_heads ? 0 : h, h_hi = shared_heads ? g.H : h + 1;
   const int nq = min(QT, g.NBq - i0);
-
-  for (int e = tid; e < QT * (D / 4); e += kSelThreads) {
-    const int ii = e / (D / 4), d4 = e % (D / 4);
-    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (ii < nq) v = *reinterpret_cast<const float4*>(a.qpool + (bh * g.NBq + i0 + ii) * D + d4 * 4);
-    *reinterpret_cast<float4*>(qs + ii * LD + d4 * 4) = v;
-  }
 
   const int ti = tid / 32, tj = tid % 32;
   for (int j0 = 0; j0 < g.NBk; j0 += kKT) {
-    __syncthreads();
-    for (int e = tid; e < kKT * (D / 4); e += kSelThreads) {
-      const int jj = e / (D / 4), d4 = e % (D / 4), j = j0 + jj;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (j < g.NBc)
-        v = *reinterpret_cast<const float4*>(a.kpool_cache + (bh * g.NBc + j) * D + d4 * 4);
-      else if (j < g.NBk)
-        v = *reinterpret_cast<const float4*>(a.kpool + (bh * g.NBq + (j - g.NBc)) * D + d4 * 4);
-      *reinterpret_cast<float4*>(ks + jj * LD + d4 * 4) = v;
-    }
-    __syncthreads();
     float acc[RPT][4];
 #pragma unroll
     for (int x = 0; x < RPT; ++x)
 #pragma unroll
       for (int m = 0; m < 4; ++m) acc[x][m] = 0.f;
-#pragma unroll 4
-    for (int d = 0; d < D; d += 4) {
-      float4 kv[4], qv[RPT];
-#pragma unroll
-      for (int m = 0; m < 4; ++m) kv[m] = *reinterpret_cast<const float4*>(ks + (tj + 32 * m) * LD + d);
-#pragma unroll
-      for (int x = 0; x < RPT; ++x) qv[x] = *reinterpret_cast<const float4*>(qs + (ti * RPT + x) * LD + d);
-#pragma unroll
-      for (int x = 0; x < RPT; ++x)
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          acc[x][m] = fmaf(qv[x].x, kv[m].x, acc[x][m]);
-          acc[x][m] = fmaf(qv[x].y, kv[m].y, acc[x][m]);
-          acc[x][m] = fmaf(qv[x].z, kv[m].z, acc[x][m]);
-          acc[x][m] = fmaf(qv[x].w, kv[m].w, acc[x][m]);
+    for (int hh = h_lo; hh < h_hi; ++hh) {
+      const size_t bh = (size_t)b * g.H + hh;
+      __syncthreads();  // the previous head / tile is no longer read
+      if (shared_heads || j0 == 0) {
+        for (int e = tid; e < QT * (D / 4); e += kSelThreads) {
+          const int ii = e / (D / 4), d4 = e % (D / 4);
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (ii < nq) v = *reinterpret_cast<const float4*>(a.qpool + (bh * g.NBq + i0 + ii) * D + d4 * 4);
+          *reinterpret_cast<float4*>(qs + ii * LD + d4 * 4) = v;
         }
+      }
+      for (int e = tid; e < kKT * (D / 4); e += kSelThreads) {
+        const int jj = e / (D / 4), d4 = e % (D / 4), j = j0 + jj;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (j < g.NBc)
+          v = *reinterpret_cast<const float4*>(a.kpool_cache + (bh * g.NBc + j) * D + d4 * 4);
+        else if (j < g.NBk)
+          v = *reinterpret_cast<const float4*>(a.kpool + (bh * g.NBq + (j - g.NBc)) * D + d4 * 4);
+        *reinterpret_cast<float4*>(ks + jj * LD + d4 * 4) = v;
+      }
+      __syncthreads();
+#pragma unroll 4
+      for (int d = 0; d < D; d += 4) {
+        float4 kv[4], qv[RPT];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) kv[m] = *reinterpret_cast<const float4*>(ks + (tj + 32 * m) * LD + d);
+#pragma unroll
+        for (int x = 0; x < RPT; ++x) qv[x] = *reinterpret_cast<const float4*>(qs + (ti * RPT + x) * LD + d);
+#pragma unroll
+        for (int x = 0; x < RPT; ++x)
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            acc[x][m] = fmaf(qv[x].x, kv[m].x, acc[x][m]);
+            acc[x][m] = fmaf(qv[x].y, kv[m].y, acc[x][m]);
+            acc[x][m] = fmaf(qv[x].z, kv[m].z, acc[x][m]);
+            acc[x][m] = fmaf(qv[x].w, kv[m].w, acc[x][m]);
+          }
+      }
     }
 #pragma unroll
     for (int x = 0; x < RPT; ++x) {
@@ -140,8 +164,11 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(const SelectA
         if (j >= g.NBk) continue;
         bool ok = true;
         if (g.chunk) ok = key_block_t0(g, j) / g.chunk <= ci;
-        // a key block always holds >= 1 valid token when the grid is padded to whole blocks
-        sc[(size_t)ii * g.NBk + j] = ok ? acc[x][m] : -INFINITY;
+        // a key block always holds >= 1 valid token when the grid is padded to whole blocks;
+        // the own block (same frames, so never masked) ranks above every finite score
+        float v = ok ? acc[x][m] : -INFINITY;
+        if (force_self && j == g.NBc + i) v = INFINITY;
+        sc[(size_t)ii * g.NBk + j] = v;
       }
     }
   }
@@ -152,7 +179,6 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(const SelectA
   const unsigned lt_mask = (1u << lane) - 1u;
   for (int ii = warp; ii < nq; ii += 8) {
     const float* srow = sc + (size_t)ii * g.NBk;
-    const size_t row = bh * g.NBq + i0 + ii;
     int nfin = 0;
     for (int j = lane; j < g.NBk; j += 32) nfin += (srow[j] > -INFINITY) ? 1 : 0;
 #pragma unroll
@@ -203,7 +229,6 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(const SelectA
     }
     // emit ascending: keys above the threshold, then the first k keys equal to it
     int written = 0, eq_seen = 0;
-    int* out = a.idx + row * a.r;
     if (reff > 0) {
       for (int base = 0; base < g.NBk; base += 32) {
         const int j = base + lane;
@@ -220,30 +245,44 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(const SelectA
         const bool take = gt || (eq && eq_seen + __popc(eqm & lt_mask) < k);
         const unsigned tm = __ballot_sync(0xffffffffu, take);
         const int pos = written + __popc(tm & lt_mask);
-        if (take && pos < a.r) out[pos] = j;
+        if (take && pos < a.r)
+          for (int hh = h_lo; hh < h_hi; ++hh)
+            a.idx[(((size_t)b * g.H + hh) * g.NBq + i0 + ii) * a.r + pos] = j;
         written += __popc(tm);
         eq_seen += __popc(eqm);
       }
     }
     written = min(written, a.r);
-    for (int e = written + lane; e < a.r; e += 32) out[e] = -1;
-    if (lane == 0) a.cnt[row] = written;
+    for (int hh = h_lo; hh < h_hi; ++hh) {
+      const size_t row = ((size_t)b * g.H + hh) * g.NBq + i0 + ii;
+      for (int e = written + lane; e < a.r; e += 32) a.idx[row * a.r + e] = -1;
+      if (lane == 0) a.cnt[row] = written;
+    }
   }
 }
 
-cudaError_t launch_pool(const __nv_bfloat16* x, int frames, int nb, const Geo& g, float* out,
-                        cudaStream_t s) {
+template <int D>
+static cudaError_t launch_pool_d(const __nv_bfloat16* x, int frames, int nb, const Geo& g,
+                                 int mode, float* out, cudaStream_t s) {
   dim3 grid(nb, g.H, g.B);
-  if (g.D == 128) pool_kernel<128><<<grid, kPoolThreads, 0, s>>>(x, frames, nb, g, out);
-  else pool_kernel<64><<<grid, kPoolThreads, 0, s>>>(x, frames, nb, g, out);
+  if (mode == kPoolSum) pool_kernel<D, kPoolSum><<<grid, kPoolThreads, 0, s>>>(x, frames, nb, g, out);
+  else if (mode == kPoolMax) pool_kernel<D, kPoolMax><<<grid, kPoolThreads, 0, s>>>(x, frames, nb, g, out);
+  else pool_kernel<D, kPoolMean><<<grid, kPoolThreads, 0, s>>>(x, frames, nb, g, out);
   return cudaGetLastError();
 }
 
+cudaError_t launch_pool(const __nv_bfloat16* x, int frames, int nb, const Geo& g, float* out,
+                        cudaStream_t s, int mode = kPoolMean) {
+  return g.D == 128 ? launch_pool_d<128>(x, frames, nb, g, mode, out, s)
+                    : launch_pool_d<64>(x, frames, nb, g, mode, out, s);
+}
+
+// query rows per CTA: the largest of 32 / 16 / 8 whose tiles and score rows (QT * NBk * 4
+// bytes) fit the 227 KB of shared memory a CTA may have; 0 if none does
 int select_rows_per_cta(const Geo& g) {
-  // keep shared memory under ~200 KB: scores take QT * NBk * 4 bytes
   for (int qt : {32, 16, 8}) {
     size_t bytes = (size_t)(qt + kKT) * (g.D + 4) * 4 + (size_t)qt * g.NBk * 4 + 8 * 256 * 4;
-    if (bytes <= 200 * 1024) return qt;
+    if (bytes <= 227 * 1024) return qt;
   }
   return 0;
 }
@@ -255,7 +294,7 @@ size_t select_smem_bytes(const Geo& g, int qt) {
 template <int D, int RPT>
 static cudaError_t launch_sel_t(const SelectArgs& a, cudaStream_t s) {
   const Geo& g = a.g;
-  dim3 grid((g.NBq + a.qt - 1) / a.qt, g.H, g.B);
+  dim3 grid((g.NBq + a.qt - 1) / a.qt, (a.flags & kRouteSharedHeads) ? 1 : g.H, g.B);
   size_t smem = select_smem_bytes(g, a.qt);
   cudaError_t e = cudaFuncSetAttribute(score_select_kernel<D, RPT>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -47,6 +47,8 @@ extern "C" BSA_API bsa_status_t bsa_route_noalloc(const bsa_geom_t* gi, int32_t 
   for (const void* p : ptrs)
     if (p && !aligned(p, 16)) return fail(BSA_ERR_INVALID_ARG, "inputs must be 16-byte aligned");
   const RouteWs w = route_ws(g);
+  if (select_rows_per_cta(g) == 0)
+    return fail(BSA_ERR_UNSUPPORTED, "%d key blocks do not fit the select kernel", g.NBk);
   if (w.total > kNoallocScratchBytes)
     return fail(BSA_ERR_UNSUPPORTED,
                 "bsa_route_noalloc needs %zu scratch bytes but holds %zu (B*H*NBq*D*8 must not "

@@ -9,9 +9,10 @@ from typing import Dict, Optional
 
 import torch
 
-from . import (WS_BWD, WS_PROLOGUE_BWD, WS_ROUTE, Geometry, blocked_shape, bsa_attn_bwd,
-               bsa_attn_fwd, bsa_cache_append, bsa_route, bsa_workspace_size,
-               rope3d_qknorm_prologue, rope3d_qknorm_prologue_bwd)
+from . import (POOL_MAX, POOL_SUM, ROUTE_POOL_MAX, ROUTE_POOL_SUM, WS_BWD, WS_PROLOGUE_BWD,
+               WS_ROUTE, Geometry, blocked_shape, bsa_attn_bwd, bsa_attn_fwd, bsa_block_pool,
+               bsa_cache_append, bsa_route_ex, bsa_workspace_size, rope3d_qknorm_prologue,
+               rope3d_qknorm_prologue_bwd)
 
 
 class BsaPipeline:
@@ -26,6 +27,7 @@ class BsaPipeline:
                  qknorm: bool = True, eps: float = 1e-6, with_bwd: bool = False,
                  device: str = "cuda"):
         self.g, self.r, self.theta, self.eps, self.qknorm = g, top_r, rope_theta, eps, qknorm
+        self.route_flags = 0  # ROUTE_* variant used by forward()
         dev = torch.device(device)
         bf = dict(dtype=torch.bfloat16, device=dev)
         shp = blocked_shape(g)
@@ -95,10 +97,19 @@ class BsaPipeline:
                                self.gamma_k if self.qknorm else None, self.eps, self.theta,
                                self.q, self.k, self.v, self.q_pool, self.k_pool, stream=stream)
 
-    def route(self, stream=None, use_pools: bool = True):
-        bsa_route(self.g, self.r, self.q, self.k, self.q_pool if use_pools else None,
-                  self.k_pool if use_pools else None, self.kc_pool, self.idx, self.cnt,
-                  self.ws_route, stream=stream)
+    def route(self, stream=None, use_pools: bool = True, flags: int = 0):
+        """Top-r routing into idx / cnt.  ``flags``: ROUTE_* variants.  A pooling variant pools
+        q / k (and the cache's keys) itself instead of using the prologue's block means."""
+        kc_pool = self.kc_pool
+        pool_mode = POOL_SUM if flags & ROUTE_POOL_SUM else POOL_MAX if flags & ROUTE_POOL_MAX else 0
+        if pool_mode:
+            use_pools = False
+            if self.kc is not None:
+                kc_pool = torch.empty_like(self.kc_pool)
+                bsa_block_pool(self.g, self.g.cached_t, pool_mode, self.kc, kc_pool, stream=stream)
+        bsa_route_ex(self.g, self.r, flags, self.q, self.k, self.q_pool if use_pools else None,
+                     self.k_pool if use_pools else None, kc_pool, self.idx, self.cnt,
+                     self.ws_route, stream=stream)
 
     def attn_fwd(self, stream=None):
         bsa_attn_fwd(self.g, self.r, self.q, self.k, self.v, self.kc, self.vc, self.idx,
@@ -106,7 +117,7 @@ class BsaPipeline:
 
     def forward(self, q_raster, k_raster, v_raster, stream=None) -> Dict[str, torch.Tensor]:
         self.prologue(q_raster, k_raster, v_raster, stream)
-        self.route(stream)
+        self.route(stream, flags=self.route_flags)
         self.attn_fwd(stream)
         return {"o": self.o, "lse": self.lse, "idx": self.idx, "cnt": self.cnt}
 

@@ -175,6 +175,39 @@ BSA_API bsa_status_t bsa_route(const bsa_geom_t* g, int32_t top_r, const void* q
                        const float* kpool_cache, int32_t* idx, int32_t* cnt, void* ws,
                        size_t ws_bytes, bsa_stream_t stream);
 
+/* Routing variants for bsa_route_ex (bit flags).  The pages leave the routing rule open
+ * ("LongCat-Video : Generate 1 minute long AI videos with this model", section "Sparse
+ * attention", likens a block to one that always sits with its own table plus the meaningful
+ * neighbouring ones); these are the variants of that reading.
+ *   BSA_ROUTE_FORCE_SELF   every query block i keeps its own key block NBc + i; the other
+ *                          top_r - 1 places go to the best of the rest (same tie rule).
+ *   BSA_ROUTE_SHARED_HEADS key blocks ranked by s_ij = sum_h qbar_hi . kbar_hj; every head of
+ *                          (b, i) gets that one selection (idx/cnt rows identical across h).
+ *   BSA_ROUTE_POOL_SUM     block vectors are sums over the valid tokens (not means).
+ *   BSA_ROUTE_POOL_MAX     block vectors are channel-wise maxima over the valid tokens.
+ * A pooling flag pools q_blk / k_blk itself (q_pool / k_pool must be NULL, ws required);
+ * kpool_cache must then hold the cached key blocks pooled the same way (bsa_block_pool). */
+#define BSA_ROUTE_FORCE_SELF 1u
+#define BSA_ROUTE_SHARED_HEADS 2u
+#define BSA_ROUTE_POOL_SUM 4u
+#define BSA_ROUTE_POOL_MAX 8u
+/* bsa_route with variant flags (0 = bsa_route).  Unknown bits or both pooling flags:
+ * BSA_ERR_INVALID_ARG. */
+BSA_API bsa_status_t bsa_route_ex(const bsa_geom_t* g, int32_t top_r, uint32_t flags,
+                                  const void* q_blk, const void* k_blk, const float* q_pool,
+                                  const float* k_pool, const float* kpool_cache, int32_t* idx,
+                                  int32_t* cnt, void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Block pooling of a blocked bf16 tensor x_blk [B, H, NB, BS, D] over `frames` frames
+ * (NB = ceil(frames / blk_t) * NBh * NBw) into out fp32 [B, H, NB, D]: the mean
+ * (BSA_POOL_MEAN), sum (BSA_POOL_SUM) or channel-wise maximum (BSA_POOL_MAX) over each
+ * block's valid tokens (pad slots excluded).  Used to pool a cache for a pooling variant. */
+#define BSA_POOL_MEAN 0
+#define BSA_POOL_SUM 1
+#define BSA_POOL_MAX 2
+BSA_API bsa_status_t bsa_block_pool(const bsa_geom_t* g, int32_t frames, int32_t mode,
+                                    const void* x_blk, float* out, bsa_stream_t stream);
+
 /* Sparse attention forward over the selected blocks (tcgen05 tensor cores, TMA).
  * Source: "LongCat-Video视频生成模型发布…", section 块稀疏注意力（BSA）.
  * For every (b, h, query block i) and valid query slot:

@@ -129,3 +129,23 @@ def test_cache_append_host_validation():
     with pytest.raises(bsa.BsaError) as ei:  # misaligned output
         bsa.bsa_cache_append(g, 16, 16, 16, 16, 16, 16, 24, 16, 16, stream=0)
     assert ei.value.code == 1
+
+
+def test_route_variant_host_validation():
+    g = _g()
+    args = (16, 16, None, None, None, 16, 16, 16)
+    with pytest.raises(bsa.BsaError) as ei:  # unknown flag bit
+        bsa.bsa_route_ex(g, 4, 16, *args, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # two pooling modes
+        bsa.bsa_route_ex(g, 4, bsa.ROUTE_POOL_SUM | bsa.ROUTE_POOL_MAX, *args, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # a pooling variant cannot take the prologue's means
+        bsa.bsa_route_ex(g, 4, bsa.ROUTE_POOL_MAX, 16, 16, 16, 16, None, 16, 16, 16, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # unknown pooling mode
+        bsa.bsa_block_pool(g, 24, 3, 16, 16, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:
+        bsa.bsa_block_pool(g, 0, bsa.POOL_MAX, 16, 16, stream=0)
+    assert ei.value.code == 1
