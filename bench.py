@@ -51,7 +51,7 @@ KERNEL_NAMES = {"fwd": "bsa_fwd_kernel", "bwd_dkdv": "bsa_bwd_dkdv_kernel",
 # selected block pair (fwd, dq) or a pair with a current key block (dkdv).  Traffic grows with
 # the pairs a launch processes, so a full launch is scaled from it.  None = not captured for
 # the kernel as it now stands.
-DRAM_BYTES_PER_PAIR = {"fwd": 3854, "bwd_dkdv": 5764, "bwd_dq": None}
+DRAM_BYTES_PER_PAIR = {"fwd": 3854, "bwd_dkdv": 5764, "bwd_dq": 4842}
 
 
 def traffic_per_launch(kernel, workload, n_pairs, n_pairs_cur):
@@ -411,6 +411,25 @@ def main():
                                      "gbs": c_bytes / (c_ms * 1e-3) / 1e9,
                                      "cached_t": gc.cached_t}
         del kc_n, vc_n, kp_n
+
+    # routing variants (bsa_route_ex flags) on this workload's q / k: ms per route call
+    rv = {}
+    for vname, vflags in (("plain", 0), ("force_self", bsa.ROUTE_FORCE_SELF),
+                          ("shared_heads", bsa.ROUTE_SHARED_HEADS),
+                          ("pool_sum", bsa.ROUTE_POOL_SUM), ("pool_max", bsa.ROUTE_POOL_MAX)):
+        for _ in range(2):
+            pipe.route(stream, flags=vflags)
+        torch.cuda.synchronize()
+        r0 = torch.cuda.Event(enable_timing=True)
+        r1 = torch.cuda.Event(enable_timing=True)
+        r0.record(stream)
+        for _ in range(args.steps):
+            pipe.route(stream, flags=vflags)
+        r1.record(stream)
+        torch.cuda.synchronize()
+        rv[vname] = r0.elapsed_time(r1) / args.steps
+    pipe.route(stream)  # leave the plain selection in place
+    next_rows["route_variants_ms"] = rv
 
     peaks = load_peaks()
     peak = peaks["bf16_tflops_sustained"]
