@@ -123,7 +123,7 @@ def cpu_oracle_sample(w, budget_s: float = 12.0):
     one head plus forward attention of as many query blocks of that head as fit the budget,
     and backward of a few; reported in TFLOP/s of the same tile-FLOP convention."""
     import oracle
-    grid = oracle.Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t)
+    grid = oracle.Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t, w.cond_t)
     x = make_raster_inputs(w, with_grad=True)
     from synth import bf16_bits_to_f64
     h = 0

@@ -45,7 +45,7 @@ class _Geom(ctypes.Structure):
                 ("t_frames", ctypes.c_int32), ("grid_h", ctypes.c_int32), ("grid_w", ctypes.c_int32),
                 ("cached_t", ctypes.c_int32), ("blk_t", ctypes.c_int32), ("blk_h", ctypes.c_int32),
                 ("blk_w", ctypes.c_int32), ("causal_chunk_t", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float)]
+                ("softmax_scale", ctypes.c_float), ("cond_t", ctypes.c_int32)]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -61,11 +61,12 @@ class Geometry:
     cached_t: int = 0
     causal_chunk_t: int = 0
     softmax_scale: float = 0.0
+    cond_t: int = 0
 
     def c(self) -> _Geom:
         return _Geom(self.batch, self.heads, self.head_dim, self.t_frames, self.grid_h,
                      self.grid_w, self.cached_t, self.blk[0], self.blk[1], self.blk[2],
-                     self.causal_chunk_t, float(self.softmax_scale))
+                     self.causal_chunk_t, float(self.softmax_scale), self.cond_t)
 
     @property
     def bs(self) -> int:
@@ -90,7 +91,7 @@ class Geometry:
     @classmethod
     def from_workload(cls, w) -> "Geometry":
         return cls(w.batch, w.heads, w.head_dim, w.t_frames, w.grid_h, w.grid_w, tuple(w.blk),
-                   w.cached_t, w.chunk_t)
+                   w.cached_t, w.chunk_t, cond_t=getattr(w, "cond_t", 0))
 
 
 def blocked_shape(g: Geometry, frames: Optional[int] = None):

@@ -104,6 +104,8 @@ bsa_status_t make_geo(const bsa_geom_t* gi, Geo* out) {
   if (a.causal_chunk_t < 0 || (a.causal_chunk_t && a.causal_chunk_t % a.blk_t))
     return fail(BSA_ERR_INVALID_ARG, "causal_chunk_t %d must be 0 or a multiple of blk_t",
                 a.causal_chunk_t);
+  if (a.cond_t < 0 || a.cond_t % a.blk_t)
+    return fail(BSA_ERR_INVALID_ARG, "cond_t %d must be >= 0 and a multiple of blk_t", a.cond_t);
   if (!(a.softmax_scale >= 0.f) || std::isinf(a.softmax_scale))
     return fail(BSA_ERR_INVALID_ARG, "softmax_scale must be finite and >= 0");
   Geo g;
@@ -127,6 +129,7 @@ bsa_status_t make_geo(const bsa_geom_t* gi, Geo* out) {
     return fail(BSA_ERR_UNSUPPORTED, "problem too large for 32-bit TMA row coordinates");
   g.NBq = (int)nbq; g.NBc = (int)nbc; g.NBk = (int)(nbq + nbc);
   g.chunk = a.causal_chunk_t;
+  g.cond = a.cond_t;
   g.scale = a.softmax_scale > 0.f ? a.softmax_scale : 1.0f / std::sqrt((float)a.head_dim);
   *out = g;
   return BSA_OK;

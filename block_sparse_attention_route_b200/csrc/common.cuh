@@ -28,6 +28,7 @@ struct Geo {
   int nbt_q, nbt_c;     // blocks along t for current / cached frames
   int NBq, NBc, NBk;    // query blocks, cached key blocks, all key blocks
   int chunk;            // causal chunk in frames (0 = none)
+  int cond;             // frames of the conditioning segment (0 = none)
   float scale;          // softmax scale
 };
 
@@ -49,6 +50,12 @@ __host__ __device__ inline int key_block_t0(const Geo& g, int j) {
 }
 __host__ __device__ inline int query_block_t0(const Geo& g, int i) {
   return g.Tc + (i / (g.nbh * g.nbw)) * g.bt;
+}
+// Mask segment of absolute frame t: key block j is allowed for query block i iff
+// frame_segment(t0(j)) <= frame_segment(t0(i)); only meaningful when g.chunk or g.cond is set.
+__host__ __device__ inline int frame_segment(const Geo& g, int t) {
+  if (t < g.cond) return 0;
+  return 1 + (g.chunk ? (t - g.cond) / g.chunk : 0);
 }
 
 // ------------------------------------------------------------------ small helpers

@@ -9,7 +9,8 @@
 //                    channel-wise max are the pooling variants.
 // score_select     : s_ij = qbar_i . kbar_j in fp32 on CUDA cores (ranking needs fp32, the
 //                    work is ~NBq*NBk*D FMAs per head, tiny next to the attention), masked
-//                    to -inf by the block-causal rule, then an exact warp-level radix select
+//                    to -inf by the block-causal rule (causal chunks and / or the two-segment
+//                    conditioning form), then an exact warp-level radix select
 //                    of the top r per row on order-preserving 32-bit keys, ties resolved to
 //                    the lower block index, emitted in ascending block order.
 // Variants (the pages leave the routing rule open): the own key block NBc + i forced into
@@ -157,13 +158,14 @@ __global__ void __launch_bounds__(kSelThreads) score_select_kernel(const SelectA
     for (int x = 0; x < RPT; ++x) {
       const int ii = ti * RPT + x, i = i0 + ii;
       if (ii >= nq) continue;
-      const int ci = g.chunk ? query_block_t0(g, i) / g.chunk : 0;
+      const bool masked = g.chunk || g.cond;
+      const int ci = masked ? frame_segment(g, query_block_t0(g, i)) : 0;
 #pragma unroll
       for (int m = 0; m < 4; ++m) {
         const int j = j0 + tj + 32 * m;
         if (j >= g.NBk) continue;
         bool ok = true;
-        if (g.chunk) ok = key_block_t0(g, j) / g.chunk <= ci;
+        if (masked) ok = frame_segment(g, key_block_t0(g, j)) <= ci;
         // a key block always holds >= 1 valid token when the grid is padded to whole blocks;
         // the own block (same frames, so never masked) ranks above every finite score
         float v = ok ? acc[x][m] : -INFINITY;

@@ -50,7 +50,7 @@
 extern "C" {
 #endif
 
-#define BSA_ABI_VERSION 1
+#define BSA_ABI_VERSION 2
 
 #if defined(__GNUC__)
 #define BSA_API __attribute__((visibility("default")))
@@ -71,7 +71,7 @@ typedef enum bsa_status {
 } bsa_status_t;
 
 /* Geometry of one problem.  Supported: head_dim in {64, 128}; blk_t*blk_h*blk_w in {32, 128};
- * cached_t and causal_chunk_t multiples of blk_t. */
+ * cached_t, causal_chunk_t and cond_t multiples of blk_t. */
 typedef struct bsa_geom {
   int32_t batch;          /* B */
   int32_t heads;          /* H */
@@ -82,10 +82,17 @@ typedef struct bsa_geom {
   int32_t cached_t;       /* leading latent frames whose K/V come from the cache (0 = none);
                              current frame f sits at absolute frame cached_t + f */
   int32_t blk_t, blk_h, blk_w; /* 3D block shape */
-  int32_t causal_chunk_t; /* 0 = no mask; else key block j is allowed for query block i iff
-                             floor(t0(j)/C) <= floor(t0(i)/C), t0 = first absolute frame */
+  int32_t causal_chunk_t; /* C: 0 = no causal chunks */
   float softmax_scale;    /* logits = q.k * scale; 0 selects 1/sqrt(head_dim) */
+  int32_t cond_t;         /* leading absolute frames of the conditioning segment (0 = none) */
 } bsa_geom_t;
+/* Block-causal mask (applied by the routing): with t0 the first absolute frame of a block and
+ * seg(t) = 0 for t < cond_t, else 1 + (C ? floor((t - cond_t) / C) : 0), key block j is allowed
+ * for query block i iff seg(t0(j)) <= seg(t0(i)).  cond_t = 0 gives plain chunks
+ * floor(t/C); C = 0 with cond_t > 0 gives the two-segment form of the continuation task
+ * (conditioning frames attend only among themselves, the frames to generate attend to all;
+ * "LongCat-Video 高效長視頻生成探索世界模型的第壹步", section 2.1, Block-Causal attention);
+ * both 0: no mask.  cond_t must be a multiple of blk_t. */
 
 enum { BSA_WS_ROUTE = 1, BSA_WS_FWD = 2, BSA_WS_BWD = 3, BSA_WS_PROLOGUE_BWD = 4 };
 

@@ -55,7 +55,13 @@ class Grid:
     ``t_frames`` current frames (query tokens and current key tokens); ``cached_t`` leading
     frames whose keys and values come from a cache (absolute frames 0..cached_t-1, the
     current frames follow at cached_t..); ``blk`` = (bt, bh, bw); ``chunk_t`` = block-causal
-    chunk length in frames (0 = no mask).
+    chunk length in frames (0 = no chunks); ``cond_t`` = leading absolute frames of the
+    conditioning segment (0 = none).  Block-causal rule (the Meituan talk, section 2.1): a
+    frame's segment is 0 inside the conditioning frames and 1 + (frames past them) // chunk_t
+    after them (1 when chunk_t = 0); a query block may use a key block whose first frame lies
+    in the same or an earlier segment.  So chunk_t alone gives plain causal chunks, cond_t
+    alone the two-segment form (conditioning frames see only themselves, the frames being
+    generated see everything).
     """
     t_frames: int
     grid_h: int
@@ -63,6 +69,7 @@ class Grid:
     blk: Tuple[int, int, int]
     cached_t: int = 0
     chunk_t: int = 0
+    cond_t: int = 0
 
     def __post_init__(self):
         bt = self.blk[0]
@@ -70,6 +77,17 @@ class Grid:
             raise ValueError("cached frames must be a whole number of block frames")
         if self.chunk_t and self.chunk_t % bt:
             raise ValueError("causal chunk must be a whole number of block frames")
+        if self.cond_t % bt:
+            raise ValueError("conditioning frames must be a whole number of block frames")
+
+    @property
+    def masked(self) -> bool:
+        return bool(self.chunk_t or self.cond_t)
+
+    def frame_segment(self, t: int) -> int:
+        if t < self.cond_t:
+            return 0
+        return 1 + ((t - self.cond_t) // self.chunk_t if self.chunk_t else 0)
 
     @property
     def nbt(self) -> int:
@@ -135,17 +153,18 @@ class Grid:
         return out
 
     def query_block_chunk(self, i: int) -> int:
-        """Causal chunk of query block i (its first absolute frame // chunk_t)."""
+        """Mask segment of query block i (of its first absolute frame)."""
         t0 = self.cached_t + (i // (self.nbh * self.nbw)) * self.blk[0]
-        return t0 // self.chunk_t
+        return self.frame_segment(t0)
 
     def key_block_chunk(self, j: int) -> int:
+        """Mask segment of global key block j (cached blocks first)."""
         per_t = self.nbh * self.nbw
         if j < self.nbc:
             t0 = (j // per_t) * self.blk[0]
         else:
             t0 = self.cached_t + ((j - self.nbc) // per_t) * self.blk[0]
-        return t0 // self.chunk_t
+        return self.frame_segment(t0)
 
 
 # ----------------------------------------------------------------------------------------
@@ -302,7 +321,7 @@ def block_scores(qbar: np.ndarray, kbar: np.ndarray, grid: Grid,
     """s[b, h, i, j] = qbar_i . kbar_j (unscaled), -inf where the block-causal rule forbids
     key block j for query block i or key block j holds no valid token."""
     s = np.einsum("bhid,bhjd->bhij", qbar, kbar)
-    if grid.chunk_t:
+    if grid.masked:
         allowed = np.array([[grid.key_block_chunk(j) <= grid.query_block_chunk(i)
                              for j in range(grid.nbk)] for i in range(grid.nbq)])
         s = np.where(allowed[None, None], s, NEG_INF)

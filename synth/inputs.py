@@ -26,7 +26,8 @@ class Workload:
     ``t_frames`` latent frames of current tokens (queries and current keys) on a
     ``grid_h`` x ``grid_w`` grid; ``cached_t`` leading frames whose keys/values come from a
     cache; ``blk`` the 3D block (t, h, w); ``top_r`` key blocks kept per query block;
-    ``chunk_t`` the block-causal chunk in frames (0 = no mask).
+    ``chunk_t`` the block-causal chunk in frames (0 = no chunks); ``cond_t`` the leading
+    conditioning frames of the two-segment block-causal form (0 = none).
     """
     name: str
     batch: int
@@ -44,6 +45,7 @@ class Workload:
     theta: float = 10000.0
     eps: float = 1e-6
     unit_gamma: bool = True
+    cond_t: int = 0
 
     @property
     def n_tokens(self) -> int:

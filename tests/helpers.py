@@ -7,7 +7,7 @@ from synth import bf16_bits_to_f64
 
 
 def grid_of(w):
-    return oracle.Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t)
+    return oracle.Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t, w.cond_t)
 
 
 def to_dev(bits, device="cuda"):

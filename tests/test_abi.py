@@ -23,7 +23,7 @@ def test_library_exports_every_declared_symbol():
     L = bsa.lib()
     for n in names:
         assert hasattr(L, n), n
-    assert L.bsa_abi_version() == 1
+    assert L.bsa_abi_version() == 2
 
 
 def test_error_strings():
@@ -52,7 +52,7 @@ def test_workspace_sizes_720p():
 
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(blk=(4, 4, 4)), dict(cached_t=3),
-                                 dict(causal_chunk_t=6), dict(batch=0), dict(grid_w=0),
+                                 dict(causal_chunk_t=6), dict(cond_t=6), dict(cond_t=-4), dict(batch=0), dict(grid_w=0),
                                  dict(softmax_scale=-1.0)])
 def test_bad_geometry_rejected_on_host(bad):
     g = _g(**bad)

@@ -20,7 +20,7 @@ pytestmark = pytest.mark.filterwarnings("ignore::UserWarning")
 
 
 def _grid(w):
-    return Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t)
+    return Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t, w.cond_t)
 
 
 def _inputs(name):
@@ -159,7 +159,7 @@ def _brute_route(q, k, grid, r):
                 sc = []
                 for j in range(grid.nbk):
                     s = sum(means[0][i][d] * means[1][j][d] for d in range(D))
-                    if grid.chunk_t and grid.key_block_chunk(j) > grid.query_block_chunk(i):
+                    if grid.masked and grid.key_block_chunk(j) > grid.query_block_chunk(i):
                         s = -math.inf
                     sc.append(s)
                 chosen = []
@@ -538,7 +538,7 @@ def _brute_variant(q, k, grid, r, pool, force_self, shared):
         for hh, sc in enumerate(per_head):
             for i in range(grid.nbq):
                 allowed = [j for j in range(grid.nbk)
-                           if not (grid.chunk_t and grid.key_block_chunk(j) > grid.query_block_chunk(i))]
+                           if not (grid.masked and grid.key_block_chunk(j) > grid.query_block_chunk(i))]
                 must = [i] if force_self else []
                 rest = [j for j in allowed if j not in must]
                 m = min(r, len(allowed)) - len(must)
@@ -640,3 +640,60 @@ def test_sum_pooling_ranks_like_mean_on_whole_blocks_and_penalises_partial_ones(
         a = np.argsort(-sm[0, 0, i, whole], kind="stable")
         b = np.argsort(-ss[0, 0, i, whole], kind="stable")
         assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------------ two-segment block-causal mask
+def test_two_segment_mask_brute_force():
+    """Conditioning frames [0, cond_t) see only themselves; later frames see everything.  The
+    allowed set is written here from that sentence alone (no segment function)."""
+    g = Grid(8, 4, 8, (2, 4, 4), cond_t=4)  # 4 block-frames x 2 blocks; blocks 0-3 conditioning
+    rng = np.random.default_rng(21)
+    q = rng.standard_normal((1, 8 * 32, 1, 8))
+    k = rng.standard_normal((1, 8 * 32, 1, 8))
+    r = 3
+    idx, cnt, s = oracle.route(q, k, g, r)
+    mem = g.block_members(8)
+    t0 = [min(t // 32 for t in m) for m in mem]  # first frame of each block (32 tokens per frame)
+    qbar = [q[0, m, 0].mean(axis=0) for m in mem]
+    kbar = [k[0, m, 0].mean(axis=0) for m in mem]
+    for i in range(g.nbq):
+        allowed = [j for j in range(g.nbk) if t0[i] >= 4 or t0[j] < 4]
+        sc = {j: float(qbar[i] @ kbar[j]) for j in allowed}
+        best = sorted(sorted(allowed, key=lambda j: (-sc[j], j))[:r])
+        assert list(idx[0, 0, i, :cnt[0, 0, i]]) == best
+        assert all(np.isneginf(s[0, 0, i, j]) for j in range(g.nbk) if j not in allowed)
+    assert list(cnt[0, 0]) == [3, 3, 3, 3, 3, 3, 3, 3] and set(idx[0, 0, 0]) <= {0, 1, 2, 3}
+
+
+def test_two_segment_conditioning_rows_ignore_the_generated_frames():
+    """Changing the frames after cond_t changes nothing for the conditioning rows, which equal
+    a plain run over the conditioning frames alone; with chunk = cond_t = half the frames the
+    form equals two causal chunks."""
+    w, x = _inputs("small")  # 8 frames, 10 x 20 grid, blocks 4x4x8
+    g = Grid(8, 10, 20, (4, 4, 8), cond_t=4)
+    scale = 1.0 / math.sqrt(w.head_dim)
+    idx, cnt, _ = oracle.route(x["q"], x["k"], g, w.top_r)
+    o, lse = oracle.attend(x["q"], x["k"], x["v"], idx, g, scale)
+    ncond = 4 * 10 * 20
+    q2, k2, v2 = (a.copy() for a in (x["q"], x["k"], x["v"]))
+    rng = np.random.default_rng(4)
+    for a in (q2, k2, v2):
+        a[:, ncond:] = rng.standard_normal(a[:, ncond:].shape)
+    idx2, _, _ = oracle.route(q2, k2, g, w.top_r)
+    o2, _ = oracle.attend(q2, k2, v2, idx2, g, scale)
+    per_t = g.nbh * g.nbw
+    assert np.array_equal(idx[:, :, :per_t], idx2[:, :, :per_t])
+    np.testing.assert_array_equal(o[:, :ncond], o2[:, :ncond])
+    gc = Grid(4, 10, 20, (4, 4, 8))
+    sl = (slice(None), slice(0, ncond))
+    idc, _, _ = oracle.route(x["q"][sl], x["k"][sl], gc, w.top_r)
+    assert np.array_equal(idc, idx[:, :, :per_t])
+    oc, lsec = oracle.attend(x["q"][sl], x["k"][sl], x["v"][sl], idc, gc, scale)
+    np.testing.assert_allclose(oc, o[:, :ncond], atol=1e-13)
+    np.testing.assert_allclose(lsec, lse[:, :ncond], atol=1e-13)
+    gchunk = Grid(8, 10, 20, (4, 4, 8), chunk_t=4)
+    idk, _, _ = oracle.route(x["q"], x["k"], gchunk, w.top_r)
+    assert np.array_equal(idk, idx)
+    # the generated frames' rows are routed as without any mask
+    idn, _, _ = oracle.route(x["q"], x["k"], Grid(8, 10, 20, (4, 4, 8)), w.top_r)
+    assert np.array_equal(idn[:, :, per_t:], idx[:, :, per_t:])
