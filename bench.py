@@ -54,6 +54,25 @@ KERNEL_NAMES = {"fwd": "bsa_fwd_kernel", "bwd_dkdv": "bsa_bwd_dkdv_kernel",
 DRAM_BYTES_PER_PAIR = {"fwd": 3854, "bwd_dkdv": 5764, "bwd_dq": 4842}
 
 
+def block_token_counts(g, frames: int) -> np.ndarray:
+    """Valid tokens of each block of a `frames` x grid_h x grid_w grid (blocks t-major)."""
+    bt, bh, bw = g.blk
+    nbt, nbh, nbw = -(-frames // bt), -(-g.grid_h // bh), -(-g.grid_w // bw)
+    vt = np.minimum(bt, frames - bt * np.arange(nbt))
+    vh = np.minimum(bh, g.grid_h - bh * np.arange(nbh))
+    vw = np.minimum(bw, g.grid_w - bw * np.arange(nbw))
+    return (vt[:, None, None] * vh[None, :, None] * vw[None, None, :]).reshape(-1)
+
+
+def valid_token_flops(g, idx: np.ndarray, cnt: np.ndarray) -> float:
+    """Forward FLOPs counting valid tokens only: sum over selected pairs of 4 D n_i n_j."""
+    nq = block_token_counts(g, g.t_frames).astype(np.float64)
+    nk = nq if not g.cached_t else np.concatenate([block_token_counts(g, g.cached_t), nq])
+    sel = np.arange(idx.shape[-1])[None, None, None, :] < cnt[..., None]
+    nj = np.where(sel, nk[np.clip(idx, 0, None)], 0.0).sum(axis=-1)  # [B, H, NBq]
+    return float(4.0 * g.head_dim * (nj * nq[None, None, :]).sum())
+
+
 def traffic_per_launch(kernel, workload, n_pairs, n_pairs_cur):
     b = DRAM_BYTES_PER_PAIR.get(kernel)
     if b is None:
@@ -273,6 +292,7 @@ def main():
     n_pairs_cur = int(((pipe.idx >= g.nbc) & sel).sum().item())  # pairs with a current key block
     fl_fwd = tile_flops(g.bs, g.head_dim, n_pairs)
     fl_step = fl_fwd * (3.5 if with_bwd else 1.0)
+    fl_fwd_valid = valid_token_flops(g, pipe.idx.cpu().numpy(), pipe.cnt.cpu().numpy())
 
     barrier()
     torch.cuda.synchronize()
@@ -457,6 +477,7 @@ def main():
         "config": {"workload": args.workload, "tokens": w.n_tokens, "padded_tokens": g.nbq * g.bs,
                    "heads": w.heads, "head_dim": w.head_dim, "block": list(w.blk),
                    "top_r": w.top_r, "selected_pairs": n_pairs, "with_bwd": with_bwd,
+                   "fwd_tflop_tiles": fl_fwd / 1e12, "fwd_tflop_valid_tokens": fl_fwd_valid / 1e12,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (126 MB)"},
         "ms_per_call": parts,
         "kernels": kernels,

@@ -122,3 +122,10 @@ def test_kernel_timing_counts_each_attention_launch():
         bsa.bsa_kernel_timing(False)
     assert {k: n for k, (n, _) in t.items()} == {"fwd": 1, "bwd_dkdv": 1, "bwd_dq": 1}
     assert all(ms > 0 for _, ms in t.values())
+
+
+def test_backward_two_segment_mask():
+    from synth import Workload
+    w = Workload("two_segment", 1, 2, 128, 12, 10, 20, (4, 4, 8), 5, rope=True, cond_t=4)
+    pipe, x = run_fwd_bwd(w)
+    check_bwd(w, pipe, x, [0, 1])

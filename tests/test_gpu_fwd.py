@@ -278,3 +278,21 @@ def test_bounded_wait_times_out_and_context_survives(torch_cuda):
     w = WORKLOADS["tiny"]
     pipe, _ = run_forward(w)
     check_attention(w, pipe, [0, 1])
+
+
+@pytest.mark.parametrize("cond_t,chunk_t", [(4, 0), (4, 4), (8, 0)])
+def test_two_segment_mask(torch_cuda, cond_t, chunk_t):
+    """Conditioning frames [0, cond_t) attend only among themselves; the frames after them
+    attend to everything (or, with chunk_t, to their own and earlier chunks)."""
+    from synth import Workload
+    w = Workload("two_segment", 1, 2, 128, 12, 10, 20, (4, 4, 8), 5, chunk_t=chunk_t, rope=True,
+                 cond_t=cond_t)
+    pipe, _ = run_forward(w)
+    grid = grid_of(w)
+    idx = pipe.idx.cpu().numpy()
+    per_t = grid.nbh * grid.nbw
+    n_cond = (cond_t // 4) * per_t
+    assert np.all(idx[:, :, :n_cond] < n_cond)  # conditioning rows never see later blocks
+    assert np.any(idx[:, :, n_cond:] >= n_cond)
+    assert check_route(w, pipe, [0, 1]) == 0
+    check_attention(w, pipe, [0, 1])
