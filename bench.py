@@ -36,7 +36,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from synth import WORKLOADS, make_raster_inputs  # noqa: E402
+from synth import WORKLOADS, add_smooth_field, make_raster_inputs  # noqa: E402
 
 
 def tile_flops(bs: int, d: int, n_pairs: int) -> float:
@@ -71,6 +71,19 @@ def valid_token_flops(g, idx: np.ndarray, cnt: np.ndarray) -> float:
     sel = np.arange(idx.shape[-1])[None, None, None, :] < cnt[..., None]
     nj = np.where(sel, nk[np.clip(idx, 0, None)], 0.0).sum(axis=-1)  # [B, H, NBq]
     return float(4.0 * g.head_dim * (nj * nq[None, None, :]).sum())
+
+
+def selection_locality(g, idx: np.ndarray, cnt: np.ndarray) -> float:
+    """Share of selected key blocks within one block (t, h or w) of their query block."""
+    per_t = -(-g.grid_h // g.blk[1]) * -(-g.grid_w // g.blk[2])
+    nbw = -(-g.grid_w // g.blk[2])
+    nbc = (g.cached_t // g.blk[0]) * per_t
+    sel = np.arange(idx.shape[-1])[None, None, None, :] < cnt[..., None]
+    i = np.arange(idx.shape[2])[None, None, :, None] + nbc  # global position of the query block
+    j = np.clip(idx, 0, None)
+    d = np.maximum(np.abs(i // per_t - j // per_t),
+                   np.maximum(np.abs((i % per_t) // nbw - (j % per_t) // nbw), np.abs(i % nbw - j % nbw)))
+    return float(((d <= 1) & sel).sum() / max(1, sel.sum()))
 
 
 def traffic_per_launch(kernel, workload, n_pairs, n_pairs_cur):
@@ -193,6 +206,8 @@ def main():
     ap.add_argument("--workload", default="720p", choices=["720p", "480p", "480p_cont"])
     ap.add_argument("--no-bwd", action="store_true", help="forward path only")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--structured", action="store_true",
+                    help="q and k share a smooth low-frequency field (video-like routing locality)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -242,6 +257,8 @@ def main():
 
     g = bsa.Geometry.from_workload(w)
     x = make_raster_inputs(w, with_grad=with_bwd, seed_offset=0)
+    if args.structured:
+        x = add_smooth_field(w, x)
 
     def dev_bf16(a):
         return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
@@ -292,7 +309,9 @@ def main():
     n_pairs_cur = int(((pipe.idx >= g.nbc) & sel).sum().item())  # pairs with a current key block
     fl_fwd = tile_flops(g.bs, g.head_dim, n_pairs)
     fl_step = fl_fwd * (3.5 if with_bwd else 1.0)
-    fl_fwd_valid = valid_token_flops(g, pipe.idx.cpu().numpy(), pipe.cnt.cpu().numpy())
+    idx_h, cnt_h = pipe.idx.cpu().numpy(), pipe.cnt.cpu().numpy()
+    fl_fwd_valid = valid_token_flops(g, idx_h, cnt_h)
+    locality = selection_locality(g, idx_h, cnt_h)
 
     barrier()
     torch.cuda.synchronize()
@@ -473,11 +492,13 @@ def main():
         "metric": "BSA fwd(+bwd) effective TFLOP/s at 720p tokens",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic, q/k with a shared smooth field" if args.structured else "synthetic",
         "config": {"workload": args.workload, "tokens": w.n_tokens, "padded_tokens": g.nbq * g.bs,
                    "heads": w.heads, "head_dim": w.head_dim, "block": list(w.blk),
                    "top_r": w.top_r, "selected_pairs": n_pairs, "with_bwd": with_bwd,
                    "fwd_tflop_tiles": fl_fwd / 1e12, "fwd_tflop_valid_tokens": fl_fwd_valid / 1e12,
+                   "selections_within_one_block": locality,
                    "parallelism": f"replicas{world}", "l2": "inputs larger than L2 (126 MB)"},
         "ms_per_call": parts,
         "kernels": kernels,

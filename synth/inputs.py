@@ -144,3 +144,46 @@ def make_raster_inputs(w: Workload, with_grad: bool = False,
             out["gamma_q"] = (1.0 + 0.25 * rng.standard_normal(w.head_dim)).astype(np.float32)
             out["gamma_k"] = (1.0 + 0.25 * rng.standard_normal(w.head_dim)).astype(np.float32)
     return out
+
+
+SEED_FIELD = 9
+
+
+def add_smooth_field(w: Workload, x: Dict[str, Optional[np.ndarray]], alpha: float = 1.0,
+                     n_modes: int = 8, frames: Optional[int] = None,
+                     t_offset: int = 0) -> Dict[str, Optional[np.ndarray]]:
+    """Structured variant of the i.i.d. inputs: q and k get the same smooth low-frequency
+    field over (t, h, w), so neighbouring tokens have similar q and k, as in real video
+    latents (i.i.d. N(0,1) tokens have no locality at all).
+
+    Field per head: F(t, y, x) = sum_c cos(2 pi (a_c t/T + b_c y/Hg + c_c x/Wg) + phi_c) W[c, :]
+    with integer wave numbers a, b, c in {0, 1, 2}, random phases and W ~ N(0, 1/n_modes) per
+    head, so each channel of the field has unit variance; q = q_iid + alpha F, k = k_iid +
+    alpha F (bf16 RNE).  Cached frames get the field of their own absolute frames.  Returns a
+    new dict; v, dO and the cache values are unchanged.
+    """
+    rng = np.random.Generator(np.random.PCG64(SEED_FIELD))
+    T = w.cached_t + w.t_frames
+    waves = rng.integers(0, 3, size=(n_modes, 3)).astype(np.float32)
+    waves[0] = (0.0, 1.0, 1.0)  # at least one mode varies in space
+    phase = rng.uniform(0.0, 2.0 * np.pi, size=n_modes).astype(np.float32)
+    W = (rng.standard_normal((w.heads, n_modes, w.head_dim), dtype=np.float32)
+         / np.float32(np.sqrt(n_modes)))
+
+    def field(f0: int, nf: int) -> np.ndarray:
+        t = np.arange(f0, f0 + nf, dtype=np.float32)[:, None, None]
+        yy = np.arange(w.grid_h, dtype=np.float32)[None, :, None]
+        xx = np.arange(w.grid_w, dtype=np.float32)[None, None, :]
+        feats = np.stack([np.cos(2 * np.pi * (a * t / T + b * yy / w.grid_h + c * xx / w.grid_w) + p)
+                          for (a, b, c), p in zip(waves, phase)], axis=-1)  # [nf, Hg, Wg, C]
+        feats = feats.reshape(-1, n_modes)
+        wm = np.ascontiguousarray(W.transpose(1, 0, 2).reshape(n_modes, -1))  # [C, H*D]
+        return (feats @ wm).reshape(-1, w.heads, w.head_dim)  # [N, H, D]
+
+    out = dict(x)
+    cur = field(w.cached_t, w.t_frames)[None] * np.float32(alpha)
+    for name in ("q", "k"):
+        out[name] = bf16_bits_from_f32(bf16_bits_to_f32(x[name]) + cur)
+    if w.cached_t and x.get("kc") is not None:
+        out["kc"] = bf16_bits_from_f32(bf16_bits_to_f32(x["kc"]) + field(0, w.cached_t)[None] * np.float32(alpha))
+    return out

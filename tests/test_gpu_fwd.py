@@ -296,3 +296,17 @@ def test_two_segment_mask(torch_cuda, cond_t, chunk_t):
     assert np.any(idx[:, :, n_cond:] >= n_cond)
     assert check_route(w, pipe, [0, 1]) == 0
     check_attention(w, pipe, [0, 1])
+
+
+@pytest.mark.parametrize("name", ["small", "small_b2", "small_cont_rope"])
+def test_structured_inputs_parity(torch_cuda, name):
+    """Inputs with a smooth field shared by q and k (video-like locality): the routing picks
+    mostly neighbouring blocks; prologue, selections and attention still match the oracle."""
+    from synth import add_smooth_field
+    w = WORKLOADS[name]
+    x = add_smooth_field(w, make_raster_inputs(w))
+    pipe, _ = run_forward(w, x=x)
+    heads = list(range(w.heads))
+    check_prologue(w, pipe, x, heads)
+    assert check_route(w, pipe, heads) == 0
+    check_attention(w, pipe, heads)
