@@ -21,6 +21,9 @@ __all__ = [
     "bsa_selftest_bounded_wait", "bsa_route_noalloc", "rope3d_qknorm_prologue_bwd",
     "bsa_cache_append", "bsa_route_ex", "bsa_block_pool", "ROUTE_FORCE_SELF",
     "ROUTE_SHARED_HEADS", "ROUTE_POOL_SUM", "ROUTE_POOL_MAX", "POOL_MEAN", "POOL_SUM", "POOL_MAX",
+    "Shards", "MAX_SHARDS", "IPC_HANDLE_BYTES", "rope3d_qknorm_prologue_sharded",
+    "rope3d_qknorm_prologue_bwd_sharded", "bsa_blocked_to_raster_sharded", "bsa_ipc_export",
+    "bsa_ipc_import", "bsa_ipc_close",
     "bsa_kernel_timing", "bsa_kernel_times",
     "WS_ROUTE", "WS_FWD", "WS_BWD", "WS_PROLOGUE_BWD",
 ]
@@ -46,6 +49,28 @@ class _Geom(ctypes.Structure):
                 ("cached_t", ctypes.c_int32), ("blk_t", ctypes.c_int32), ("blk_h", ctypes.c_int32),
                 ("blk_w", ctypes.c_int32), ("causal_chunk_t", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("cond_t", ctypes.c_int32)]
+
+
+MAX_SHARDS, IPC_HANDLE_BYTES = 8, 128
+
+
+class _Shards(ctypes.Structure):
+    _fields_ = [("n_shards", ctypes.c_int32), ("shard_frames", ctypes.c_int32),
+                ("heads_total", ctypes.c_int32), ("head0", ctypes.c_int32)]
+
+
+@dataclasses.dataclass(frozen=True)
+class Shards:
+    """Mirror of ``bsa_shards_t``: raster tensors split by frames into ``n_shards`` pieces of
+    ``shard_frames`` frames with ``heads_total`` heads per row; a call processes heads
+    ``head0`` .. ``head0 + g.heads - 1``."""
+    n_shards: int
+    shard_frames: int
+    heads_total: int
+    head0: int = 0
+
+    def c(self) -> _Shards:
+        return _Shards(self.n_shards, self.shard_frames, self.heads_total, self.head0)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -112,6 +137,7 @@ def lib() -> ctypes.CDLL:
         L = ctypes.CDLL(LIB_PATH)
         P, I32, F, S = ctypes.c_void_p, ctypes.c_int32, ctypes.c_float, ctypes.c_size_t
         G = ctypes.POINTER(_Geom)
+        SH = ctypes.POINTER(_Shards)
         sig = {
             "bsa_abi_version": (I32, []),
             "bsa_workspace_size": (S, [G, I32, I32]),
@@ -128,6 +154,14 @@ def lib() -> ctypes.CDLL:
             "bsa_route_noalloc": (I32, [G, I32, P, P, P, P, P, P]),
             "bsa_kernel_timing": (I32, [I32]),
             "bsa_cache_append": (I32, [G, P, P, P, P, P, P, P, P, P, P]),
+            "rope3d_qknorm_prologue_sharded": (I32, [G, I32, I32, SH, P, P, P, P, P, F, F, P, P,
+                                                     P, P, P, P]),
+            "rope3d_qknorm_prologue_bwd_sharded": (I32, [G, I32, I32, SH, P, P, P, P, F, F, P, P,
+                                                         P, P, P, P, P, P, P, S, P]),
+            "bsa_blocked_to_raster_sharded": (I32, [G, I32, SH, P, P, P]),
+            "bsa_ipc_export": (I32, [P, P]),
+            "bsa_ipc_import": (I32, [P, ctypes.POINTER(ctypes.c_void_p)]),
+            "bsa_ipc_close": (I32, [P]),
             "bsa_kernel_times": (I32, [P, P]),
             "bsa_error_string": (ctypes.c_char_p, [I32]),
             "bsa_last_error_detail": (ctypes.c_char_p, []),
@@ -194,6 +228,73 @@ def rope3d_qknorm_prologue_bwd(g: Geometry, frames: int, t_offset: int, q, k, ga
         eps, rope_theta, _ptr(dq_blk), _ptr(dk_blk), _ptr(dv_blk), _ptr(dq), _ptr(dk), _ptr(dv),
         _ptr(dgamma_q), _ptr(dgamma_k), _ptr(ws), _nbytes(ws) if ws is not None else 0,
         _stream(stream)), "rope3d_qknorm_prologue_bwd")
+
+
+def _ptr_array(ts):
+    """Host array of device pointers (one per shard), or None."""
+    if ts is None:
+        return None
+    arr = (ctypes.c_void_p * len(ts))(*[_ptr(t) for t in ts])
+    return ctypes.cast(arr, ctypes.c_void_p), arr  # keep `arr` alive for the call
+
+
+def _arr(x):
+    return None if x is None else x[0]
+
+
+def rope3d_qknorm_prologue_sharded(g: Geometry, frames: int, t_offset: int, sh: Shards,
+                                   q_shards, k_shards, v_shards, gamma_q, gamma_k, eps: float,
+                                   rope_theta: float, q_blk, k_blk, v_blk, q_pool=None,
+                                   k_pool=None, stream=None):
+    """The prologue reading raster inputs from frame shards (lists of tensors or pointers)."""
+    qa, ka, va = _ptr_array(q_shards), _ptr_array(k_shards), _ptr_array(v_shards)
+    _check(lib().rope3d_qknorm_prologue_sharded(
+        ctypes.byref(g.c()), frames, t_offset, ctypes.byref(sh.c()), _arr(qa), _arr(ka), _arr(va),
+        _ptr(gamma_q), _ptr(gamma_k), eps, rope_theta, _ptr(q_blk), _ptr(k_blk), _ptr(v_blk),
+        _ptr(q_pool), _ptr(k_pool), _stream(stream)), "rope3d_qknorm_prologue_sharded")
+
+
+def rope3d_qknorm_prologue_bwd_sharded(g: Geometry, frames: int, t_offset: int, sh: Shards,
+                                       q_shards, k_shards, gamma_q, gamma_k, eps: float,
+                                       rope_theta: float, dq_blk, dk_blk, dv_blk, dq_shards,
+                                       dk_shards, dv_shards, dgamma_q=None, dgamma_k=None,
+                                       ws=None, stream=None):
+    qa, ka = _ptr_array(q_shards), _ptr_array(k_shards)
+    dqa, dka, dva = _ptr_array(dq_shards), _ptr_array(dk_shards), _ptr_array(dv_shards)
+    _check(lib().rope3d_qknorm_prologue_bwd_sharded(
+        ctypes.byref(g.c()), frames, t_offset, ctypes.byref(sh.c()), _arr(qa), _arr(ka),
+        _ptr(gamma_q), _ptr(gamma_k), eps, rope_theta, _ptr(dq_blk), _ptr(dk_blk), _ptr(dv_blk),
+        _arr(dqa), _arr(dka), _arr(dva), _ptr(dgamma_q), _ptr(dgamma_k), _ptr(ws),
+        _nbytes(ws) if ws is not None else 0, _stream(stream)), "rope3d_qknorm_prologue_bwd_sharded")
+
+
+def bsa_blocked_to_raster_sharded(g: Geometry, frames: int, sh: Shards, x_blk, x_shards,
+                                  stream=None):
+    xa = _ptr_array(x_shards)
+    _check(lib().bsa_blocked_to_raster_sharded(
+        ctypes.byref(g.c()), frames, ctypes.byref(sh.c()), _ptr(x_blk), _arr(xa), _stream(stream)),
+        "bsa_blocked_to_raster_sharded")
+
+
+def bsa_ipc_export(t) -> bytes:
+    """IPC handle (IPC_HANDLE_BYTES bytes) of the device buffer holding tensor / pointer t."""
+    buf = ctypes.create_string_buffer(IPC_HANDLE_BYTES)
+    _check(lib().bsa_ipc_export(_ptr(t), buf), "bsa_ipc_export")
+    return buf.raw
+
+
+def bsa_ipc_import(handle: bytes) -> int:
+    """Device pointer (int) mapping another process's buffer; release with bsa_ipc_close."""
+    if len(handle) != IPC_HANDLE_BYTES:
+        raise ValueError("bad IPC handle length")
+    out = ctypes.c_void_p()
+    _check(lib().bsa_ipc_import(ctypes.create_string_buffer(handle, IPC_HANDLE_BYTES),
+                                ctypes.byref(out)), "bsa_ipc_import")
+    return int(out.value)
+
+
+def bsa_ipc_close(ptr: int):
+    _check(lib().bsa_ipc_close(ptr), "bsa_ipc_close")
 
 
 def bsa_cache_append(g: Geometry, kc_blk, vc_blk, kc_pool, k_blk, v_blk, k_pool, kc_new, vc_new,

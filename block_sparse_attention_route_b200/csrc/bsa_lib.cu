@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "timing.cuh"
@@ -223,12 +224,37 @@ size_t bsa_workspace_size(const bsa_geom_t* gi, int32_t top_r, int32_t which) {
   return 0;
 }
 
-bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
-                                    const void* q_raster, const void* k_raster,
-                                    const void* v_raster, const float* gamma_q,
-                                    const float* gamma_k, float eps, float rope_theta,
-                                    void* q_blk, void* k_blk, void* v_blk, float* q_pool,
-                                    float* k_pool, bsa_stream_t stream) {
+// Shards of the raster tensors: NULL = one shard holding every frame and head of the call.
+static bsa_status_t make_shards(const Geo& g, int32_t frames, const bsa_shards_t* sd,
+                                RasterShards* out) {
+  RasterShards r{1, frames, g.H, 0};
+  if (sd) {
+    if (sd->n_shards < 1 || sd->n_shards > kMaxShards)
+      return fail(BSA_ERR_INVALID_ARG, "n_shards %d (supported: 1..%d)", sd->n_shards, kMaxShards);
+    if (sd->shard_frames < 1 || (long)sd->n_shards * sd->shard_frames != frames)
+      return fail(BSA_ERR_INVALID_ARG, "n_shards * shard_frames must equal frames (%d)", frames);
+    if (sd->head0 < 0 || sd->heads_total < 1 || (long)sd->head0 + g.H > sd->heads_total)
+      return fail(BSA_ERR_INVALID_ARG, "heads head0 .. head0 + heads - 1 must lie in 0 .. heads_total - 1");
+    r = RasterShards{sd->n_shards, sd->shard_frames, sd->heads_total, sd->head0};
+  }
+  if (((long)r.frames * g.GH * g.GW) * (long)g.B * r.h_stride * g.D >= (1L << 40))
+    return fail(BSA_ERR_UNSUPPORTED, "tensor too large");
+  *out = r;
+  return BSA_OK;
+}
+
+// Every shard pointer of a given tensor present and 16-byte aligned.
+static bool shard_ptrs_ok(const void* const* p, int n) {
+  for (int s = 0; s < n; ++s)
+    if (p[s] == nullptr || !aligned(p[s], 16)) return false;
+  return true;
+}
+
+static bsa_status_t prologue_impl(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
+                                  const bsa_shards_t* sd, const void* const* const xsh[3],
+                                  const float* gamma_q, const float* gamma_k, float eps,
+                                  float rope_theta, void* q_blk, void* k_blk, void* v_blk,
+                                  float* q_pool, float* k_pool, bsa_stream_t stream) {
   t_detail.clear();
   Geo g;
   bsa_status_t st = make_geo(gi, &g);
@@ -237,23 +263,22 @@ bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* gi, int32_t frames, int32_
   if (t_offset < 0) return fail(BSA_ERR_INVALID_ARG, "t_offset must be >= 0");
   if (!(eps >= 0.f) || !(rope_theta >= 0.f) || std::isinf(rope_theta))
     return fail(BSA_ERR_INVALID_ARG, "eps and rope_theta must be finite and >= 0");
-  const void* xs[3] = {q_raster, k_raster, v_raster};
+  RasterShards sh;
+  if ((st = make_shards(g, frames, sd, &sh)) != BSA_OK) return st;
   void* ys[3] = {q_blk, k_blk, v_blk};
   bool any = false;
   for (int i = 0; i < 3; ++i) {
-    if ((xs[i] == nullptr) != (ys[i] == nullptr))
+    if ((xsh[i] == nullptr) != (ys[i] == nullptr))
       return fail(BSA_ERR_INVALID_ARG, "input %d and its output must both be given or both NULL", i);
-    if (xs[i] && (!aligned(xs[i], 16) || !aligned(ys[i], 16)))
-      return fail(BSA_ERR_INVALID_ARG, "tensor %d not 16-byte aligned", i);
-    any |= xs[i] != nullptr;
+    if (xsh[i] && (!shard_ptrs_ok(xsh[i], sh.n) || !aligned(ys[i], 16)))
+      return fail(BSA_ERR_INVALID_ARG, "tensor %d: a shard is NULL or a tensor is not 16-byte aligned", i);
+    any |= xsh[i] != nullptr;
   }
   if (!any) return fail(BSA_ERR_INVALID_ARG, "no tensor to process");
-  if ((q_pool && !q_raster) || (k_pool && !k_raster))
+  if ((q_pool && !xsh[0]) || (k_pool && !xsh[1]))
     return fail(BSA_ERR_INVALID_ARG, "a pool output needs its tensor");
   if ((q_pool && !aligned(q_pool, 16)) || (k_pool && !aligned(k_pool, 16)))
     return fail(BSA_ERR_INVALID_ARG, "pool outputs must be 16-byte aligned");
-  if (((long)frames * g.GH * g.GW) * (long)g.B * g.H * g.D >= (1L << 40))
-    return fail(BSA_ERR_UNSUPPORTED, "tensor too large");
   st = check_device(nullptr);
   if (st != BSA_OK) return st;
   PrologueArgs a;
@@ -261,8 +286,10 @@ bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* gi, int32_t frames, int32_
   a.frames = frames;
   a.t_offset = t_offset;
   a.nbt = (frames + g.bt - 1) / g.bt;
+  a.sh = sh;
   for (int i = 0; i < 3; ++i) {
-    a.x[i] = static_cast<const __nv_bfloat16*>(xs[i]);
+    for (int s2 = 0; s2 < kMaxShards; ++s2)
+      a.x[i][s2] = (xsh[i] && s2 < sh.n) ? static_cast<const __nv_bfloat16*>(xsh[i][s2]) : nullptr;
     a.y[i] = static_cast<__nv_bfloat16*>(ys[i]);
   }
   a.gamma[0] = gamma_q;
@@ -279,13 +306,42 @@ bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* gi, int32_t frames, int32_
   return BSA_OK;
 }
 
-bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
-                                        const void* q_raster, const void* k_raster,
-                                        const float* gamma_q, const float* gamma_k, float eps,
-                                        float rope_theta, const void* dq_blk, const void* dk_blk,
-                                        const void* dv_blk, void* dq, void* dk, void* dv,
-                                        float* dgamma_q, float* dgamma_k, void* ws, size_t ws_bytes,
-                                        bsa_stream_t stream) {
+bsa_status_t rope3d_qknorm_prologue(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
+                                    const void* q_raster, const void* k_raster,
+                                    const void* v_raster, const float* gamma_q,
+                                    const float* gamma_k, float eps, float rope_theta,
+                                    void* q_blk, void* k_blk, void* v_blk, float* q_pool,
+                                    float* k_pool, bsa_stream_t stream) {
+  const void* one[3][1] = {{q_raster}, {k_raster}, {v_raster}};
+  const void* const* xsh[3] = {q_raster ? one[0] : nullptr, k_raster ? one[1] : nullptr,
+                               v_raster ? one[2] : nullptr};
+  return prologue_impl(gi, frames, t_offset, nullptr, xsh, gamma_q, gamma_k, eps, rope_theta,
+                       q_blk, k_blk, v_blk, q_pool, k_pool, stream);
+}
+
+bsa_status_t rope3d_qknorm_prologue_sharded(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
+                                            const bsa_shards_t* sh, const void* const* q_shards,
+                                            const void* const* k_shards,
+                                            const void* const* v_shards, const float* gamma_q,
+                                            const float* gamma_k, float eps, float rope_theta,
+                                            void* q_blk, void* k_blk, void* v_blk, float* q_pool,
+                                            float* k_pool, bsa_stream_t stream) {
+  if (sh == nullptr) {
+    t_detail.clear();
+    return fail(BSA_ERR_INVALID_ARG, "shard description is required");
+  }
+  const void* const* xsh[3] = {q_shards, k_shards, v_shards};
+  return prologue_impl(gi, frames, t_offset, sh, xsh, gamma_q, gamma_k, eps, rope_theta, q_blk,
+                       k_blk, v_blk, q_pool, k_pool, stream);
+}
+
+static bsa_status_t prologue_bwd_impl(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
+                                      const bsa_shards_t* sd, const void* const* const xsh[2],
+                                      const float* gamma_q, const float* gamma_k, float eps,
+                                      float rope_theta, const void* dq_blk, const void* dk_blk,
+                                      const void* dv_blk, void* const* const dxsh[3],
+                                      float* dgamma_q, float* dgamma_k, void* ws, size_t ws_bytes,
+                                      bsa_stream_t stream) {
   t_detail.clear();
   Geo g;
   bsa_status_t st = make_geo(gi, &g);
@@ -294,30 +350,30 @@ bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* gi, int32_t frames, in
   if (t_offset < 0) return fail(BSA_ERR_INVALID_ARG, "t_offset must be >= 0");
   if (!(eps >= 0.f) || !(rope_theta >= 0.f) || std::isinf(rope_theta))
     return fail(BSA_ERR_INVALID_ARG, "eps and rope_theta must be finite and >= 0");
+  RasterShards sh;
+  if ((st = make_shards(g, frames, sd, &sh)) != BSA_OK) return st;
   const void* dz[3] = {dq_blk, dk_blk, dv_blk};
-  void* dxs[3] = {dq, dk, dv};
-  const void* xs[2] = {q_raster, k_raster};
   const float* gams[2] = {gamma_q, gamma_k};
   float* dgs[2] = {dgamma_q, dgamma_k};
   bool any = false, any_gain = false;
   for (int i = 0; i < 3; ++i) {
-    if ((dz[i] == nullptr) != (dxs[i] == nullptr))
+    if ((dz[i] == nullptr) != (dxsh[i] == nullptr))
       return fail(BSA_ERR_INVALID_ARG, "gradient %d and its output must both be given or both NULL", i);
-    if (dz[i] && (!aligned(dz[i], 16) || !aligned(dxs[i], 16)))
-      return fail(BSA_ERR_INVALID_ARG, "tensor %d not 16-byte aligned", i);
+    if (dz[i] && (!aligned(dz[i], 16) ||
+                  !shard_ptrs_ok(reinterpret_cast<const void* const*>(dxsh[i]), sh.n)))
+      return fail(BSA_ERR_INVALID_ARG, "tensor %d: a shard is NULL or a tensor is not 16-byte aligned", i);
     any |= dz[i] != nullptr;
   }
   if (!any) return fail(BSA_ERR_INVALID_ARG, "no tensor to process");
   for (int i = 0; i < 2; ++i) {
     if (dz[i] && gams[i]) {
-      if (!xs[i] || !dgs[i])
+      if (!xsh[i] || !dgs[i])
         return fail(BSA_ERR_INVALID_ARG, "with a gain, tensor %d needs its raster input and a dgamma output", i);
-      if (!aligned(xs[i], 16)) return fail(BSA_ERR_INVALID_ARG, "raster input %d not 16-byte aligned", i);
+      if (!shard_ptrs_ok(xsh[i], sh.n))
+        return fail(BSA_ERR_INVALID_ARG, "raster input %d: a shard is NULL or not 16-byte aligned", i);
       any_gain = true;
     }
   }
-  if (((long)frames * g.GH * g.GW) * (long)g.B * g.H * g.D >= (1L << 40))
-    return fail(BSA_ERR_UNSUPPORTED, "tensor too large");
   const int nbt = (frames + g.bt - 1) / g.bt;
   const size_t part_bytes = align256((size_t)prologue_bwd_ctas(g, nbt) * g.D * sizeof(float));
   if (any_gain && (ws == nullptr || ws_bytes < 2 * part_bytes || !aligned(ws, 256)))
@@ -331,7 +387,11 @@ bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* gi, int32_t frames, in
   f.frames = frames;
   f.t_offset = t_offset;
   f.nbt = nbt;
-  for (int i = 0; i < 3; ++i) { f.x[i] = nullptr; f.y[i] = nullptr; }
+  f.sh = sh;
+  for (int i = 0; i < 3; ++i) {
+    for (int s2 = 0; s2 < kMaxShards; ++s2) f.x[i][s2] = nullptr;
+    f.y[i] = nullptr;
+  }
   f.gamma[0] = dq_blk ? gamma_q : nullptr;
   f.gamma[1] = dk_blk ? gamma_k : nullptr;
   f.pool[0] = f.pool[1] = nullptr;
@@ -342,17 +402,63 @@ bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* gi, int32_t frames, in
   f.dt = g.D - 2 * f.dh;
   for (int i = 0; i < 3; ++i) {
     a.dz[i] = static_cast<const __nv_bfloat16*>(dz[i]);
-    a.dx[i] = static_cast<__nv_bfloat16*>(dxs[i]);
+    for (int s2 = 0; s2 < kMaxShards; ++s2)
+      a.dx[i][s2] = (dxsh[i] && s2 < sh.n) ? static_cast<__nv_bfloat16*>(dxsh[i][s2]) : nullptr;
   }
   for (int i = 0; i < 2; ++i) {
-    a.x[i] = static_cast<const __nv_bfloat16*>(xs[i]);
-    a.part[i] = (dz[i] && gams[i]) ? reinterpret_cast<float*>(static_cast<char*>(ws) + i * part_bytes)
-                                   : nullptr;
-    if (!(dz[i] && gams[i])) dgs[i] = nullptr;
+    const bool gain = dz[i] && gams[i];
+    for (int s2 = 0; s2 < kMaxShards; ++s2)
+      a.x[i][s2] = (gain && s2 < sh.n) ? static_cast<const __nv_bfloat16*>(xsh[i][s2]) : nullptr;
+    a.part[i] = gain ? reinterpret_cast<float*>(static_cast<char*>(ws) + i * part_bytes) : nullptr;
+    if (!gain) dgs[i] = nullptr;
   }
   cudaError_t e = launch_prologue_bwd(a, dgs, reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "prologue backward launch");
   return BSA_OK;
+}
+
+bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* gi, int32_t frames, int32_t t_offset,
+                                        const void* q_raster, const void* k_raster,
+                                        const float* gamma_q, const float* gamma_k, float eps,
+                                        float rope_theta, const void* dq_blk, const void* dk_blk,
+                                        const void* dv_blk, void* dq, void* dk, void* dv,
+                                        float* dgamma_q, float* dgamma_k, void* ws, size_t ws_bytes,
+                                        bsa_stream_t stream) {
+  const void* xone[2][1] = {{q_raster}, {k_raster}};
+  const void* const* xsh[2] = {q_raster ? xone[0] : nullptr, k_raster ? xone[1] : nullptr};
+  void* done[3][1] = {{dq}, {dk}, {dv}};
+  void* const* dxsh[3] = {dq ? done[0] : nullptr, dk ? done[1] : nullptr, dv ? done[2] : nullptr};
+  return prologue_bwd_impl(gi, frames, t_offset, nullptr, xsh, gamma_q, gamma_k, eps, rope_theta,
+                           dq_blk, dk_blk, dv_blk, dxsh, dgamma_q, dgamma_k, ws, ws_bytes, stream);
+}
+
+bsa_status_t rope3d_qknorm_prologue_bwd_sharded(
+    const bsa_geom_t* gi, int32_t frames, int32_t t_offset, const bsa_shards_t* sh,
+    const void* const* q_shards, const void* const* k_shards, const float* gamma_q,
+    const float* gamma_k, float eps, float rope_theta, const void* dq_blk, const void* dk_blk,
+    const void* dv_blk, void* const* dq_shards, void* const* dk_shards, void* const* dv_shards,
+    float* dgamma_q, float* dgamma_k, void* ws, size_t ws_bytes, bsa_stream_t stream) {
+  if (sh == nullptr) {
+    t_detail.clear();
+    return fail(BSA_ERR_INVALID_ARG, "shard description is required");
+  }
+  const void* const* xsh[2] = {q_shards, k_shards};
+  void* const* dxsh[3] = {dq_shards, dk_shards, dv_shards};
+  return prologue_bwd_impl(gi, frames, t_offset, sh, xsh, gamma_q, gamma_k, eps, rope_theta,
+                           dq_blk, dk_blk, dv_blk, dxsh, dgamma_q, dgamma_k, ws, ws_bytes, stream);
+}
+
+bsa_status_t bsa_blocked_to_raster_sharded(const bsa_geom_t* gi, int32_t frames,
+                                           const bsa_shards_t* sh, const void* x_blk,
+                                           void* const* x_shards, bsa_stream_t stream) {
+  if (sh == nullptr || x_blk == nullptr || x_shards == nullptr) {
+    t_detail.clear();
+    return fail(BSA_ERR_INVALID_ARG, "shard description, x_blk and x_shards are required");
+  }
+  const void* const* xsh[2] = {nullptr, nullptr};
+  void* const* dxsh[3] = {nullptr, nullptr, x_shards};
+  return prologue_bwd_impl(gi, frames, 0, sh, xsh, nullptr, nullptr, 0.f, 0.f, nullptr, nullptr,
+                           x_blk, dxsh, nullptr, nullptr, nullptr, 0, stream);
 }
 
 bsa_status_t bsa_cache_append(const bsa_geom_t* gi, const void* kc_blk, const void* vc_blk,
@@ -651,5 +757,104 @@ bsa_status_t bsa_device_status(bsa_stream_t stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- CUDA IPC of shard buffers
+// A handle is the cudaIpcMemHandle of the allocation holding the pointer followed by the
+// pointer's byte offset in it (the caching allocators above the library hand out pieces of
+// larger allocations).  Imported mappings are remembered so that bsa_ipc_close can unmap the
+// allocation base.
+namespace {
+typedef CUresult (*AddressRangeFn)(CUdeviceptr*, size_t*, CUdeviceptr);
+struct IpcHandle {
+  cudaIpcMemHandle_t mem;
+  uint64_t offset;
+};
+static_assert(sizeof(IpcHandle) <= BSA_IPC_HANDLE_BYTES, "IPC handle size");
+struct IpcMapping {
+  cudaIpcMemHandle_t mem;
+  void* base;
+  int refs;
+};
+std::mutex g_ipc_mu;
+std::vector<IpcMapping> g_ipc_bases;              // one mapping per peer allocation
+std::vector<std::pair<void*, void*>> g_ipc_maps;  // (imported pointer, mapped base), per import
+
+AddressRangeFn address_range_fn() {
+  static AddressRangeFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuMemGetAddressRange", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<AddressRangeFn>(f);
+  });
+  return fn;
+}
+}  // namespace
+
+bsa_status_t bsa_ipc_export(const void* dev_ptr, void* handle) {
+  t_detail.clear();
+  if (!dev_ptr || !handle) return fail(BSA_ERR_INVALID_ARG, "dev_ptr and handle are required");
+  AddressRangeFn range = address_range_fn();
+  if (!range) return fail(BSA_ERR_CUDA, "cuMemGetAddressRange is not available");
+  CUdeviceptr base = 0;
+  size_t bytes = 0;
+  if (range(&base, &bytes, reinterpret_cast<CUdeviceptr>(dev_ptr)) != CUDA_SUCCESS)
+    return fail(BSA_ERR_INVALID_ARG, "dev_ptr is not device memory of this process");
+  IpcHandle h;
+  std::memset(&h, 0, sizeof(h));
+  cudaError_t e = cudaIpcGetMemHandle(&h.mem, reinterpret_cast<void*>(base));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaIpcGetMemHandle");
+  h.offset = reinterpret_cast<uintptr_t>(dev_ptr) - static_cast<uintptr_t>(base);
+  std::memset(handle, 0, BSA_IPC_HANDLE_BYTES);
+  std::memcpy(handle, &h, sizeof(h));
+  return BSA_OK;
+}
+
+bsa_status_t bsa_ipc_import(const void* handle, void** dev_ptr) {
+  t_detail.clear();
+  if (!handle || !dev_ptr) return fail(BSA_ERR_INVALID_ARG, "handle and dev_ptr are required");
+  IpcHandle h;
+  std::memcpy(&h, handle, sizeof(h));
+  std::lock_guard<std::mutex> lk(g_ipc_mu);
+  void* base = nullptr;
+  for (IpcMapping& m : g_ipc_bases)  // an allocation is mapped once per process
+    if (std::memcmp(&m.mem, &h.mem, sizeof(h.mem)) == 0) {
+      base = m.base;
+      ++m.refs;
+      break;
+    }
+  if (!base) {
+    cudaError_t e = cudaIpcOpenMemHandle(&base, h.mem, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+    g_ipc_bases.push_back(IpcMapping{h.mem, base, 1});
+  }
+  void* p = static_cast<char*>(base) + h.offset;
+  g_ipc_maps.emplace_back(p, base);
+  *dev_ptr = p;
+  return BSA_OK;
+}
+
+bsa_status_t bsa_ipc_close(void* dev_ptr) {
+  t_detail.clear();
+  std::lock_guard<std::mutex> lk(g_ipc_mu);
+  void* base = nullptr;
+  for (size_t k = 0; k < g_ipc_maps.size(); ++k)
+    if (g_ipc_maps[k].first == dev_ptr) {
+      base = g_ipc_maps[k].second;
+      g_ipc_maps.erase(g_ipc_maps.begin() + (long)k);
+      break;
+    }
+  if (!base) return fail(BSA_ERR_INVALID_ARG, "pointer was not imported by bsa_ipc_import");
+  for (size_t k = 0; k < g_ipc_bases.size(); ++k)
+    if (g_ipc_bases[k].base == base && --g_ipc_bases[k].refs == 0) {
+      g_ipc_bases.erase(g_ipc_bases.begin() + (long)k);
+      cudaError_t e = cudaIpcCloseMemHandle(base);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaIpcCloseMemHandle");
+      break;
+    }
+  return BSA_OK;
+}
 
 #include "route_noalloc.cu"

@@ -15,10 +15,32 @@
 
 namespace bsa {
 
+// Raster tensors may be split along frames into shards (one per rank of a sequence-parallel
+// group, each possibly on another GPU): shard s holds frames [s * frames, (s + 1) * frames)
+// of the grid as [B, frames * GH * GW, h_stride, D], and this call processes raster heads
+// h0 .. h0 + g.H - 1 of it.  One shard with h_stride = g.H and h0 = 0 is the plain layout.
+// Reading or writing the shards of other ranks through their pointers is the sequence <->
+// head exchange of Ulysses parallelism, fused into the relayout.
+constexpr int kMaxShards = 8;
+struct RasterShards {
+  int n, frames;     // shards, frames per shard
+  int h_stride, h0;  // heads of every raster row, first head processed
+};
+
+// Shard and element offset of (b, frame t of the grid, row hh, column ww, head h, channel c0).
+__device__ __forceinline__ size_t shard_elem(const RasterShards& sh, const Geo& g, int b, int t,
+                                             int hh, int ww, int h, int c0, int& s) {
+  s = t / sh.frames;
+  const size_t n = ((size_t)(t - s * sh.frames) * g.GH + hh) * g.GW + ww;
+  const size_t per_shard = (size_t)sh.frames * g.GH * g.GW;
+  return (((size_t)b * per_shard + n) * sh.h_stride + sh.h0 + h) * (size_t)g.D + c0;
+}
+
 struct PrologueArgs {
   Geo g;
   int frames, t_offset, nbt;  // grid being processed: frames, RoPE frame offset, t-blocks
-  const __nv_bfloat16* x[3];
+  RasterShards sh;
+  const __nv_bfloat16* x[3][kMaxShards];  // raster inputs per shard (x[w][0] == NULL: skip)
   __nv_bfloat16* y[3];
   const float* gamma[2];
   float* pool[2];
@@ -81,7 +103,6 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
   const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
   const int rows = kHeadsPerCta * g.BS;  // (slot, head) pairs; heads >= heads_here are skipped
-  const size_t n_raster = (size_t)a.frames * g.GH * g.GW;
 
   // RoPE coordinates of this lane's 4 channel pairs: axis (0 t, 1 h, 2 w) and pair index.
   int ax[4], pi[4];
@@ -94,9 +115,8 @@ __global__ void __launch_bounds__(kPrologueThreads)
   }
 
   for (int which = 0; which < 3; ++which) {
-    const __nv_bfloat16* __restrict__ x = a.x[which];
     __nv_bfloat16* __restrict__ y = a.y[which];
-    if (x == nullptr) continue;
+    if (a.x[which][0] == nullptr) continue;
     const bool qk = which < 2;
     const float* gam = qk ? a.gamma[which] : nullptr;
     const bool do_rope = qk && rope;
@@ -118,9 +138,9 @@ __global__ void __launch_bounds__(kPrologueThreads)
       float v[8];
       if (valid) {
         const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
-        const size_t n = ((size_t)t * g.GH + hh) * g.GW + ww;
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(
-            x + (((size_t)b * n_raster + n) * g.H + h) * D + c0));
+        int sidx;
+        const size_t off = shard_elem(a.sh, g, b, t, hh, ww, h, c0, sidx);
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(a.x[which][sidx] + off));
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -190,7 +210,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
   __syncthreads();
   for (int which = 0; which < 2; ++which) {
     float* out = a.pool[which];
-    if (out == nullptr || a.x[which] == nullptr) continue;
+    if (out == nullptr || a.x[which][0] == nullptr) continue;
     const float inv = nvalid > 0 ? 1.0f / (float)nvalid : 0.f;
     for (int e = tid; e < heads_here * D; e += kPrologueThreads) {
       const int hl = e / D, d = e % D, h = hg * kHeadsPerCta + hl;
@@ -235,8 +255,8 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s) {
 struct PrologueBwdArgs {
   PrologueArgs f;                 // geometry, RoPE widths, frames, t_offset, gamma, eps, theta
   const __nv_bfloat16* dz[3];     // blocked gradients of the outputs (NULL = skip)
-  const __nv_bfloat16* x[2];      // raster forward inputs q, k (needed with a gain)
-  __nv_bfloat16* dx[3];           // raster gradients of the inputs
+  const __nv_bfloat16* x[2][kMaxShards];  // raster forward inputs q, k per shard (with a gain)
+  __nv_bfloat16* dx[3][kMaxShards];       // raster gradients of the inputs per shard (f.sh)
   float* part[2];                 // [n_cta][D] dgamma partials of q, k
 };
 
@@ -267,7 +287,6 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
   const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
   const int rows = kHeadsPerCta * g.BS;
-  const size_t n_raster = (size_t)f.frames * g.GH * g.GW;
   int ax[4], pi[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -278,11 +297,9 @@ __global__ void __launch_bounds__(kPrologueThreads)
   }
   for (int which = 0; which < 3; ++which) {
     const __nv_bfloat16* __restrict__ dz = a.dz[which];
-    __nv_bfloat16* __restrict__ dx = a.dx[which];
     if (dz == nullptr) continue;
     const bool qk = which < 2;
     const float* gam = qk ? f.gamma[which] : nullptr;
-    const __nv_bfloat16* __restrict__ xin = qk ? a.x[which] : nullptr;
     const bool do_rope = qk && rope;
     float gv[8], gacc[8];
 #pragma unroll
@@ -297,10 +314,10 @@ __global__ void __launch_bounds__(kPrologueThreads)
 #pragma unroll
       for (int e = 0; e < 8; ++e) { v[e] = 0.f; xv[e] = 0.f; }
       size_t xoff = 0;
+      int sidx = 0;
       if (valid) {
         const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
-        const size_t n = ((size_t)t * g.GH + hh) * g.GW + ww;
-        xoff = (((size_t)b * n_raster + n) * g.H + h) * D + c0;
+        xoff = shard_elem(f.sh, g, b, t, hh, ww, h, c0, sidx);
         const uint4 rz = __ldg(reinterpret_cast<const uint4*>(
             dz + ((((size_t)b * g.H + h) * (size_t)(f.nbt * per_t) + blk) * g.BS + slot) * D + c0));
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rz);
@@ -310,7 +327,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
           v[2 * e] = ff.x; v[2 * e + 1] = ff.y;
         }
         if (gam) {
-          const uint4 rx = __ldg(reinterpret_cast<const uint4*>(xin + xoff));
+          const uint4 rx = __ldg(reinterpret_cast<const uint4*>(a.x[which][sidx] + xoff));
           const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&rx);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -357,7 +374,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
         uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) o32[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-        *reinterpret_cast<uint4*>(dx + xoff) = outv;
+        *reinterpret_cast<uint4*>(a.dx[which][sidx] + xoff) = outv;
       }
     }
     if (gam && a.part[which] != nullptr) {

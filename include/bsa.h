@@ -166,6 +166,66 @@ BSA_API bsa_status_t rope3d_qknorm_prologue_bwd(const bsa_geom_t* g, int32_t fra
                                                 float* dgamma_k, void* ws, size_t ws_bytes,
                                                 bsa_stream_t stream);
 
+/* ---- Sequence-parallel (Ulysses) form of the relayouts --------------------------------
+ * Source: "LongCat-Video : Generate 1 minute long AI videos with this model", section
+ * "How to run it" (multi-GPU inference with context parallelism, Ulysses) and the Meituan
+ * talk, section 2.2 (the sparse attention is trained in parallel).  With the raster tensors of
+ * a DiT split by frames over R ranks, rank r runs routing and attention for a slice of the
+ * heads over the whole video: the sequence -> head exchange is folded into the prologue, which
+ * reads every rank's frame shard directly (device pointers of peer GPUs, e.g. from
+ * bsa_ipc_import), and the head -> sequence exchange into the inverse relayout, which writes
+ * into every rank's shard.  No collective library call sits on this path; the caller orders
+ * it with a barrier before the reads of peer shards and after the writes into them.
+ *
+ * Shard s of a raster tensor holds frames [s * shard_frames, (s + 1) * shard_frames) of the
+ * grid being processed as bf16 [B, shard_frames * grid_h * grid_w, heads_total, D]; a call
+ * processes raster heads head0 .. head0 + g->heads - 1 (the geometry describes the local
+ * head slice).  Each shard pointer must be 16-byte aligned; a shard array holds n_shards
+ * pointers (host memory, read during the call). */
+#define BSA_MAX_SHARDS 8
+typedef struct bsa_shards {
+  int32_t n_shards;     /* 1 .. BSA_MAX_SHARDS; n_shards * shard_frames == frames */
+  int32_t shard_frames; /* frames per shard */
+  int32_t heads_total;  /* heads of each raster row */
+  int32_t head0;        /* first raster head of this call */
+} bsa_shards_t;
+
+/* rope3d_qknorm_prologue reading its raster inputs from shards (q_shards / k_shards /
+ * v_shards: arrays of n_shards pointers, or NULL to skip that tensor).  Outputs as there, for
+ * the g->heads local heads. */
+BSA_API bsa_status_t rope3d_qknorm_prologue_sharded(
+    const bsa_geom_t* g, int32_t frames, int32_t t_offset, const bsa_shards_t* sh,
+    const void* const* q_shards, const void* const* k_shards, const void* const* v_shards,
+    const float* gamma_q, const float* gamma_k, float eps, float rope_theta, void* q_blk,
+    void* k_blk, void* v_blk, float* q_pool, float* k_pool, bsa_stream_t stream);
+
+/* rope3d_qknorm_prologue_bwd with sharded raster inputs (q_shards / k_shards, needed with a
+ * gain) and outputs (dq_shards / dk_shards / dv_shards).  dgamma_q / dgamma_k are the
+ * gradients over this call's heads only: the caller sums them over the ranks. */
+BSA_API bsa_status_t rope3d_qknorm_prologue_bwd_sharded(
+    const bsa_geom_t* g, int32_t frames, int32_t t_offset, const bsa_shards_t* sh,
+    const void* const* q_shards, const void* const* k_shards, const float* gamma_q,
+    const float* gamma_k, float eps, float rope_theta, const void* dq_blk, const void* dk_blk,
+    const void* dv_blk, void* const* dq_shards, void* const* dk_shards, void* const* dv_shards,
+    float* dgamma_q, float* dgamma_k, void* ws, size_t ws_bytes, bsa_stream_t stream);
+
+/* Inverse relayout of a blocked bf16 tensor (e.g. the attention output O) of the g->heads
+ * local heads into raster shards (pad slots dropped): the head -> sequence exchange. */
+BSA_API bsa_status_t bsa_blocked_to_raster_sharded(const bsa_geom_t* g, int32_t frames,
+                                                   const bsa_shards_t* sh, const void* x_blk,
+                                                   void* const* x_shards, bsa_stream_t stream);
+
+/* CUDA IPC of device buffers between the processes of one node (plumbing for the shard
+ * pointers above).  bsa_ipc_export writes BSA_IPC_HANDLE_BYTES bytes describing the device
+ * allocation that holds dev_ptr and dev_ptr's offset in it; the exporting process must keep
+ * the buffer alive until every importer has closed it.  bsa_ipc_import maps such a handle from
+ * another process and returns the pointer to the same byte; bsa_ipc_close unmaps it.  A
+ * process cannot import its own handle (BSA_ERR_CUDA). */
+#define BSA_IPC_HANDLE_BYTES 128
+BSA_API bsa_status_t bsa_ipc_export(const void* dev_ptr, void* handle);
+BSA_API bsa_status_t bsa_ipc_import(const void* handle, void** dev_ptr);
+BSA_API bsa_status_t bsa_ipc_close(void* dev_ptr);
+
 /* Block-pooled top-r routing.
  * Sources: "LongCat-Video : Generate 1 minute long AI videos with this model", section
  * "Sparse attention" (blocks chosen by similarity); "LongCat-Video视频生成模型发布…",
