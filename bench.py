@@ -451,6 +451,49 @@ def main():
                                      "cached_t": gc.cached_t}
         del kc_n, vc_n, kp_n
 
+    # sequence-parallel relayouts of one rank of 8 (all shards on this GPU): the sharded
+    # prologue reading 8 frame shards for its 1/8 of the heads, and the inverse relayout of its
+    # O into the 8 shards; bytes = its share of the raster reads / writes plus blocked outputs
+    if w.t_frames % 8 == 0 and w.heads % 8 == 0 and not w.cached_t:
+        from block_sparse_attention_route_b200.ulysses import UlyssesPlan
+        plan = UlyssesPlan(8, 0, w.heads, w.t_frames)
+        gl = plan.local_geometry(g)
+        tps = plan.shard_tokens(g)
+        shq, shk, shv = ([t[:, s * tps:(s + 1) * tps] for s in range(8)] for t in (q_d, k_d, v_d))
+        o_ras = torch.empty_like(q_d)
+        sho = [o_ras[:, s * tps:(s + 1) * tps] for s in range(8)]
+        blk = [torch.empty(bsa.blocked_shape(gl), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+        pools = [torch.empty(bsa.blocked_shape(gl)[:3] + (g.head_dim,), dtype=torch.float32,
+                             device=dev) for _ in range(2)]
+        gq = pipe.gamma_q if w.qknorm else None
+        gk = pipe.gamma_k if w.qknorm else None
+
+        def u_pro():
+            bsa.rope3d_qknorm_prologue_sharded(gl, w.t_frames, 0, plan.shards(), shq, shk, shv, gq,
+                                               gk, w.eps, w.theta if w.rope else 0.0, blk[0],
+                                               blk[1], blk[2], pools[0], pools[1], stream=stream)
+
+        def u_out():
+            bsa.bsa_blocked_to_raster_sharded(gl, w.t_frames, plan.shards(), blk[0], sho,
+                                              stream=stream)
+        u_rows = {}
+        for nm, fn, nbytes in (("prologue", u_pro, 3 * (q_d.numel() // 8) * 2 + 3 * blk[0].numel() * 2),
+                               ("o_relayout", u_out, (q_d.numel() // 8) * 2 + blk[0].numel() * 2)):
+            for _ in range(2):
+                fn()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            for _ in range(args.steps):
+                fn()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            u_rows[nm] = {"ms_per_call": ms, "bytes": nbytes, "gbs": nbytes / (ms * 1e-3) / 1e9}
+        next_rows["ulysses_rank_of_8_local_shards"] = u_rows
+        del blk, pools, o_ras, sho
+
     # routing variants (bsa_route_ex flags) on this workload's q / k: ms per route call
     rv = {}
     for vname, vflags in (("plain", 0), ("force_self", bsa.ROUTE_FORCE_SELF),
