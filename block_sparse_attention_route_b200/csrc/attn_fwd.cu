@@ -16,7 +16,12 @@
 //               w/4 (D/4 columns) of the output
 //   warp 16     TMA producer (one thread)
 //   warp 17     MMA issuer (one thread); owns the TMEM allocation
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D).  S is double buffered: while the
+// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D), Q slots [256+D, 256+2D) (two of
+// D/2 columns: bf16 pairs).  Q is the A operand of S = Q K^T straight from TMEM, so the
+// tensor cores read only K from shared memory for S (a shared-memory-bandwidth saving: an SS
+// MMA pair of 128x16 bf16 tiles reads 8 KB per 64 clocks, the whole 128 B/clock).  The
+// softmax warps copy each item's Q from its staging tile into a Q slot one item ahead.
+// S is double buffered: while the
 // softmax turns S(n) into P(n) (bf16, written over the first BS/2 columns of its buffer),
 // the tensor cores already compute S(n+1).  MMA order: S(0), S(1), then per step PV(n) and
 // S(n+2) into the buffer P(n) came from (tcgen05 MMAs of one thread run in issue order, so
@@ -34,9 +39,13 @@
 // units), so O is rarely touched (and then only after the previous PV has completed, which
 // the pv_done barrier tells); the final O / l and LSE are exact either way.
 //
-// Shared memory: two Q buffers (the next item's Q streams in while the current item runs)
-// and a ring of K/V tiles consumed strictly in the order the MMA thread uses them; the
-// producer walks the identical schedule.
+// Shared memory: two Q staging buffers and a ring of K/V tiles consumed strictly in the order
+// the MMA thread uses them; the producer walks the identical schedule.  Q of the j-th
+// non-empty item of a CTA is staged in buffer j & 1 and copied to TMEM slot j & 1: the
+// producer loads Q(j+1) before the K/V tiles of item j, the softmax warps copy it during step
+// 0 of item j (its slot's previous Q, item j-1's, is no longer read: every S of item j-1
+// completed before S(0) of item j) and free the staging buffer, and the MMA thread waits for
+// the copy before the first S of item j+1.
 #include "common.cuh"
 
 namespace bsa {
@@ -64,8 +73,8 @@ struct FwdLayout {
   static constexpr int kQOff = 0;
   static constexpr int kRingOff = 2 * kQBytes;
   static constexpr int kBarOff = kRingOff + kFwdStages * kKVBytes;
-  // q_full[2] q_empty[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done o_full fin
-  static constexpr int kNumBars = 4 + 2 * kFwdStages + 2 + 2 + 3;
+  // q_full[2] q_empty[2] qt_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done o_full fin
+  static constexpr int kNumBars = 6 + 2 * kFwdStages + 2 + 2 + 3;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kXchOff = kMiscOff + 16;               // float [2 parity][4 groups][128]
   static constexpr int kSumOff = kXchOff + 2 * 4 * 128 * 4;   // float [4 groups][128]
@@ -103,9 +112,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars;            // [2]
-  uint64_t* q_empty = bars + 2;       // [2]
-  uint64_t* kv_full = bars + 4;       // [S]
+  uint64_t* q_full = bars;            // [2] Q staged (TMA)
+  uint64_t* q_empty = bars + 2;       // [2] staging buffer copied out (kSoftmaxThreads arrivals)
+  uint64_t* qt_full = bars + 4;       // [2] Q in its TMEM slot (kSoftmaxThreads arrivals)
+  uint64_t* kv_full = bars + 6;       // [S]
   uint64_t* kv_empty = kv_full + S;   // [S]
   uint64_t* s_full = kv_empty + S;    // [2] S(n) in buffer n & 1
   uint64_t* p_full = s_full + 2;      // [2] P(n) written into buffer n & 1 (kSoftmaxThreads arrivals)
@@ -121,7 +131,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   if (tid == 0) {
     for (int i = 0; i < 2; ++i) {
       mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], 1);
+      mbar_init(&q_empty[i], kSoftmaxThreads);
+      mbar_init(&qt_full[i], kSoftmaxThreads);
       mbar_init(&s_full[i], 1);
       mbar_init(&p_full[i], kSoftmaxThreads);
     }
@@ -153,11 +164,17 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const uint32_t t_o0 = tmem_base + 256;
+  const uint32_t t_q0 = tmem_base + 256 + D;  // Q slot b at t_q0 + b * D / 2
+  // next item with a non-empty selection at or after `it` in this CTA's sequence
+  auto next_item = [&](int it) {
+    while (it < p.n_items && load_cnt(p, it) == 0) it += gridDim.x;
+    return it;
+  };
 
   if (warp == kProducerWarp) {
     // ================================================================ TMA producer
-    // Load order = MMA consumption order: per item Q (own buffer), K(0), K(1), then per step
-    // n: V(n), K(n+2).
+    // Load order = MMA consumption order: per item K(0), K(1), then per step n: V(n),
+    // K(n+2); Q of the next non-empty item is staged before the current item's tiles.
     if (lane == 0) {
       int seq = 0, items = 0;
       bool ok = true;
@@ -179,22 +196,31 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ++seq;
         return true;
       };
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        const int cnt = load_cnt(p, item);
-        if (cnt == 0) continue;
+      // Q of the `items`-th non-empty item into staging buffer items & 1 (free once the
+      // softmax warps copied out the Q two items back)
+      auto q_tile = [&](int item) -> bool {
         const int qb = items & 1;
-        if (items >= 2 && !mbar_wait(&q_empty[qb], ((items >> 1) - 1) & 1, abort_flag)) { ok = false; break; }
+        if (items >= 2 && !mbar_wait(&q_empty[qb], ((items >> 1) - 1) & 1, abort_flag)) return false;
         mbar_expect_tx(&q_full[qb], L::kQBytes);
 #pragma unroll
         for (int half = 0; half < D / 64; ++half)
           tma_load_2d(smem + L::kQOff + qb * L::kQBytes + half * kTileM * 128, &tmQ, half * 64,
                       item * BS, &q_full[qb]);
         ++items;
-        ok = kv_tile(item, 0, false) && (cnt < 2 || kv_tile(item, 1, false));
+        return true;
+      };
+      int item = next_item(blockIdx.x);
+      if (item < p.n_items) ok = q_tile(item);
+      while (item < p.n_items && ok) {
+        const int cnt = load_cnt(p, item);
+        const int nxt = next_item(item + gridDim.x);
+        if (nxt < p.n_items) ok = q_tile(nxt);
+        ok = ok && kv_tile(item, 0, false) && (cnt < 2 || kv_tile(item, 1, false));
         for (int n = 0; n < cnt && ok; ++n) {
           ok = kv_tile(item, n, true);
           if (ok && n + 2 < cnt) ok = kv_tile(item, n + 2, false);
         }
+        item = nxt;
       }
       // drain: every issued TMA load must land before the CTA may exit
       for (int st = 0; st < S; ++st) {
@@ -211,7 +237,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTileM, BS, 0, 0);
       constexpr uint32_t idPV = idesc_bf16(kTileM, D, 0, 1);
-      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
       const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
       const uint64_t dv = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
       int seq = 0, items = 0, gs = 0, gp = 0;  // ring position, items, S issued, P consumed
@@ -222,15 +247,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tc_fence_after();
         return stage;
       };
-      // S(gs) = Q K^T into buffer gs & 1 from the K tile in ring stage `stage`
-      auto mma_S = [&](uint64_t dq, int stage) {
+      // S(gs) = Q K^T into buffer gs & 1: A = Q from TMEM slot a_q (K16 slice kk at column
+      // 8 kk), B = the K tile in ring stage `stage`
+      auto mma_S = [&](uint32_t a_q, int stage) {
         const uint64_t kb = dk + (uint64_t)((stage * L::kKVBytes) >> 4);
         const uint32_t d_s = tmem_base + (gs & 1) * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t offq = ((kk / 4) * (kTileM * 128) + (kk % 4) * 32) >> 4;
           const uint32_t offk = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
-          mma_ss(d_s, dq + offq, kb + offk, idS, kk > 0 ? 1u : 0u);
+          mma_ts(d_s, a_q + kk * 8, kb + offk, idS, kk > 0 ? 1u : 0u);
         }
       };
       // Every wait comes before the MMAs it guards, so each step issues one uninterrupted
@@ -242,7 +267,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         cnt_next = item + (int)gridDim.x < p.n_items ? load_cnt(p, item + gridDim.x) : 0;
         if (cnt == 0) continue;
         const int qb = items & 1;
-        if (!mbar_wait(&q_full[qb], (items >> 1) & 1, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&qt_full[qb], (items >> 1) & 1, abort_flag)) { ok = false; break; }
         ++items;
         const int k0 = wait_tile();
         ++seq;
@@ -250,7 +275,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (cnt >= 2) ++seq;
         if (k0 < 0 || (cnt >= 2 && k1 < 0)) { ok = false; break; }
         tc_fence_after();
-        const uint64_t dq = dq0 + (uint64_t)((qb * L::kQBytes) >> 4);
+        const uint32_t dq = t_q0 + qb * (D / 2);
         const int gs0 = gs;
         mma_S(dq, k0);
         ++gs;
@@ -281,10 +306,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             ++gs;
           }
           mma_commit(pv_done);
-          if (n == cnt - 1) {
-            mma_commit(o_full);
-            mma_commit(&q_empty[qb]);
-          }
+          if (n == cnt - 1) mma_commit(o_full);
           mma_commit(&kv_empty[sv]);
           if (more) mma_commit(&kv_empty[sk]);
           ++gp;
@@ -307,6 +329,33 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     const float sl2 = g.scale * 1.4426950408889634f;
     int gstep = 0, ocons = 0;  // global step (= S buffer use / P / PV index)
     bool ok = true;
+    // This thread's part of Q (row `row`, dims [cg*D/4, (cg+1)*D/4)) of the jj-th non-empty
+    // item: from the 128-byte-swizzled staging tile into TMEM slot jj & 1 as bf16 pairs.
+    auto copy_q = [&](int jj) -> bool {
+      const int qb = jj & 1;
+      bool w_ok = mbar_wait(&q_full[qb], (jj >> 1) & 1, abort_flag);
+      w_ok = __all_sync(0xffffffffu, w_ok);
+      if (!w_ok) return false;
+      constexpr int DC = D / 4;
+      const int d0 = cg * DC, half = d0 / 64, c0 = (d0 % 64) / 8;
+      const unsigned char* tile = smem + L::kQOff + qb * L::kQBytes + half * (kTileM * 128) + row * 128;
+      uint32_t w[DC / 2];
+#pragma unroll
+      for (int c = 0; c < DC / 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(tile + (((c0 + c) ^ (row & 7)) << 4));
+        w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
+      }
+      const uint32_t dst = t_q0 + t_lane + qb * (D / 2) + cg * (DC / 2);
+      if constexpr (DC == 32) tmem_st16(dst, w);
+      else tmem_st8(dst, w);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&qt_full[qb]);
+      mbar_arrive(&q_empty[qb]);
+      return true;
+    };
+    int jq = -1;  // non-empty items started
+    if (next_item(blockIdx.x) < p.n_items) ok = copy_q(0);
     int cnt_next = (int)blockIdx.x < p.n_items ? load_cnt(p, blockIdx.x) : 0;
     for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
       const int cnt = cnt_next;  // the next item's count is fetched one item ahead
@@ -331,6 +380,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         continue;
       }
+      ++jq;
+      const bool has_next = next_item(item + gridDim.x) < p.n_items;
       float m = -INFINITY, l = 0.f;
       // Key-block indices come 32 steps at a time (lane e holds step n0 + e), the next chunk's
       // load in flight while the current one runs; per chunk a ballot marks the steps whose
@@ -428,6 +479,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
+        // the next item's Q into the other slot (every S of the previous item, the slot's
+        // last reader, completed before S(0) of this one)
+        if (n == 0 && has_next && !copy_q(jq + 1)) { ok = false; break; }
       }
       if (!ok) break;
       // combine the four partial row sums
