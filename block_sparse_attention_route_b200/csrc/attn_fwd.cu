@@ -63,7 +63,8 @@ struct FwdParams {
 constexpr int kFwdThreads = 576;
 constexpr int kSoftmaxThreads = 512;
 constexpr int kProducerWarp = 16, kMmaWarp = 17;
-constexpr int kFwdStages = 4;
+constexpr int kFwdStages = 5;
+constexpr int kQBufs = 1;  // Q staging buffers (Q leaves for TMEM at step 0 of the item before)
 constexpr int kTileM = 128;
 
 template <int BS, int D>
@@ -71,7 +72,7 @@ struct FwdLayout {
   static constexpr int kQBytes = kTileM * D * 2;
   static constexpr int kKVBytes = BS * D * 2;
   static constexpr int kQOff = 0;
-  static constexpr int kRingOff = 2 * kQBytes;
+  static constexpr int kRingOff = kQBufs * kQBytes;
   static constexpr int kBarOff = kRingOff + kFwdStages * kKVBytes;
   // q_full[2] q_empty[2] qt_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done o_full fin
   static constexpr int kNumBars = 6 + 2 * kFwdStages + 2 + 2 + 3;
@@ -196,11 +197,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ++seq;
         return true;
       };
-      // Q of the `items`-th non-empty item into staging buffer items & 1 (free once the
-      // softmax warps copied out the Q two items back)
+      // Q of the `items`-th non-empty item into staging buffer items % kQBufs (free once the
+      // softmax warps copied out the Q kQBufs items back)
       auto q_tile = [&](int item) -> bool {
-        const int qb = items & 1;
-        if (items >= 2 && !mbar_wait(&q_empty[qb], ((items >> 1) - 1) & 1, abort_flag)) return false;
+        const int qb = items % kQBufs;
+        if (items >= kQBufs &&
+            !mbar_wait(&q_empty[qb], ((items / kQBufs) - 1) & 1, abort_flag)) return false;
         mbar_expect_tx(&q_full[qb], L::kQBytes);
 #pragma unroll
         for (int half = 0; half < D / 64; ++half)
@@ -227,8 +229,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int loads = seq / S + (st < seq % S ? 1 : 0);
         if (loads > 0) mbar_wait_drain(&kv_full[st], (loads - 1) & 1);
       }
-      for (int b = 0; b < 2; ++b) {
-        const int loads = items / 2 + (b < (items & 1) ? 1 : 0);
+      for (int b = 0; b < kQBufs; ++b) {
+        const int loads = items / kQBufs + (b < items % kQBufs ? 1 : 0);
         if (loads > 0) mbar_wait_drain(&q_full[b], (loads - 1) & 1);
       }
     }
@@ -332,8 +334,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // This thread's part of Q (row `row`, dims [cg*D/4, (cg+1)*D/4)) of the jj-th non-empty
     // item: from the 128-byte-swizzled staging tile into TMEM slot jj & 1 as bf16 pairs.
     auto copy_q = [&](int jj) -> bool {
-      const int qb = jj & 1;
-      bool w_ok = mbar_wait(&q_full[qb], (jj >> 1) & 1, abort_flag);
+      const int qb = jj % kQBufs, slot = jj & 1;
+      bool w_ok = mbar_wait(&q_full[qb], (jj / kQBufs) & 1, abort_flag);
       w_ok = __all_sync(0xffffffffu, w_ok);
       if (!w_ok) return false;
       constexpr int DC = D / 4;
@@ -345,12 +347,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const uint4 v = *reinterpret_cast<const uint4*>(tile + (((c0 + c) ^ (row & 7)) << 4));
         w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
       }
-      const uint32_t dst = t_q0 + t_lane + qb * (D / 2) + cg * (DC / 2);
+      const uint32_t dst = t_q0 + t_lane + slot * (D / 2) + cg * (DC / 2);
       if constexpr (DC == 32) tmem_st16(dst, w);
       else tmem_st8(dst, w);
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(&qt_full[qb]);
+      mbar_arrive(&qt_full[slot]);
       mbar_arrive(&q_empty[qb]);
       return true;
     };
