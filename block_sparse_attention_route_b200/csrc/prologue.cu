@@ -27,13 +27,23 @@ struct RasterShards {
   int h_stride, h0;  // heads of every raster row, first head processed
 };
 
-// Shard and element offset of (b, frame t of the grid, row hh, column ww, head h, channel c0).
-__device__ __forceinline__ size_t shard_elem(const RasterShards& sh, const Geo& g, int b, int t,
-                                             int hh, int ww, int h, int c0, int& s) {
-  s = t / sh.frames;
-  const size_t n = ((size_t)(t - s * sh.frames) * g.GH + hh) * g.GW + ww;
-  const size_t per_shard = (size_t)sh.frames * g.GH * g.GW;
-  return (((size_t)b * per_shard + n) * sh.h_stride + sh.h0 + h) * (size_t)g.D + c0;
+// Element offset of (b, frame t of the grid, row hh, column ww, head h, channel c0) in its
+// shard, and the shard s.  kSharded = false (every single-GPU call: one shard, all heads)
+// compiles to the plain raster offset.
+// n_raster: tokens of the plain tensor (frames * GH * GW).
+template <bool kSharded, int D>
+__device__ __forceinline__ size_t shard_elem(const RasterShards& sh, const Geo& g, size_t n_raster,
+                                             int b, int t, int hh, int ww, int h, int c0, int& s) {
+  if constexpr (!kSharded) {
+    s = 0;
+    const size_t n = ((size_t)t * g.GH + hh) * g.GW + ww;
+    return (((size_t)b * n_raster + n) * g.H + h) * D + c0;
+  } else {
+    s = t / sh.frames;
+    const size_t n = ((size_t)(t - s * sh.frames) * g.GH + hh) * g.GW + ww;
+    const size_t per_shard = (size_t)sh.frames * g.GH * g.GW;
+    return (((size_t)b * per_shard + n) * sh.h_stride + sh.h0 + h) * D + c0;
+  }
 }
 
 struct PrologueArgs {
@@ -73,7 +83,7 @@ __device__ void build_rope_table(const PrologueArgs& a, int ibt, int ibh, int ib
   }
 }
 
-template <int D>
+template <int D, bool kSharded>
 __global__ void __launch_bounds__(kPrologueThreads)
     prologue_kernel(const PrologueArgs a) {
   constexpr int LPR = D / 8;                     // lanes per row
@@ -103,6 +113,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
   const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
   const int rows = kHeadsPerCta * g.BS;  // (slot, head) pairs; heads >= heads_here are skipped
+  const size_t n_raster = (size_t)a.frames * g.GH * g.GW;
 
   // RoPE coordinates of this lane's 4 channel pairs: axis (0 t, 1 h, 2 w) and pair index.
   int ax[4], pi[4];
@@ -116,7 +127,8 @@ __global__ void __launch_bounds__(kPrologueThreads)
 
   for (int which = 0; which < 3; ++which) {
     __nv_bfloat16* __restrict__ y = a.y[which];
-    if (a.x[which][0] == nullptr) continue;
+    const __nv_bfloat16* __restrict__ x0 = a.x[which][0];  // the one shard of a plain call
+    if (x0 == nullptr) continue;
     const bool qk = which < 2;
     const float* gam = qk ? a.gamma[which] : nullptr;
     const bool do_rope = qk && rope;
@@ -139,8 +151,8 @@ __global__ void __launch_bounds__(kPrologueThreads)
       if (valid) {
         const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
         int sidx;
-        const size_t off = shard_elem(a.sh, g, b, t, hh, ww, h, c0, sidx);
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>(a.x[which][sidx] + off));
+        const size_t off = shard_elem<kSharded, D>(a.sh, g, n_raster, b, t, hh, ww, h, c0, sidx);
+        const uint4 raw = __ldg(reinterpret_cast<const uint4*>((kSharded ? a.x[which][sidx] : x0) + off));
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -229,15 +241,13 @@ cudaError_t launch_prologue(const PrologueArgs& a, cudaStream_t s) {
   const Geo& g = a.g;
   dim3 grid(a.nbt * g.nbh * g.nbw, (g.H + kHeadsPerCta - 1) / kHeadsPerCta, g.B);
   size_t smem = prologue_smem_bytes(g, a.dt, a.dh, a.dw);
-  if (g.D == 128) {
-    cudaFuncSetAttribute(prologue_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    prologue_kernel<128><<<grid, kPrologueThreads, smem, s>>>(a);
-  } else {
-    cudaFuncSetAttribute(prologue_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         (int)smem);
-    prologue_kernel<64><<<grid, kPrologueThreads, smem, s>>>(a);
-  }
+  const bool plain = a.sh.n == 1 && a.sh.h_stride == g.H && a.sh.h0 == 0;
+  auto go = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<grid, kPrologueThreads, smem, s>>>(a);
+  };
+  if (g.D == 128) plain ? go(prologue_kernel<128, false>) : go(prologue_kernel<128, true>);
+  else plain ? go(prologue_kernel<64, false>) : go(prologue_kernel<64, true>);
   return cudaGetLastError();
 }
 
@@ -260,7 +270,7 @@ struct PrologueBwdArgs {
   float* part[2];                 // [n_cta][D] dgamma partials of q, k
 };
 
-template <int D>
+template <int D, bool kSharded>
 __global__ void __launch_bounds__(kPrologueThreads)
     prologue_bwd_kernel(const PrologueBwdArgs a) {
   constexpr int LPR = D / 8;                     // lanes per row
@@ -287,6 +297,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
   const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
   const int rows = kHeadsPerCta * g.BS;
+  const size_t n_raster = (size_t)f.frames * g.GH * g.GW;
   int ax[4], pi[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) {
@@ -301,6 +312,9 @@ __global__ void __launch_bounds__(kPrologueThreads)
     const bool qk = which < 2;
     const float* gam = qk ? f.gamma[which] : nullptr;
     const bool do_rope = qk && rope;
+    // the one shard of a plain call
+    const __nv_bfloat16* __restrict__ xin0 = qk ? a.x[which][0] : nullptr;
+    __nv_bfloat16* __restrict__ dx0 = a.dx[which][0];
     float gv[8], gacc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) { gv[e] = gam ? gam[c0 + e] : 1.f; gacc[e] = 0.f; }
@@ -317,7 +331,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
       int sidx = 0;
       if (valid) {
         const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
-        xoff = shard_elem(f.sh, g, b, t, hh, ww, h, c0, sidx);
+        xoff = shard_elem<kSharded, D>(f.sh, g, n_raster, b, t, hh, ww, h, c0, sidx);
         const uint4 rz = __ldg(reinterpret_cast<const uint4*>(
             dz + ((((size_t)b * g.H + h) * (size_t)(f.nbt * per_t) + blk) * g.BS + slot) * D + c0));
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rz);
@@ -327,7 +341,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
           v[2 * e] = ff.x; v[2 * e + 1] = ff.y;
         }
         if (gam) {
-          const uint4 rx = __ldg(reinterpret_cast<const uint4*>(a.x[which][sidx] + xoff));
+          const uint4 rx = __ldg(reinterpret_cast<const uint4*>((kSharded ? a.x[which][sidx] : xin0) + xoff));
           const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&rx);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
@@ -374,7 +388,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
         uint32_t* o32 = reinterpret_cast<uint32_t*>(&outv);
 #pragma unroll
         for (int e = 0; e < 4; ++e) o32[e] = pack_bf16x2(v[2 * e], v[2 * e + 1]);
-        *reinterpret_cast<uint4*>(a.dx[which][sidx] + xoff) = outv;
+        *reinterpret_cast<uint4*>((kSharded ? a.dx[which][sidx] : dx0) + xoff) = outv;
       }
     }
     if (gam && a.part[which] != nullptr) {
@@ -409,13 +423,13 @@ cudaError_t launch_prologue_bwd(const PrologueBwdArgs& a, float* dgamma[2], cuda
   dim3 grid(a.f.nbt * g.nbh * g.nbw, (g.H + kHeadsPerCta - 1) / kHeadsPerCta, g.B);
   const size_t smem = (size_t)2 * g.D * sizeof(float) +
                       (size_t)(g.bt * (a.f.dt / 2) + g.bh * (a.f.dh / 2) + g.bw * (a.f.dw / 2)) * sizeof(float2);
-  if (g.D == 128) {
-    cudaFuncSetAttribute(prologue_bwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    prologue_bwd_kernel<128><<<grid, kPrologueThreads, smem, s>>>(a);
-  } else {
-    cudaFuncSetAttribute(prologue_bwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    prologue_bwd_kernel<64><<<grid, kPrologueThreads, smem, s>>>(a);
-  }
+  const bool plain = a.f.sh.n == 1 && a.f.sh.h_stride == g.H && a.f.sh.h0 == 0;
+  auto go = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<grid, kPrologueThreads, smem, s>>>(a);
+  };
+  if (g.D == 128) plain ? go(prologue_bwd_kernel<128, false>) : go(prologue_bwd_kernel<128, true>);
+  else plain ? go(prologue_bwd_kernel<64, false>) : go(prologue_bwd_kernel<64, true>);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int n_cta = (int)(grid.x * grid.y * grid.z);
