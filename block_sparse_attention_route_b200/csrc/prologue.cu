@@ -112,7 +112,11 @@ __global__ void __launch_bounds__(kPrologueThreads)
 
   const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
   const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
-  const int rows = kHeadsPerCta * g.BS;  // (slot, head) pairs; heads >= heads_here are skipped
+  // (slot, head) pairs, head fastest.  A sharded call (a rank's slice of the heads, often
+  // fewer than 8) spreads its rows over the heads present; the plain path keeps the constant
+  // stride and skips the missing heads of a last, partial group.
+  const int hpc = kSharded ? heads_here : kHeadsPerCta;
+  const int rows = hpc * g.BS;
   const size_t n_raster = (size_t)a.frames * g.GH * g.GW;
 
   // RoPE coordinates of this lane's 4 channel pairs: axis (0 t, 1 h, 2 w) and pair index.
@@ -142,7 +146,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
     int cur_h = -1;
     for (int base = 0; base < rows; base += RPP) {
       const int row = base + rid;
-      const int hl = row % kHeadsPerCta, slot = row / kHeadsPerCta;
+      const int hl = row % hpc, slot = row / hpc;
       const bool in = row < rows && hl < heads_here;
       const int h = hg * kHeadsPerCta + hl;
       const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
@@ -296,7 +300,8 @@ __global__ void __launch_bounds__(kPrologueThreads)
 
   const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
   const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
-  const int rows = kHeadsPerCta * g.BS;
+  const int hpc = kSharded ? heads_here : kHeadsPerCta;  // as in the forward
+  const int rows = hpc * g.BS;
   const size_t n_raster = (size_t)f.frames * g.GH * g.GW;
   int ax[4], pi[4];
 #pragma unroll
@@ -320,7 +325,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
     for (int e = 0; e < 8; ++e) { gv[e] = gam ? gam[c0 + e] : 1.f; gacc[e] = 0.f; }
     for (int base = 0; base < rows; base += RPP) {
       const int row = base + rid;
-      const int hl = row % kHeadsPerCta, slot = row / kHeadsPerCta;
+      const int hl = row % hpc, slot = row / hpc;
       const int h = hg * kHeadsPerCta + hl;
       const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
       const bool valid = row < rows && hl < heads_here && lt < vt && lh < vh && lw < vw;
