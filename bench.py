@@ -325,7 +325,7 @@ def main():
             all_marks.append(step(True))
         t1.record(stream)
         torch.cuda.synchronize()
-    ktimes = bsa.bsa_kernel_times()
+    ktimes = bsa.bsa_kernel_time_stats()
     bsa.bsa_kernel_timing(False)
     barrier()
     ms = t0.elapsed_time(t1) / args.steps
@@ -522,12 +522,12 @@ def main():
               "bwd_dkdv": 2 * tile_flops(g.bs, g.head_dim, n_pairs_cur),
               "bwd_dq": 1.5 * tile_flops(g.bs, g.head_dim, n_pairs)}
     kernels = {}
-    for kname, (nl, tot_ms) in ktimes.items():
+    for kname, (nl, tot_ms, min_ms, med_ms) in ktimes.items():
         if nl == 0:
             continue
         avg = tot_ms / nl
-        kernels[kname] = {"launches": nl, "ms_per_launch": avg,
-                          "tflops": kflops[kname] / (avg * 1e-3) / 1e12}
+        kernels[kname] = {"launches": nl, "ms_per_launch": avg, "ms_median": med_ms,
+                          "ms_min": min_ms, "tflops": kflops[kname] / (avg * 1e-3) / 1e12}
     dom = max(kernels, key=lambda k_: kernels[k_]["ms_per_launch"])
     achieved = kernels[dom]["tflops"]
     value = world * fl_step / (ms_max * 1e-3) / 1e12

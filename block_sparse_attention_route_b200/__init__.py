@@ -24,7 +24,7 @@ __all__ = [
     "Shards", "MAX_SHARDS", "IPC_HANDLE_BYTES", "rope3d_qknorm_prologue_sharded",
     "rope3d_qknorm_prologue_bwd_sharded", "bsa_blocked_to_raster_sharded", "bsa_ipc_export",
     "bsa_ipc_import", "bsa_ipc_close",
-    "bsa_kernel_timing", "bsa_kernel_times",
+    "bsa_kernel_timing", "bsa_kernel_times", "bsa_kernel_time_stats",
     "WS_ROUTE", "WS_FWD", "WS_BWD", "WS_PROLOGUE_BWD",
 ]
 
@@ -163,6 +163,7 @@ def lib() -> ctypes.CDLL:
             "bsa_ipc_import": (I32, [P, ctypes.POINTER(ctypes.c_void_p)]),
             "bsa_ipc_close": (I32, [P]),
             "bsa_kernel_times": (I32, [P, P]),
+            "bsa_kernel_time_stats": (I32, [P, P, P, P]),
             "bsa_error_string": (ctypes.c_char_p, [I32]),
             "bsa_last_error_detail": (ctypes.c_char_p, []),
         }
@@ -371,6 +372,18 @@ def bsa_kernel_times() -> dict:
     ms = (ctypes.c_float * len(TIMED_KERNELS))()
     _check(lib().bsa_kernel_times(ctypes.addressof(n), ctypes.addressof(ms)), "bsa_kernel_times")
     return {k: (int(n[i]), float(ms[i])) for i, k in enumerate(TIMED_KERNELS)}
+
+
+def bsa_kernel_time_stats() -> dict:
+    """Per timed kernel: (launches, total ms, min ms, median ms) since the last call."""
+    k_ = len(TIMED_KERNELS)
+    n = (ctypes.c_int32 * k_)()
+    tot, mn, med = ((ctypes.c_float * k_)() for _ in range(3))
+    _check(lib().bsa_kernel_time_stats(ctypes.addressof(n), ctypes.addressof(tot),
+                                       ctypes.addressof(mn), ctypes.addressof(med)),
+           "bsa_kernel_time_stats")
+    return {k: (int(n[i]), float(tot[i]), float(mn[i]), float(med[i]))
+            for i, k in enumerate(TIMED_KERNELS)}
 
 
 def bsa_device_status(stream=None) -> int:

@@ -4,6 +4,7 @@
 // the single per-device status word without relocatable device code.  Host code here
 // validates arguments, derives the block geometry, encodes TMA tensor maps and enqueues the
 // kernels on the caller's stream.  It allocates no device memory.
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -716,15 +717,18 @@ bsa_status_t bsa_kernel_timing(int32_t on) {
   return BSA_OK;
 }
 
-bsa_status_t bsa_kernel_times(int32_t* launches, float* total_ms) {
+bsa_status_t bsa_kernel_time_stats(int32_t* launches, float* total_ms, float* min_ms,
+                                   float* median_ms) {
   t_detail.clear();
   if (!launches || !total_ms) return fail(BSA_ERR_INVALID_ARG, "launches and total_ms are required");
   KernelTimer& t = kernel_timer();
   std::lock_guard<std::mutex> lk(t.mu);
   bsa_status_t st = BSA_OK;
+  std::vector<float> each;
   for (int k = 0; k < kNumTimed; ++k) {
     launches[k] = 0;
     total_ms[k] = 0.f;
+    each.clear();
     for (auto& pr : t.pending[k]) {
       float ms = 0.f;
       cudaError_t e = cudaEventSynchronize(pr.second);
@@ -732,12 +736,21 @@ bsa_status_t bsa_kernel_times(int32_t* launches, float* total_ms) {
       if (e != cudaSuccess && st == BSA_OK) st = cuda_fail(e, "kernel timing event");
       ++launches[k];
       total_ms[k] += ms;
+      each.push_back(ms);
       t.pool.push_back(pr.first);
       t.pool.push_back(pr.second);
     }
     t.pending[k].clear();
+    std::sort(each.begin(), each.end());
+    const size_t n = each.size();
+    if (min_ms) min_ms[k] = n ? each[0] : 0.f;
+    if (median_ms) median_ms[k] = n ? (n % 2 ? each[n / 2] : 0.5f * (each[n / 2 - 1] + each[n / 2])) : 0.f;
   }
   return st;
+}
+
+bsa_status_t bsa_kernel_times(int32_t* launches, float* total_ms) {
+  return bsa_kernel_time_stats(launches, total_ms, nullptr, nullptr);
 }
 
 bsa_status_t bsa_device_status(bsa_stream_t stream) {

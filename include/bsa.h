@@ -316,6 +316,10 @@ BSA_API bsa_status_t bsa_attn_bwd(const bsa_geom_t* g, int32_t top_r, const void
 #define BSA_NUM_TIMED 3
 BSA_API bsa_status_t bsa_kernel_timing(int32_t on);
 BSA_API bsa_status_t bsa_kernel_times(int32_t* launches, float* total_ms);
+/* As bsa_kernel_times, plus the shortest and the median launch of each kernel (min_ms,
+ * median_ms: BSA_NUM_TIMED entries each, or NULL); 0 for a kernel with no launch. */
+BSA_API bsa_status_t bsa_kernel_time_stats(int32_t* launches, float* total_ms, float* min_ms,
+                                           float* median_ms);
 
 /* Waits for `stream`, then reads and clears the current device's status word.
  * Returns BSA_OK, BSA_ERR_TIMEOUT or BSA_ERR_BAD_INDEX (or BSA_ERR_CUDA). */

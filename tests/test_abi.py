@@ -96,6 +96,7 @@ def test_kernel_timing_bookkeeping_without_launches():
     assert bsa.bsa_kernel_times() == {k: (0, 0.0) for k in bsa.TIMED_KERNELS}
     bsa.bsa_kernel_timing(False)
     assert bsa.bsa_kernel_times() == {k: (0, 0.0) for k in bsa.TIMED_KERNELS}
+    assert bsa.bsa_kernel_time_stats() == {k: (0, 0.0, 0.0, 0.0) for k in bsa.TIMED_KERNELS}
 
 
 def test_prologue_bwd_host_validation():

@@ -124,6 +124,23 @@ def test_kernel_timing_counts_each_attention_launch():
     assert all(ms > 0 for _, ms in t.values())
 
 
+def test_kernel_time_stats_min_median():
+    """Three forward launches: min <= median <= mean, all three counted."""
+    import block_sparse_attention_route_b200 as bsa
+    w = WORKLOADS["small"]
+    pipe, _ = run_fwd_bwd(w)
+    bsa.bsa_kernel_timing(True)
+    try:
+        for _ in range(3):
+            pipe.attn_fwd()
+        st = bsa.bsa_kernel_time_stats()
+    finally:
+        bsa.bsa_kernel_timing(False)
+    n, tot, mn, med = st["fwd"]
+    assert n == 3 and st["bwd_dkdv"][0] == 0
+    assert 0 < mn <= med <= tot / n * 1.5 and mn <= tot / n
+
+
 def test_backward_two_segment_mask():
     from synth import Workload
     w = Workload("two_segment", 1, 2, 128, 12, 10, 20, (4, 4, 8), 5, rope=True, cond_t=4)
