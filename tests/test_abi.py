@@ -150,3 +150,29 @@ def test_route_variant_host_validation():
     with pytest.raises(bsa.BsaError) as ei:
         bsa.bsa_block_pool(g, 0, bsa.POOL_MAX, 16, 16, stream=0)
     assert ei.value.code == 1
+
+
+def test_sharded_relayout_host_validation():
+    g = _g(heads=4)  # a rank's slice: 4 of 32 heads
+    ok = bsa.Shards(8, 3, 32, 28)
+    cases = [  # (shards, q shard list) -> expected code
+        (bsa.Shards(9, 3, 32, 0), [16] * 9),    # more shards than supported
+        (bsa.Shards(8, 2, 32, 0), [16] * 8),    # 8 x 2 frames != 24
+        (bsa.Shards(8, 3, 32, 29), [16] * 8),   # heads 29..32 outside 0..31
+        (bsa.Shards(8, 3, 2, 0), [16] * 8),     # fewer raster heads than the call's
+        (ok, [16] * 7 + [None]),                # a missing shard
+        (ok, [16] * 7 + [24]),                  # a misaligned shard
+    ]
+    for sh, qs in cases:
+        with pytest.raises(bsa.BsaError) as ei:
+            bsa.rope3d_qknorm_prologue_sharded(g, 24, 0, sh, qs, None, None, None, None, 1e-6,
+                                               1e4, 16, None, None, stream=0)
+        assert ei.value.code == 1, (sh, qs)
+    with pytest.raises(bsa.BsaError) as ei:  # the inverse relayout needs its shard table
+        bsa.bsa_blocked_to_raster_sharded(g, 24, ok, 16, None, stream=0)
+    assert ei.value.code == 1
+    with pytest.raises(bsa.BsaError) as ei:  # a gain needs the raster q shards
+        bsa.rope3d_qknorm_prologue_bwd_sharded(g, 24, 0, ok, None, None, 16, None, 1e-6, 1e4,
+                                               16, None, None, [16] * 8, None, None, 16, None,
+                                               stream=0)
+    assert ei.value.code == 1
