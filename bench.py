@@ -425,14 +425,15 @@ def main():
                                      "gbs": p_bytes / (p_ms * 1e-3) / 1e9}
 
     # the continuation cache for the next round: this geometry's blocked K, V and key-block
-    # means appended to a cache of as many frames (the same tensors stand in for it)
+    # means appended to a cache of as many frames (the blocked Q, O and Q means stand in for
+    # it: distinct buffers, so no source is read twice through L2)
     if w.t_frames % w.blk[0] == 0:
         gc = dataclasses.replace(g, cached_t=w.t_frames)
         cshape = (g.batch, g.heads, 2 * g.nbq, g.bs, g.head_dim)
         kc_n = torch.empty(cshape, dtype=torch.bfloat16, device=dev)
         vc_n = torch.empty_like(kc_n)
         kp_n = torch.empty(cshape[:3] + (g.head_dim,), dtype=torch.float32, device=dev)
-        ca = lambda: bsa.bsa_cache_append(gc, pipe.k, pipe.v, pipe.k_pool, pipe.k, pipe.v,  # noqa: E731
+        ca = lambda: bsa.bsa_cache_append(gc, pipe.q, pipe.o, pipe.q_pool, pipe.k, pipe.v,  # noqa: E731
                                           pipe.k_pool, kc_n, vc_n, kp_n, stream=stream)
         for _ in range(2):
             ca()
