@@ -184,33 +184,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   return d;
 }
 
-// 2^x for a pair on the FMA pipe (no MUFU): Cody-Waite style split x = j + f with j the
-// nearest integer (magic-constant rounding) and f in [-1/2, 1/2], a degree-3 polynomial
-// for 2^f (coefficients fitted here to a 7.5e-5 relative error bound, far below the bf16
-// rounding of P), then j added to the exponent field.  Inputs must be finite and >= -126
-// (the caller clamps); outputs for x in [-126, 8] are within 1e-4 relative of 2^x.
-__device__ __forceinline__ void exp2_poly2(uint64_t x, float& r0, float& r1) {
-  const uint64_t kRnd = f2pack(12582912.0f, 12582912.0f);     // 1.5 * 2^23
-  const uint64_t kNRnd = f2pack(-12582912.0f, -12582912.0f);
-  const uint64_t kNeg1 = f2pack(-1.0f, -1.0f);
-  const uint64_t c3 = f2pack(0.055171605f, 0.055171605f);
-  const uint64_t c2 = f2pack(0.24261111f, 0.24261111f);
-  const uint64_t c1 = f2pack(0.69326097f, 0.69326097f);
-  const uint64_t c0 = f2pack(0.99992806f, 0.99992806f);
-  const uint64_t t = add2(x, kRnd);           // j + 1.5*2^23 (j in the low mantissa bits)
-  const uint64_t j = add2(t, kNRnd);          // j as float
-  const uint64_t f = fma2(j, kNeg1, x);       // x - j, exact
-  uint64_t pp = fma2(f, c3, c2);
-  pp = fma2(pp, f, c1);
-  pp = fma2(pp, f, c0);
-  float p0, p1, t0, t1;
-  f2unpack(pp, p0, p1);
-  f2unpack(t, t0, t1);
-  // (bits(t) << 23) == (j << 23) modulo 2^32, since the magic constant's bits vanish
-  r0 = __uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23));
-  r1 = __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23));
-}
-
 // Valid-key mask of a block with valid extents (vt, vh, vw) out of (bt, bh, bw): bit c of
 // the BS-bit mask is set iff slot c = (lt*bh + lh)*bw + lw is a real token.  Division-free.
 template <int BS>
