@@ -22,7 +22,12 @@ What it computes, with the page passages each step follows:
 * Block-causal mask and cached conditioning-frame K/V -- the Meituan talk, section 2.1
   ("Block-Causal" attention enabling a cache for continuation); "LongCat-Video : Generate 1
   minute long AI videos with this model", section "The core idea" (KV caching of the fixed
-  conditioning frames).
+  conditioning frames).  Causal chunks and the two-segment form (conditioning frames attend
+  only among themselves) are one segment rule on absolute frames (``Grid``).
+* Routing variants the pages leave open -- "LongCat-Video : Generate 1 minute long AI videos
+  with this model", section "Sparse attention" (a block keeps its own company plus the
+  relevant neighbours): the forced self-block, one selection shared by all heads (scores
+  summed over the heads), and sum / channel-max block pooling (``route`` keywords).
 
 Where the pages are silent, this file takes these readings: mean pooling
 over valid tokens, unscaled block scores, routing per (batch, head) on post-prologue q/k,
