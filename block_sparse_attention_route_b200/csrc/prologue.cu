@@ -144,7 +144,26 @@ __global__ void __launch_bounds__(kPrologueThreads)
     }
     float psum[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     int cur_h = -1;
+    // this lane's 16 bytes of the row of pass `bs` (zero for pad slots and absent heads); the
+    // next pass's load is issued before the current pass is processed, so two are in flight
+    auto fetch = [&](int bs) -> uint4 {
+      const int row = bs + rid;
+      const int hl = row % hpc, slot = row / hpc;
+      const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
+      uint4 r = make_uint4(0u, 0u, 0u, 0u);
+      if (row < rows && hl < heads_here && lt < vt && lh < vh && lw < vw) {
+        const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
+        int sidx;
+        const size_t off = shard_elem<kSharded, D>(a.sh, g, n_raster, b, t, hh, ww,
+                                                   hg * kHeadsPerCta + hl, c0, sidx);
+        r = __ldg(reinterpret_cast<const uint4*>((kSharded ? a.x[which][sidx] : x0) + off));
+      }
+      return r;
+    };
+    uint4 nxt = fetch(0);
     for (int base = 0; base < rows; base += RPP) {
+      const uint4 raw = nxt;
+      if (base + RPP < rows) nxt = fetch(base + RPP);
       const int row = base + rid;
       const int hl = row % hpc, slot = row / hpc;
       const bool in = row < rows && hl < heads_here;
@@ -152,20 +171,13 @@ __global__ void __launch_bounds__(kPrologueThreads)
       const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
       const bool valid = in && lt < vt && lh < vh && lw < vw;
       float v[8];
-      if (valid) {
-        const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
-        int sidx;
-        const size_t off = shard_elem<kSharded, D>(a.sh, g, n_raster, b, t, hh, ww, h, c0, sidx);
-        const uint4 raw = __ldg(reinterpret_cast<const uint4*>((kSharded ? a.x[which][sidx] : x0) + off));
+      {
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float2 f = __bfloat1622float2(p2[e]);
           v[2 * e] = f.x; v[2 * e + 1] = f.y;
         }
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
       }
       if (gam) {  // RMSNorm over the row: every lane takes part in the shuffles
         float ss = 0.f;
