@@ -122,3 +122,17 @@ def test_exchange_and_index_map_match_all_to_all(world):
     for p in procs:
         p.join(timeout=60)
     assert sorted(res) == [(r, "ok") for r in range(world)], res
+
+
+def test_rank_runner_rejects_inconsistent_setups_before_allocating():
+    import block_sparse_attention_route_b200 as bsa
+    from block_sparse_attention_route_b200.ulysses import UlyssesBsa
+    g = bsa.Geometry(1, 32, 128, 24, 45, 80)
+    with pytest.raises(ValueError):  # a continuation cache is not sequence-parallel here
+        UlyssesBsa(UlyssesPlan(8, 0, 32, 24), bsa.Geometry(1, 32, 128, 24, 45, 80, cached_t=4), 72, {})
+    with pytest.raises(ValueError):  # plan for other heads than the geometry's
+        UlyssesBsa(UlyssesPlan(8, 0, 16, 24), g, 72, {})
+    with pytest.raises(ValueError):  # plan for other frames
+        UlyssesBsa(UlyssesPlan(8, 0, 32, 16), g, 72, {})
+    gl = UlyssesPlan(8, 3, 32, 24).local_geometry(g)
+    assert (gl.heads, gl.t_frames, gl.grid_h) == (4, 24, 45)
