@@ -697,3 +697,31 @@ def test_two_segment_conditioning_rows_ignore_the_generated_frames():
     # the generated frames' rows are routed as without any mask
     idn, _, _ = oracle.route(x["q"], x["k"], Grid(8, 10, 20, (4, 4, 8)), w.top_r)
     assert np.array_equal(idn[:, :, per_t:], idx[:, :, per_t:])
+
+
+def test_continuation_rounds_equal_one_causal_pass():
+    """Three rounds of 4 frames, each with the earlier frames as its cache, against one pass
+    over all 12 frames with 4-frame causal chunks: same selections (global key-block ids) and
+    the same O / LSE on every round's rows."""
+    rng = np.random.default_rng(8)
+    T, gh, gw, blk, r = 12, 6, 12, (4, 4, 8), 3
+    D = 16
+    q, k, v = (rng.standard_normal((1, T * gh * gw, 2, D)) for _ in range(3))
+    full = Grid(T, gh, gw, blk, chunk_t=4)
+    scale = 1.0 / math.sqrt(D)
+    idx_f, cnt_f, _ = oracle.route(q, k, full, r)
+    o_f, lse_f = oracle.attend(q, k, v, idx_f, full, scale)
+    per_round = 4 * gh * gw
+    nb_round = full.nbq // 3
+    for rd in range(3):
+        g = Grid(4, gh, gw, blk, cached_t=4 * rd, chunk_t=4)
+        cur = slice(rd * per_round, (rd + 1) * per_round)
+        past = slice(0, rd * per_round)
+        kc = k[:, past] if rd else None
+        vc = v[:, past] if rd else None
+        idx, cnt, _ = oracle.route(q[:, cur], k[:, cur], g, r, k_cache=kc)
+        rows = slice(rd * nb_round, (rd + 1) * nb_round)
+        assert np.array_equal(idx, idx_f[:, :, rows]) and np.array_equal(cnt, cnt_f[:, :, rows])
+        o, lse = oracle.attend(q[:, cur], k[:, cur], v[:, cur], idx, g, scale, k_cache=kc, v_cache=vc)
+        np.testing.assert_allclose(o, o_f[:, cur], atol=1e-12)
+        np.testing.assert_allclose(lse, lse_f[:, cur], atol=1e-12)
