@@ -477,13 +477,18 @@ def attend(q, k, v, idx, grid: Grid, scale: float, k_cache=None, v_cache=None,
     return o, lse
 
 
-def attend_bwd(q, k, v, do, idx, grid: Grid, scale: float, k_cache=None, v_cache=None):
+def attend_bwd(q, k, v, do, idx, grid: Grid, scale: float, k_cache=None, v_cache=None,
+               query_blocks: Optional[List[Tuple[int, int, int]]] = None):
     """Gradients of sum(dO * O) for O = attend(...): closed form per query block.
 
     With P the softmax over the selected key tokens and dP = dO V^T:
       dS = P * (dP - rowsum(dO * O)),  dQ = scale * dS K,  dK += scale * dS^T Q,  dV += P^T dO.
     Gradients reach current keys/values only (cached ones are constants).  Returns raster
     dq, dk, dv [B, N, H, D].
+
+    ``query_blocks`` restricts the work to (b, h, i) triples: dQ of those blocks is then
+    complete, and dK / dV of a key block are complete when every query block that selected it
+    is listed (the rest of dK / dV holds partial sums).
     """
     cur = grid.block_members(grid.t_frames)
     cache = grid.block_members(grid.cached_t) if grid.nbc else []
@@ -491,31 +496,32 @@ def attend_bwd(q, k, v, do, idx, grid: Grid, scale: float, k_cache=None, v_cache
     dq = np.zeros((B, N, H, D))
     dk = np.zeros((B, N, H, D))
     dv = np.zeros((B, N, H, D))
-    for b in range(B):
-        for h in range(H):
-            for i in range(grid.nbq):
-                qi = cur[i]
-                toks = _key_tokens(grid, idx[b, h, i], cur, cache)
-                if not qi or not toks:
-                    continue
-                qm = np.asarray(q[b, qi, h], dtype=np.float64)
-                km = _gather(k, k_cache, toks, b, h)
-                vm = _gather(v, v_cache, toks, b, h)
-                dom = np.asarray(do[b, qi, h], dtype=np.float64)
-                logits = qm @ km.T * scale
-                e = np.exp(logits - logits.max(axis=1, keepdims=True))
-                p = e / e.sum(axis=1, keepdims=True)
-                om = p @ vm
-                dp = dom @ vm.T
-                delta = np.sum(dom * om, axis=1, keepdims=True)
-                ds = p * (dp - delta)
-                dq[b, qi, h] = scale * ds @ km
-                dkm = scale * ds.T @ qm
-                dvm = p.T @ dom
-                for row, (src, t) in enumerate(toks):
-                    if src == "k":
-                        dk[b, t, h] += dkm[row]
-                        dv[b, t, h] += dvm[row]
+    todo = query_blocks if query_blocks is not None else \
+        [(b, h, i) for b in range(B) for h in range(H) for i in range(grid.nbq)]
+    for b, h, i in todo:
+        qi = cur[i]
+        toks = _key_tokens(grid, idx[b, h, i], cur, cache)
+        if not qi or not toks:
+            continue
+        qm = np.asarray(q[b, qi, h], dtype=np.float64)
+        km = _gather(k, k_cache, toks, b, h)
+        vm = _gather(v, v_cache, toks, b, h)
+        dom = np.asarray(do[b, qi, h], dtype=np.float64)
+        logits = qm @ km.T * scale
+        e = np.exp(logits - logits.max(axis=1, keepdims=True))
+        p = e / e.sum(axis=1, keepdims=True)
+        om = p @ vm
+        dp = dom @ vm.T
+        delta = np.sum(dom * om, axis=1, keepdims=True)
+        ds = p * (dp - delta)
+        dq[b, qi, h] = scale * ds @ km
+        dkm = scale * ds.T @ qm
+        dvm = p.T @ dom
+        # scatter-add into the current keys' rows (each key token occurs once per list)
+        rows = [row for row, (src, _) in enumerate(toks) if src == "k"]
+        dst = [t for src, t in toks if src == "k"]
+        dk[b, dst, h] += dkm[rows]
+        dv[b, dst, h] += dvm[rows]
     return dq, dk, dv
 
 

@@ -66,6 +66,69 @@ def check_bwd(w, pipe, x, heads):
     return {n: float(np.max(d)) for n, d in errs}
 
 
+def check_bwd_sampled(w, pipe, x, plan, seed):
+    """Sampled backward parity.  ``plan`` lists (head, extra random key blocks); per head: dQ
+    of 6 full and 2 partial query blocks, dK / dV of the key block with the longest reverse
+    list, the least-selected one (exactly zero if no query block chose it), the most-selected
+    partial block and the random extras.  The oracle runs only the query blocks that selected
+    those key blocks (their dK / dV are then complete) and the dQ sample.  Returns the longest
+    reverse list seen."""
+    grid = grid_of(w)
+    sm = grid.slot_map(w.t_frames)
+    idx = pipe.idx.cpu().numpy()
+    nbq = grid.nbq
+    n_valid = (sm >= 0).sum(axis=1)
+    partial = np.nonzero(n_valid < grid.bs)[0]
+    full = np.setdiff1d(np.arange(nbq), partial)
+    rng = np.random.default_rng(seed)
+    errs = {"dq": [], "dk": [], "dv": []}
+    longest = 0
+    for h, n_rand in plan:
+        sel = idx[0, h]
+        uses = np.bincount(sel[sel >= 0], minlength=nbq)
+        kb = [int(np.argmax(uses)), int(np.argmin(uses))]
+        if partial.size:
+            kb.append(int(partial[np.argmax(uses[partial])]))
+        kb += [int(j) for j in rng.choice(np.setdiff1d(np.arange(nbq), kb), n_rand, replace=False)]
+        qs = [int(i) for i in rng.choice(full, min(6, full.size), replace=False)]
+        if partial.size:
+            qs += [int(i) for i in rng.choice(partial, min(2, partial.size), replace=False)]
+        longest = max(longest, int(uses.max()))
+        need = set(qs)
+        for j in kb:
+            need |= set(np.nonzero((sel == j).any(axis=1))[0].tolist())
+        q, k, v = (blocked_to_raster(bf16_dev_to_f64(getattr(pipe, n)[:, h:h + 1]), sm)
+                   for n in ("q", "k", "v"))
+        do = bf16_bits_to_f64(x["do"][:, :, h:h + 1])
+        dq, dk, dv = oracle.attend_bwd(q, k, v, do, idx[:, h:h + 1], grid, pipe.g.scale,
+                                       query_blocks=[(0, 0, i) for i in sorted(need)])
+        got = {n: bf16_dev_to_f64(getattr(pipe, n)[:, h:h + 1]) for n in ("dq", "dk", "dv")}
+        for name, ref, blocks in (("dq", dq, qs), ("dk", dk, kb), ("dv", dv, kb)):
+            for b in blocks:
+                tile = got[name][0, 0, b]
+                pad = sm[b] < 0
+                assert np.all(tile[pad] == 0.0), f"{name}: pad rows of block {b} not zero"
+                if name != "dq" and uses[b] == 0:
+                    assert np.all(tile == 0.0), f"{name}: unselected key block {b} not zero"
+                d = np.abs(tile[~pad] - ref[0, sm[b][~pad], 0])
+                assert d.max() <= MAX_ABS, (name, h, b, d.max())
+                errs[name].append(d.reshape(-1))
+    for name, e in errs.items():
+        e = np.concatenate(e)
+        assert e.mean() <= MEAN_ABS, (name, e.mean())
+    return longest
+
+
+def test_backward_720p_sampled_blocks():
+    """The bench's 720p workload (24x45x80 tokens, 720 blocks of 4x4x8, r = 72, 32 heads x 128)
+    forward and backward in the bench's launch configuration, checked on heads 0 and 21 (8 key
+    blocks and 16 query blocks in all, see check_bwd_sampled); the dK/dV pass's long reverse
+    lists (well over 150 query blocks) are among them."""
+    w = WORKLOADS["720p"]
+    pipe, x = run_fwd_bwd(w)
+    assert check_bwd_sampled(w, pipe, x, ((0, 2), (21, 0)), seed=720) > 150
+
+
 @pytest.mark.parametrize("name", ["small", "small_b2", "small_cont", "small_cont_rope"])
 def test_backward_parity_small(name):
     w = WORKLOADS[name]
