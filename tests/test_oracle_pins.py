@@ -53,6 +53,37 @@ def test_slot_map_matches_block_members():
         assert np.array_equal(allv, np.arange(g.t_frames * g.grid_h * g.grid_w))
 
 
+def test_block_numbering_worked_by_hand():
+    """Tokens of a ragged 5 x 6 x 10 grid (t, h, w) cut into 4 x 4 x 8 blocks, worked by hand.
+
+    Blocks per axis: ceil(5/4) = 2, ceil(6/4) = 2, ceil(10/8) = 2, numbered
+    (block-t * 2 + block-h) * 2 + block-w.  Raster index of a token = (t * 6 + h) * 10 + w.
+    Slot inside a block = (local t * 4 + local h) * 8 + local w (pad positions left empty):
+      (t, h, w) = (0, 0, 0): raster 0,   block 0, local (0, 0, 0), slot 0
+      (1, 2, 3):             raster 83,  block 0, local (1, 2, 3), slot (1*4 + 2)*8 + 3 = 51
+      (2, 1, 9):             raster 139, block 1, local (2, 1, 1), slot (2*4 + 1)*8 + 1 = 73
+      (3, 4, 8):             raster 228, block 3, local (3, 0, 0), slot 96
+      (4, 0, 2):             raster 242, block 4, local (0, 0, 2), slot 2
+      (4, 5, 9):             raster 299, block 7, local (0, 1, 1), slot 9
+    Valid tokens per block (t extent * h extent * w extent; the last block along an axis keeps
+    1 frame, 2 rows or 2 columns): block 0: 4*4*8 = 128, 1: 4*4*2 = 32, 2: 4*2*8 = 64,
+    3: 4*2*2 = 16, 4: 1*4*8 = 32, 5: 1*4*2 = 8, 6: 1*2*8 = 16, 7: 1*2*2 = 4.  The block grid
+    is a 2 x 2 x 2 cube, so only the order of the axes tells these ids apart.
+    """
+    g = Grid(5, 6, 10, (4, 4, 8))
+    sm = g.slot_map(5)
+    mem = g.block_members(5)
+    for (t, h, w), (raster, blk, slot) in {(0, 0, 0): (0, 0, 0), (1, 2, 3): (83, 0, 51),
+                                           (2, 1, 9): (139, 1, 73), (3, 4, 8): (228, 3, 96),
+                                           (4, 0, 2): (242, 4, 2), (4, 5, 9): (299, 7, 9)}.items():
+        assert (t * 6 + h) * 10 + w == raster
+        assert sm[blk, slot] == raster
+        assert raster in mem[blk]
+    assert [len(m) for m in mem] == [128, 32, 64, 16, 32, 8, 16, 4]
+    assert mem[7] == [280 + 8, 280 + 9, 290 + 8, 290 + 9]  # (4,4,8) (4,4,9) (4,5,8) (4,5,9)
+    assert sorted(np.nonzero(sm[7] >= 0)[0].tolist()) == [0, 1, 8, 9]
+
+
 def test_workload_geometry_matches_pages():
     """Golden geometry: latent grid and block counts of the measured workloads."""
     import json
