@@ -10,7 +10,10 @@
 // that loads the library holds it until the process exits.  Host code cannot pass the
 // array's name to a kernel (on the host it is only a stand-in symbol), so the first call on
 // each device looks up its device address with cudaGetSymbolAddress, with that device
-// current, and caches it; make that first call before any stream capture.  All calls share
+// current, and caches it; make that first call before any stream capture.  The cache keeps
+// the CUDA context the address belongs to: after cudaDeviceReset (or any re-creation of the
+// device's primary context) the next call finds a different context and looks the address up
+// again, in the new context, rather than launching on a stale one.  All calls share
 // the array: two calls whose work overlaps on the GPU (different streams, no ordering
 // between them) race on it.  Nothing in it needs to start at zero: the pooling kernel
 // overwrites every mean it later reads.
@@ -23,8 +26,29 @@ constexpr size_t kNoallocScratchBytes = 16u << 20;
 static __device__ __align__(256) unsigned char g_route_scratch[kNoallocScratchBytes];
 
 namespace {
+constexpr int kNoallocMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[64] = {nullptr};
+void* g_noalloc_ptr[kNoallocMaxDevices] = {nullptr};
+CUcontext g_noalloc_ctx[kNoallocMaxDevices] = {nullptr};  // context each address belongs to
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+CtxGetCurrentFn g_ctx_get = nullptr;
+std::once_flag g_ctx_get_once;
+
+// The calling thread's current CUDA context (nullptr if none is bound yet or the driver entry
+// point is unavailable; a null context never matches a cached one, so it forces a lookup).
+CUcontext current_ctx() {
+  std::call_once(g_ctx_get_once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get = reinterpret_cast<CtxGetCurrentFn>(f);
+  });
+  CUcontext c = nullptr;
+  if (g_ctx_get && g_ctx_get(&c) != CUDA_SUCCESS) c = nullptr;
+  return c;
+}
 }  // namespace
 
 }  // namespace bsa
@@ -60,14 +84,19 @@ extern "C" BSA_API bsa_status_t bsa_route_noalloc(const bsa_geom_t* gi, int32_t 
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kNoallocMaxDevices)
+    return fail(BSA_ERR_UNSUPPORTED, "device %d is beyond the %d devices bsa_route_noalloc tracks",
+                dev, kNoallocMaxDevices);
   void* scratch = nullptr;
   {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    const CUcontext ctx = current_ctx();
+    if (g_noalloc_ptr[dev] == nullptr || ctx == nullptr || ctx != g_noalloc_ctx[dev]) {
       void* ptr = nullptr;
       e = cudaGetSymbolAddress(&ptr, g_route_scratch);  // this device is current
       if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(route scratch)");
       g_noalloc_ptr[dev] = ptr;
+      g_noalloc_ctx[dev] = current_ctx();  // the lookup has bound the device's context
     }
     scratch = g_noalloc_ptr[dev];
   }

@@ -10,9 +10,9 @@ from typing import Dict, Optional
 import torch
 
 from . import (POOL_MAX, POOL_SUM, ROUTE_POOL_MAX, ROUTE_POOL_SUM, WS_BWD, WS_PROLOGUE_BWD,
-               WS_ROUTE, Geometry, blocked_shape, bsa_attn_bwd, bsa_attn_fwd, bsa_block_pool,
-               bsa_cache_append, bsa_route_ex, bsa_workspace_size, rope3d_qknorm_prologue,
-               rope3d_qknorm_prologue_bwd)
+               WS_ROUTE, Geometry, Shards, blocked_shape, bsa_attn_bwd, bsa_attn_fwd,
+               bsa_block_pool, bsa_blocked_to_raster_sharded, bsa_cache_append, bsa_route_ex,
+               bsa_workspace_size, rope3d_qknorm_prologue, rope3d_qknorm_prologue_bwd)
 
 
 class BsaPipeline:
@@ -48,6 +48,8 @@ class BsaPipeline:
             self.kc = torch.empty(cshp, **bf)
             self.vc = torch.empty(cshp, **bf)
             self.kc_pool = torch.empty(cshp[:3] + (g.head_dim,), dtype=torch.float32, device=dev)
+            # the cache's keys pooled by a routing variant (sum / max), filled per route call
+            self.kc_pool_variant = torch.empty_like(self.kc_pool)
         self.gamma_q = self.gamma_k = None
         self.ws_pro_bwd = None
         if with_bwd:
@@ -105,7 +107,7 @@ class BsaPipeline:
         if pool_mode:
             use_pools = False
             if self.kc is not None:
-                kc_pool = torch.empty_like(self.kc_pool)
+                kc_pool = self.kc_pool_variant
                 bsa_block_pool(self.g, self.g.cached_t, pool_mode, self.kc, kc_pool, stream=stream)
         bsa_route_ex(self.g, self.r, flags, self.q, self.k, self.q_pool if use_pools else None,
                      self.k_pool if use_pools else None, kc_pool, self.idx, self.cnt,
@@ -120,6 +122,13 @@ class BsaPipeline:
         self.route(stream, flags=self.route_flags)
         self.attn_fwd(stream)
         return {"o": self.o, "lse": self.lse, "idx": self.idx, "cnt": self.cnt}
+
+    def o_to_raster(self, o_raster, stream=None):
+        """The blocked output O back in the raster layout [B, T*H*W, heads, D] (pad slots
+        dropped): the inverse relayout, with one shard holding every frame."""
+        g = self.g
+        bsa_blocked_to_raster_sharded(g, g.t_frames, Shards(1, g.t_frames, g.heads, 0), self.o,
+                                      [o_raster], stream=stream)
 
     def load_grad(self, do_raster, stream=None):
         """Relayout the upstream gradient dO (raster) into the blocked layout."""

@@ -70,8 +70,9 @@ typedef enum bsa_status {
   BSA_ERR_WORKSPACE = 6     /* workspace pointer NULL/misaligned or smaller than required */
 } bsa_status_t;
 
-/* Geometry of one problem.  Supported: head_dim in {64, 128}; blk_t*blk_h*blk_w in {32, 128};
- * cached_t, causal_chunk_t and cond_t multiples of blk_t. */
+/* Geometry of one problem.  Supported: head_dim in {64, 128}; blk_t*blk_h*blk_w in {32, 128}
+ * (the backward, bsa_attn_bwd, takes 128 only); cached_t, causal_chunk_t and cond_t multiples
+ * of blk_t. */
 typedef struct bsa_geom {
   int32_t batch;          /* B */
   int32_t heads;          /* H */
@@ -295,7 +296,9 @@ BSA_API bsa_status_t bsa_attn_fwd(const bsa_geom_t* g, int32_t top_r, const void
  * Delta = rowsum(dO * O):  dV_j += P^T dO,  dS = P * (dO V^T - Delta),
  * dQ_i += scale * dS K_j,  dK_j += scale * dS^T Q_i, summed over the selected pairs.
  * Gradients reach current keys/values only (cached ones are constants).  Outputs dq_blk,
- * dk_blk, dv_blk are bf16 blocked (pad slots 0); ws: BSA_WS_BWD bytes. */
+ * dk_blk, dv_blk are bf16 blocked (pad slots 0); ws: BSA_WS_BWD bytes.
+ * Block size: the backward takes 128-token blocks only (the forward also takes 32);
+ * a geometry with BS = 32 returns BSA_ERR_UNSUPPORTED before any launch. */
 BSA_API bsa_status_t bsa_attn_bwd(const bsa_geom_t* g, int32_t top_r, const void* q_blk,
                           const void* k_blk, const void* v_blk, const void* k_cache_blk,
                           const void* v_cache_blk, const void* o_blk, const float* lse,
@@ -332,8 +335,10 @@ BSA_API bsa_status_t bsa_device_status(bsa_stream_t stream);
  * k_blk); the means live in a 16 MiB array inside the library, held on every device that loads
  * it until the process exits.  Rejects geometries with B*H*NBq*D*8 > 16 MiB (after 256-byte
  * rounding of each half) with BSA_ERR_UNSUPPORTED.  Allocates nothing.  The first call on a
- * device looks up that array's device address (cudaGetSymbolAddress) and caches it: make it
- * before any stream capture.  Calls share the array, so calls that overlap on the GPU race.
+ * device looks up that array's device address (cudaGetSymbolAddress) and caches it with the
+ * current CUDA context: make it before any stream capture.  After cudaDeviceReset the next
+ * call sees a new context and looks the address up again (make that call outside a capture
+ * too).  Calls share the array, so calls that overlap on the GPU race.
  * No page counterpart: this entry point exists for callers that cannot allocate. */
 BSA_API bsa_status_t bsa_route_noalloc(const bsa_geom_t* g, int32_t top_r, const void* q_blk,
                                        const void* k_blk, const float* kpool_cache, int32_t* idx,

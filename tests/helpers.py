@@ -43,4 +43,3 @@ def bf16_ulp(x):
     """Spacing of bf16 numbers at |x| (for |x| >= 2^-126)."""
     ax = np.maximum(np.abs(x), 2.0 ** -126)
     return 2.0 ** (np.floor(np.log2(ax)) - 7)
-
