@@ -224,13 +224,15 @@ struct DkdvLayout {
   static constexpr int kNumBars = 2 + 2 * kSlots + 7 + 2 * kQueue;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kQueueOff = kMiscOff + 16;  // int [kQueue]
-  static constexpr int kAlloc = kQueueOff + kQueue * 4 + 1024;
+  static constexpr int kSlotNvOff = kQueueOff + kQueue * 4;  // int [kSlots]: valid queries
+  static constexpr int kAlloc = kSlotNvOff + kSlots * 4 + 1024;
 };
 
 template <int BS, int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bsa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
+                        const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmdO16,
                         const BwdParams p) {
   using L = DkdvLayout<BS, D>;
   constexpr int NS = L::kSlots;
@@ -254,6 +256,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* iq_empty = iq_full + L::kQueue;   // [kQueue] entry read by the MMA thread and
                                               // every elementwise thread
   volatile int* iq = reinterpret_cast<volatile int*>(smem + L::kQueueOff);
+  // valid queries of the Q / dO tiles in each slot (written by the producer before the slot's
+  // q_full arrival, read by the MMA thread after waiting on it)
+  volatile int* slot_nv = reinterpret_cast<volatile int*>(smem + L::kSlotNvOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
@@ -356,13 +361,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int qrow = (bh * g.NBq + i) * BS;
           if (round > 0 && !mbar_wait(&q_empty[slot], (round - 1) & 1, abort_flag)) { ok = false; break; }
           unsigned char* vec = smem + L::kVecOff + slot * L::kVecBytes;
-          mbar_expect_tx(&q_full[slot], 2 * L::kTileBytes + L::kVecBytes);
+          const int nv = query_block_nvalid(g, i);
+          slot_nv[slot] = nv;
+          // only the rows the tensor cores read: a partial query block's valid prefix rounded
+          // up to 16, in 16-row boxes (a full block in one box per half)
+          const int nrows = nv >= BS ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
+          mbar_expect_tx(&q_full[slot], 2u * (uint32_t)nrows * 128u * (D / 64) + L::kVecBytes);
+          unsigned char* dq_ = smem + L::kQOff + slot * L::kTileBytes;
+          unsigned char* ddo = smem + L::kDOOff + slot * L::kTileBytes;
+          if (nrows == BS) {
 #pragma unroll
-          for (int half = 0; half < D / 64; ++half) {
-            tma_load_2d(smem + L::kQOff + slot * L::kTileBytes + half * BS * 128, &tmQ, half * 64,
-                        qrow, &q_full[slot]);
-            tma_load_2d(smem + L::kDOOff + slot * L::kTileBytes + half * BS * 128, &tmdO, half * 64,
-                        qrow, &q_full[slot]);
+            for (int half = 0; half < D / 64; ++half) {
+              tma_load_2d(dq_ + half * BS * 128, &tmQ, half * 64, qrow, &q_full[slot]);
+              tma_load_2d(ddo + half * BS * 128, &tmdO, half * 64, qrow, &q_full[slot]);
+            }
+          } else {
+            for (int r0 = 0; r0 < nrows; r0 += 16)
+#pragma unroll
+              for (int half = 0; half < D / 64; ++half) {
+                tma_load_2d(dq_ + half * BS * 128 + r0 * 128, &tmQ16, half * 64, qrow + r0, &q_full[slot]);
+                tma_load_2d(ddo + half * BS * 128 + r0 * 128, &tmdO16, half * 64, qrow + r0, &q_full[slot]);
+              }
           }
           bulk_load(vec, p.nlse2 + (size_t)qrow, BS * 4, &q_full[slot]);
           bulk_load(vec + BS * 4, p.ndelta + (size_t)qrow, BS * 4, &q_full[slot]);
@@ -379,8 +398,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdMma) {
     // ====================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idSS = idesc_bf16(kTile, BS, 0, 0);   // S^T, dP^T: both K-major
       constexpr uint32_t idTS = idesc_bf16(kTile, D, 0, 1);    // dV, dK: B MN-major
+      // queries of step g on the tensor cores: the query block's valid prefix rounded up to
+      // 16 (the MMA's N step), so a partial block's S^T, dP^T (N) and dV, dK (K) shrink with
+      // it; read from the slot when S^T(g) is issued and kept for the step's other MMAs
+      int nq_even = BS, nq_odd = BS;  // for steps g with g & 1 == 0 / 1
+      auto nq_step = [&](int gg) -> int { return (gg & 1) ? nq_odd : nq_even; };
       const uint64_t dK0 = smem_desc_sw128(smem_u32(smem + L::kKOff), 16, 1024);
       const uint64_t dV0 = smem_desc_sw128(smem_u32(smem + L::kVOff), 16, 1024);
       const uint64_t dQk = smem_desc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
@@ -399,6 +422,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         if (!mbar_wait(&q_full[gg & 1], (gg >> 1) & 1, abort_flag)) return false;
         tc_fence_after();
+        {
+          const int nv = slot_nv[gg & 1];
+          const int nq = nv >= BS ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
+          if (gg & 1) nq_odd = nq;
+          else nq_even = nq;
+        }
+        const uint32_t idSS = idesc_bf16(kTile, nq_step(gg), 0, 0);  // both K-major
         const uint64_t rq = dQk + (uint64_t)(((gg & 1) * L::kTileBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -412,6 +442,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       // slot); after an item's last one K_j, V_j are free
       auto issue_dP = [&](int gg, bool item_last) -> bool {
         const uint64_t rdo = dOk + (uint64_t)(((gg & 1) * L::kTileBytes) >> 4);
+        const uint32_t idSS = idesc_bf16(kTile, nq_step(gg), 0, 0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
@@ -427,10 +458,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t r = tmem_base + (gg & 1) * 128 + (is_dk ? 16 : 0);
         const uint64_t mb = (is_dk ? dQmn : dOmn) + (uint64_t)(((gg & 1) * L::kTileBytes) >> 4);
         const uint32_t acc_d = is_dk ? t_dk : t_dv;
+        const int nk = nq_step(gg) / 16;
 #pragma unroll
         for (int kk = 0; kk < BS / 16; ++kk)
-          mma_ts(acc_d, r + 32 * (kk >> 1) + 8 * (kk & 1), mb + (uint64_t)((kk * 2048) >> 4), idTS,
-                 (item_first && kk == 0) ? 0u : 1u);
+          if (kk < nk)
+            mma_ts(acc_d, r + 32 * (kk >> 1) + 8 * (kk & 1), mb + (uint64_t)((kk * 2048) >> 4),
+                   idTS, (item_first && kk == 0) ? 0u : 1u);
       };
       // Per step g: dV(g) | S^T(g+1) (into the region dP^T(g) left) | dK(g) | dP^T(g+1) (into
       // the region dV(g), dK(g) just read).  The elementwise warps form P^T(g+1) while the
@@ -495,11 +528,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int beg, end;
       item_range(item, beg, end);
       const int jc = item % g.NBq;
-      int vt, vh, vw;
-      block_extent(g, g.T, jc, vt, vh, vw);
-      const int lt = row / (g.bh * g.bw), lh = (row / g.bw) % g.bh, lw = row % g.bw;
-      const bool kvalid = lt < vt && lh < vh && lw < vw;
+      const bool kvalid = row < query_block_nvalid(g, jc);  // key slot in the valid prefix
       for (int e = beg; e < end; ++e, ++gs) {
+        // valid queries of this step's query block, from its slot (the slot's q_full phase
+        // for this step has completed: S^T(g) was issued after it), so a group whose 32 query
+        // columns all lie past a partial block's valid prefix can skip the step: the tensor
+        // cores compute and read only the first roundup16(valid) columns
+        {
+          bool w_ok = mbar_wait(&q_full[gs % NS], (gs / NS) & 1, abort_flag);
+          w_ok = __all_sync(0xffffffffu, w_ok);
+          if (!w_ok) { ok = false; break; }
+        }
+        if (cg * 32 >= slot_nv[gs % NS]) {
+          // nothing to form: keep the waits and arrivals in order
+          bool w_ok = mbar_wait(s_full, gs & 1, abort_flag);
+          w_ok = __all_sync(0xffffffffu, w_ok);
+          if (!w_ok) { ok = false; break; }
+          mbar_arrive(p_ready);
+          w_ok = mbar_wait(dp_full, gs & 1, abort_flag);
+          w_ok = __all_sync(0xffffffffu, w_ok);
+          if (!w_ok) { ok = false; break; }
+          mbar_arrive(dp_loaded);
+          mbar_arrive(ds_ready);
+          continue;
+        }
         // this group's 32 query columns of step g: P^T = exp2(S^T*sl2 - lse2[q]) as soon as
         // S^T is in, then dS^T = P^T * (dP^T - delta[q]) once dP^T is; both in bf16 back over
         // the group's own S^T columns as [P^T 16 cols | dS^T 16 cols]
@@ -631,8 +683,8 @@ struct DqLayout {
   // q_full, q_empty, kv_full[5], kv_empty[5], s_full, s_loaded, dp_full, ds_full, dq_full, fin
   static constexpr int kNumBars = 2 + 2 * kStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kMaskOff = kMiscOff + 16;  // u32 [12 shapes][BS / 32]
-  static constexpr int kAlloc = kMaskOff + 12 * (BS / 32) * 4 + 1024;
+  static constexpr int kStageNvOff = kMiscOff + 16;  // int [stages]: valid keys of the tile
+  static constexpr int kAlloc = kStageNvOff + kStages * 4 + 1024;
 };
 
 template <int BS, int D>
@@ -640,6 +692,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bsa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
+                      const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmV16,
+                      const __grid_constant__ CUtensorMap tmKc16, const __grid_constant__ CUtensorMap tmVc16,
                       const BwdParams p) {
   using L = DqLayout<BS, D>;
   constexpr int S = L::kStages;
@@ -661,6 +715,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* fin_bar = dq_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+  // valid keys of the K / V tile in each ring stage (written by the producer before the tile's
+  // kv_full arrival, read by the MMA thread after waiting on it)
+  volatile int* stage_nv = reinterpret_cast<volatile int*>(smem + L::kStageNvOff);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const Geo& g = p.g;
 
@@ -678,7 +735,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     mbar_fence_init();
   }
   if (warp == kBwdMma) { tmem_alloc(tmem_holder, 512); tmem_relinquish(); }
-  if (tid < 12) fill_shape_mask<BS>(g, tid, reinterpret_cast<uint32_t*>(smem + L::kMaskOff));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -715,18 +771,36 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int bhx = item / g.NBq;
         for (int n = 0; n < cnt && ok; ++n) {
           const int j = item_idx(item, n);
-          const CUtensorMap *mk, *mv;
+          const CUtensorMap *mk, *mv, *mk16, *mv16;
           int row;
-          if (j < g.NBc) { mk = &tmKc; mv = &tmVc; row = (bhx * g.NBc + j) * BS; }
-          else { mk = &tmK; mv = &tmV; row = (bhx * g.NBq + (j - g.NBc)) * BS; }
+          if (j < g.NBc) {
+            mk = &tmKc; mv = &tmVc; mk16 = &tmKc16; mv16 = &tmVc16;
+            row = (bhx * g.NBc + j) * BS;
+          } else {
+            mk = &tmK; mv = &tmV; mk16 = &tmK16; mv16 = &tmV16;
+            row = (bhx * g.NBq + (j - g.NBc)) * BS;
+          }
+          const int nv = key_block_nvalid(g, j);
+          // only the rows the tensor cores read: a partial block's valid prefix rounded up to
+          // 16, in 16-row boxes (a full block in one box per half)
+          const int nrows = nv >= BS ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
           for (int t = 0; t < 2; ++t) {  // K_n then V_n
             const int stage = seq % S, round = seq / S;
             if (round > 0 && !mbar_wait(&kv_empty[stage], (round - 1) & 1, abort_flag)) { ok = false; break; }
             unsigned char* dst = smem + L::kRingOff + stage * L::kKVBytes;
-            mbar_expect_tx(&kv_full[stage], L::kKVBytes);
+            stage_nv[stage] = nv;
+            mbar_expect_tx(&kv_full[stage], (uint32_t)nrows * 128u * (D / 64));
+            if (nrows == BS) {
 #pragma unroll
-            for (int half = 0; half < D / 64; ++half)
-              tma_load_2d(dst + half * BS * 128, t == 0 ? mk : mv, half * 64, row, &kv_full[stage]);
+              for (int half = 0; half < D / 64; ++half)
+                tma_load_2d(dst + half * BS * 128, t == 0 ? mk : mv, half * 64, row, &kv_full[stage]);
+            } else {
+              for (int r0 = 0; r0 < nrows; r0 += 16)
+#pragma unroll
+                for (int half = 0; half < D / 64; ++half)
+                  tma_load_2d(dst + half * BS * 128 + r0 * 128, t == 0 ? mk16 : mv16, half * 64,
+                              row + r0, &kv_full[stage]);
+            }
             ++seq;
           }
         }
@@ -740,8 +814,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdMma) {
     // ====================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(kTile, BS, 0, 0);   // S, dP: B (K or V tile) K-major
       constexpr uint32_t idQ = idesc_bf16(kTile, D, 0, 1);    // dQ: B (K tile) MN-major
+      // keys of a tile on the tensor cores: the block's valid prefix rounded up to 16 (the
+      // MMA's N step), so a partial block's S, dP (N) and dQ (K) shrink with it
+      auto tile_keys = [&](int seq) -> int {
+        const int nv = stage_nv[seq % S];
+        return nv >= BS ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
+      };
       const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
       const uint64_t dkmn = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
       int items = 0, gn = 0;  // non-empty items, global step
@@ -753,7 +832,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         return true;
       };
-      auto mma_S = [&](int n) {  // S(n) = Q K_n^T (A = Q from TMEM)
+      // S(n) = Q K_n^T (A = Q from TMEM); idS carries the step's key count (read right after
+      // the K tile's wait, so the shared-memory load stays off the issue path)
+      auto mma_S = [&](int n, uint32_t idS) {
         const uint64_t kb = dk + (uint64_t)((((seq_base + 2 * n) % S) * L::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -762,7 +843,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_commit(s_full);
       };
-      auto mma_dP = [&](int n) {  // dP(n) = dO V_n^T (A = dO from TMEM); then V_n is done
+      auto mma_dP = [&](int n, uint32_t idS) {  // dP(n) = dO V_n^T (A = dO from TMEM); then V_n is done
         const int seq = seq_base + 2 * n + 1;
         const uint64_t vb = dk + (uint64_t)(((seq % S) * L::kKVBytes) >> 4);
 #pragma unroll
@@ -785,15 +866,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (gn > 0 && !mbar_wait(s_loaded, (gn - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (!wait_tile(seq_base) || !wait_tile(seq_base + 1)) { ok = false; break; }
-        mma_S(0);
-        mma_dP(0);
+        int nkeys = tile_keys(seq_base);  // keys of step n on the tensor cores (K_n, V_n alike)
+        {
+          const uint32_t id0 = idesc_bf16(kTile, nkeys, 0, 0);
+          mma_S(0, id0);
+          mma_dP(0, id0);
+        }
         for (int n = 0; n < cnt && ok; ++n, ++gn) {
           const bool more = n + 1 < cnt;
+          int nkeys_next = BS;
+          uint32_t id_next = 0;
           if (more) {  // S(n+1) once S(n) was read out
             if (!mbar_wait(s_loaded, gn & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             if (!wait_tile(seq_base + 2 * (n + 1))) { ok = false; break; }
-            mma_S(n + 1);
+            nkeys_next = tile_keys(seq_base + 2 * (n + 1));
+            id_next = idesc_bf16(kTile, nkeys_next, 0, 0);
+            mma_S(n + 1, id_next);
             if (!wait_tile(seq_base + 2 * (n + 1) + 1)) { ok = false; break; }  // V_{n+1}, early
           }
           // dQ += dS(n) K_n (A = dS over the dP columns), then dP(n+1) into those columns
@@ -801,12 +890,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
           const int kseq = seq_base + 2 * n;
           const uint64_t kb = dkmn + (uint64_t)(((kseq % S) * L::kKVBytes) >> 4);
+          const int nk = nkeys / 16;
 #pragma unroll
           for (int kk = 0; kk < BS / 16; ++kk)  // dS of keys [16kk, 16kk+16): group kk/2's columns
-            mma_ts(tmem_base + kTdq, tmem_base + kTdp + 32 * (kk >> 1) + 8 * (kk & 1),
-                   kb + (uint64_t)((kk * 2048) >> 4), idQ, (n > 0 || kk > 0) ? 1u : 0u);
+            if (kk < nk)
+              mma_ts(tmem_base + kTdq, tmem_base + kTdp + 32 * (kk >> 1) + 8 * (kk & 1),
+                     kb + (uint64_t)((kk * 2048) >> 4), idQ, (n > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&kv_empty[kseq % S]);  // K_n done
-          if (more) mma_dP(n + 1);
+          if (more) mma_dP(n + 1, id_next);
+          nkeys = nkeys_next;
         }
         if (!ok) break;
         mma_commit(dq_full);
@@ -869,16 +961,32 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float nd = row < BS ? p.ndelta[qrow] : 0.f;
       const uint64_t nl2x2 = f2pack(nl2, nl2), ndx2 = f2pack(nd, nd), sl2x2 = f2pack(sl2, sl2);
       // key-block indices 32 steps at a time, the next chunk's load in flight; per chunk a
-      // ballot of the partial blocks and each lane's shape code (as in the forward)
+      // ballot of the partial blocks and each lane's valid-key count (as in the forward)
       int jnext = lane < cnt ? item_idx(item, lane) : 0;
-      int creg = 0;
+      int nreg = BS;
       uint32_t partial = 0;
       for (int n = 0; n < cnt; ++n, ++gn) {
         if ((n & 31) == 0) {
           const int jcur = jnext;
           jnext = n + 32 + lane < cnt ? item_idx(item, n + 32 + lane) : 0;
-          creg = n + lane < cnt ? key_shape_code(g, jcur) : 0;
-          partial = __ballot_sync(0xffffffffu, creg != 0);
+          nreg = n + lane < cnt ? key_block_nvalid(g, jcur) : BS;
+          partial = __ballot_sync(0xffffffffu, nreg < BS);
+        }
+        // A group whose keys all lie past a partial block's valid prefix has nothing to do in
+        // this step (the tensor cores compute only the first roundup16(valid) keys and read
+        // dS of those only); it keeps the waits and arrivals, in order, so no barrier phase
+        // can be overrun.
+        const int nvb = ((partial >> (n & 31)) & 1u) ? __shfl_sync(0xffffffffu, nreg, n & 31) : BS;
+        if (cg * KC >= nvb) {
+          bool w_ok = mbar_wait(s_full, gn & 1, abort_flag);
+          w_ok = __all_sync(0xffffffffu, w_ok);
+          if (!w_ok) { ok = false; break; }
+          mbar_arrive(s_loaded);
+          w_ok = mbar_wait(dp_full, gn & 1, abort_flag);
+          w_ok = __all_sync(0xffffffffu, w_ok);
+          if (!w_ok) { ok = false; break; }
+          mbar_arrive(ds_full);
+          continue;
         }
         // P = exp2(S*sl2 - lse2) for this group's KC keys as soon as S(n) is in
         bool w_ok = mbar_wait(s_full, gn & 1, abort_flag);
@@ -889,12 +997,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32_wait(t_s + cg * KC, reinterpret_cast<uint32_t*>(pf));
         tc_fence_before();
         mbar_arrive(s_loaded);  // S may take S(n+1)
-        if ((partial >> (n & 31)) & 1u) {  // pad keys of a partial key block: P = 0
-          const int code = __shfl_sync(0xffffffffu, creg, n & 31);
-          const uint32_t word = reinterpret_cast<const uint32_t*>(smem + L::kMaskOff)[code * (BS / 32) + cg];
+        if (nvb < BS) {  // pad keys (slots >= the valid count): P = 0
+          const int nv = nvb - cg * KC;
 #pragma unroll
           for (int c = 0; c < KC; ++c)
-            if (!((word >> c) & 1u)) pf[c] = -INFINITY;
+            if (c >= nv) pf[c] = -INFINITY;
         }
 #pragma unroll
         for (int e2 = 0; e2 < KC / 2; ++e2) {
@@ -960,7 +1067,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ------------------------------------------------------------------------------ host side
-// maps: 0 Q (box 128 rows), 1 K, 2 V, 3 K cache, 4 V cache (box BS rows), 5 dO (box 128 rows)
+// maps: 0 Q (box 128 rows), 1 K, 2 V, 3 K cache, 4 V cache (box BS rows), 5 dO (box 128 rows);
+// 6-9 K, V, K cache, V cache and 10-11 Q, dO with 16-row boxes
 bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, const CUtensorMap* maps,
                      int n_sm, cudaStream_t s) {
   if (g.BS != 128) return BSA_ERR_UNSUPPORTED;  // the key-major pass needs 128-token blocks
@@ -1014,7 +1122,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
       return BSA_ERR_CUDA;                                                                        \
     cudaEvent_t e1;                                                                               \
     const int w1 = timed_begin(BSA_TIMED_BWD_DKDV, s, &e1);                                       \
-    k1<<<grid, kBwdThreads, s1, s>>>(maps[1], maps[2], maps[0], maps[5], a);                      \
+    k1<<<grid, kBwdThreads, s1, s>>>(maps[1], maps[2], maps[0], maps[5], maps[10], maps[11], a);  \
     timed_end(w1, s, e1);                                                                         \
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;                                   \
     BwdParams c = bp;                                                                             \
@@ -1026,7 +1134,8 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
       return BSA_ERR_CUDA;                                                                        \
     cudaEvent_t e2;                                                                               \
     const int w2 = timed_begin(BSA_TIMED_BWD_DQ, s, &e2);                                         \
-    k2<<<grid, kBwdThreads, s2, s>>>(maps[0], maps[5], maps[1], maps[2], maps[3], maps[4], c);   \
+    k2<<<grid, kBwdThreads, s2, s>>>(maps[0], maps[5], maps[1], maps[2], maps[3], maps[4],      \
+                                     maps[6], maps[7], maps[8], maps[9], c);                     \
     timed_end(w2, s, e2);                                                                         \
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;                                   \
   } while (0)

@@ -23,7 +23,7 @@ struct Geo {
   int T, GH, GW;        // current frames and valid grid
   int Tc;               // cached frames
   int bt, bh, bw, BS;   // block shape (powers of two: BS is 32 or 128)
-  int lbh, lbw;         // log2(bh), log2(bw): slot (lt, lh, lw) = (s >> (lbh+lbw), (s >> lbw) & (bh-1), s & (bw-1))
+  int lbh, lbw;         // log2(bh), log2(bw): slot of a full block (lt, lh, lw) = (s >> (lbh+lbw), (s >> lbw) & (bh-1), s & (bw-1))
   int nbh, nbw;         // blocks along h and w
   int nbt_q, nbt_c;     // blocks along t for current / cached frames
   int NBq, NBc, NBk;    // query blocks, cached key blocks, all key blocks
@@ -41,6 +41,39 @@ __host__ __device__ inline void block_extent(const Geo& g, int frames, int blk, 
   vt = min(g.bt, frames - ibt * g.bt);
   vh = min(g.bh, g.GH - ibh * g.bh);
   vw = min(g.bw, g.GW - ibw * g.bw);
+}
+
+// Slot order inside a block: the block's valid tokens first, numbered row-major over its
+// valid extents (vt, vh, vw) -- slot = (lt * vh + lh) * vw + lw -- then its pad slots
+// (slot >= vt * vh * vw).  A full block is plain (lt, lh, lw) row-major over (bt, bh, bw).
+// With the valid tokens a prefix, a partial block's tiles can shrink to its valid count.
+// `full` (vh == bh and vw == bw) takes the shift-only decode.
+__host__ __device__ __forceinline__ void slot_local(const Geo& g, int s, int vh, int vw, bool full,
+                                                    int& lt, int& lh, int& lw) {
+  if (full) {
+    lt = s >> (g.lbh + g.lbw);
+    lh = (s >> g.lbw) & (g.bh - 1);
+    lw = s & (g.bw - 1);
+  } else {
+    const int hw = vh * vw;
+    lt = s / hw;
+    const int r = s - lt * hw;
+    lh = r / vw;
+    lw = r - lh * vw;
+  }
+}
+
+// Valid tokens of query block i (current frames) and of global key block j (cached first).
+__host__ __device__ inline int query_block_nvalid(const Geo& g, int i) {
+  int vt, vh, vw;
+  block_extent(g, g.T, i, vt, vh, vw);
+  return vt * vh * vw;
+}
+__host__ __device__ inline int key_block_nvalid(const Geo& g, int j) {
+  int vt, vh, vw;
+  if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
+  else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
+  return vt * vh * vw;
 }
 
 // First absolute frame of global key block j / query block i.
@@ -182,48 +215,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float d;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
-}
-
-// Valid-key mask of a block with valid extents (vt, vh, vw) out of (bt, bh, bw): bit c of
-// the BS-bit mask is set iff slot c = (lt*bh + lh)*bw + lw is a real token.  Division-free.
-template <int BS>
-__device__ __forceinline__ void block_valid_mask(const Geo& g, int vt, int vh, int vw,
-                                                 uint32_t (&m)[BS / 32]) {
-#pragma unroll
-  for (int w = 0; w < BS / 32; ++w) m[w] = 0u;
-  for (int lt = 0; lt < vt; ++lt)
-    for (int lh = 0; lh < vh; ++lh) {
-      const int pos = (lt * g.bh + lh) * g.bw;  // bw divides 32 or is a multiple of 32
-      for (int x = 0; x < vw; x += 32) {
-        const int p = pos + x;
-        const uint32_t bits = (vw - x) >= 32 ? 0xFFFFFFFFu : ((1u << (vw - x)) - 1u);
-#pragma unroll
-        for (int w = 0; w < BS / 32; ++w)
-          if ((p >> 5) == w) m[w] |= bits << (p & 31);
-      }
-    }
-}
-
-// Shape code of key block j: (t class * 2 + h partial) * 2 + w partial, where t class is 0
-// for a full t extent, 1 for the last (partial) t-block of the cache grid, 2 for the last
-// (partial) t-block of the current grid.  Code 0 = full block.
-__device__ __forceinline__ int key_shape_code(const Geo& g, int j) {
-  int vt, vh, vw;
-  if (j < g.NBc) block_extent(g, g.Tc, j, vt, vh, vw);
-  else block_extent(g, g.T, j - g.NBc, vt, vh, vw);
-  const int tcls = vt < g.bt ? (j < g.NBc ? 1 : 2) : 0;
-  return (tcls * 2 + (vh < g.bh ? 1 : 0)) * 2 + (vw < g.bw ? 1 : 0);
-}
-// Valid-slot mask of shape code `code` (see key_shape_code) into tab[code * BS/32 ..].
-template <int BS>
-__device__ __forceinline__ void fill_shape_mask(const Geo& g, int code, uint32_t* tab) {
-  const int tcls = code >> 2, hp = (code >> 1) & 1, wp = code & 1;
-  const int rt = tcls == 1 ? g.Tc % g.bt : g.T % g.bt, rh = g.GH % g.bh, rw = g.GW % g.bw;
-  const int vt = tcls == 0 ? g.bt : rt, vh = hp ? rh : g.bh, vw = wp ? rw : g.bw;
-  uint32_t mw[BS / 32];
-  block_valid_mask<BS>(g, vt, vh, vw, mw);
-#pragma unroll
-  for (int w2 = 0; w2 < BS / 32; ++w2) tab[code * (BS / 32) + w2] = mw[w2];
 }
 
 // ------------------------------------------------------------------ TMA

@@ -5,7 +5,8 @@
 // pairing, the norm placement (before RoPE) and eps are this library's documented readings.
 //
 // HBM-bound: every (token, head) row of q, k, v is read once (D bf16) and written once to
-// its slot of the blocked layout; pad slots are written as zeros.  One CTA handles one
+// its slot of the blocked layout (a block's valid tokens first, see slot_local); pad slots
+// are written as zeros.  One CTA handles one
 // block of the padded grid for 8 heads; D/8 lanes own one row (16-byte vectors).  Rows are
 // visited slot-major, head-minor, so consecutive row groups read consecutive heads of one
 // token (a contiguous 8 x D x 2-byte run of the raster) and every lane keeps one head.
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
   int vt, vh, vw;
   block_extent(g, a.frames, blk, vt, vh, vw);
   const int nvalid = max(vt, 0) * max(vh, 0) * max(vw, 0);
+  const bool full = vh == g.bh && vw == g.bw;  // slot decode by shifts
   const bool rope = a.theta > 0.f;
 
   // ---- cos/sin table: axis t rows [0,bt), h rows [bt, bt+bh), w rows after; each row
@@ -149,9 +151,10 @@ __global__ void __launch_bounds__(kPrologueThreads)
     auto fetch = [&](int bs) -> uint4 {
       const int row = bs + rid;
       const int hl = row % hpc, slot = row / hpc;
-      const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
       uint4 r = make_uint4(0u, 0u, 0u, 0u);
-      if (row < rows && hl < heads_here && lt < vt && lh < vh && lw < vw) {
+      if (row < rows && hl < heads_here && slot < nvalid) {
+        int lt, lh, lw;
+        slot_local(g, slot, vh, vw, full, lt, lh, lw);
         const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
         int sidx;
         const size_t off = shard_elem<kSharded, D>(a.sh, g, n_raster, b, t, hh, ww,
@@ -168,8 +171,9 @@ __global__ void __launch_bounds__(kPrologueThreads)
       const int hl = row % hpc, slot = row / hpc;
       const bool in = row < rows && hl < heads_here;
       const int h = hg * kHeadsPerCta + hl;
-      const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
-      const bool valid = in && lt < vt && lh < vh && lw < vw;
+      const bool valid = in && slot < nvalid;
+      int lt = 0, lh = 0, lw = 0;
+      if (valid) slot_local(g, slot, vh, vw, full, lt, lh, lw);
       float v[8];
       {
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
@@ -303,6 +307,8 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const int ibt = blk / per_t, ibh = (blk % per_t) / g.nbw, ibw = blk % g.nbw;
   int vt, vh, vw;
   block_extent(g, f.frames, blk, vt, vh, vw);
+  const int nvalid = max(vt, 0) * max(vh, 0) * max(vw, 0);
+  const bool full = vh == g.bh && vw == g.bw;  // slot decode by shifts
   const bool rope = f.theta > 0.f;
   const int pt = f.dt / 2, ph = f.dh / 2;
   const int off_h = g.bt * pt, off_w = off_h + g.bh * ph;
@@ -339,8 +345,9 @@ __global__ void __launch_bounds__(kPrologueThreads)
       const int row = base + rid;
       const int hl = row % hpc, slot = row / hpc;
       const int h = hg * kHeadsPerCta + hl;
-      const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
-      const bool valid = row < rows && hl < heads_here && lt < vt && lh < vh && lw < vw;
+      const bool valid = row < rows && hl < heads_here && slot < nvalid;
+      int lt = 0, lh = 0, lw = 0;
+      if (valid) slot_local(g, slot, vh, vw, full, lt, lh, lw);
       float v[8], xv[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) { v[e] = 0.f; xv[e] = 0.f; }

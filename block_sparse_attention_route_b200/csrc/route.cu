@@ -40,9 +40,9 @@ __global__ void __launch_bounds__(kPoolThreads)
   float acc[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) acc[e] = kInit;
-  for (int slot = rg; slot < g.BS; slot += RG) {
-    const int lt = slot >> (g.lbh + g.lbw), lh = (slot >> g.lbw) & (g.bh - 1), lw = slot & (g.bw - 1);
-    if (lt < vt && lh < vh && lw < vw) {
+  const int nvalid = max(vt, 0) * max(vh, 0) * max(vw, 0);
+  for (int slot = rg; slot < nvalid; slot += RG) {  // valid tokens are the first slots
+    {
       const uint4 raw = __ldg(reinterpret_cast<const uint4*>(base + (size_t)slot * D + cc * 8));
       const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
@@ -59,7 +59,6 @@ __global__ void __launch_bounds__(kPoolThreads)
 #pragma unroll
   for (int e = 0; e < 8; ++e) red[rg][cc * 8 + e] = acc[e];
   __syncthreads();
-  const int nvalid = max(vt, 0) * max(vh, 0) * max(vw, 0);
   for (int d = tid; d < D; d += kPoolThreads) {
     float s = kInit;
     for (int r = 0; r < RG; ++r) s = MODE == kPoolMax ? fmaxf(s, red[r][d]) : s + red[r][d];

@@ -20,9 +20,14 @@
  * LAYOUTS (all tensors contiguous, row-major, device memory unless stated)
  *   raster  : bf16 [B, N, H, D], N = frames * grid_h * grid_w tokens ordered (t, h, w).
  *   blocked : bf16 [B, H, NB, BS, D].  The grid is padded up to whole blocks; blocks are
- *             numbered (block-t, block-h, block-w) row-major; the BS = blk_t*blk_h*blk_w
- *             slots of a block are ordered (local t, local h, local w) row-major.  Pad
- *             slots hold zeros (written by the prologue, written as zeros in O/dQ/dK/dV).
+ *             numbered (block-t, block-h, block-w) row-major.  Of the BS = blk_t*blk_h*blk_w
+ *             slots of a block with valid extents (vt, vh, vw) (the last block along an
+ *             axis may hold fewer frames, rows or columns than the block shape), the first
+ *             n = vt*vh*vw hold its tokens, row-major over those extents: slot
+ *             (local t * vh + local h) * vw + local w.  A full block is therefore plain
+ *             (local t, local h, local w) row-major.  Pad slots (>= n) follow and hold zeros
+ *             (written by the prologue, written as zeros in O/dQ/dK/dV).  The valid prefix
+ *             lets the attention kernels shrink a partial block's tiles.
  *   pooled  : fp32 [B, H, NB, D], mean over the valid (non-pad) tokens of each block.
  *   idx     : int32 [B, H, NBq, top_r], selected global key-block ids in ascending order,
  *             -1 after the first cnt entries.  cnt: int32 [B, H, NBq].

@@ -143,17 +143,25 @@ class Grid:
     def slot_map(self, frames: int) -> np.ndarray:
         """[NB, BS] raster index held by each slot of the padded block layout (-1 = pad).
 
-        Slot order inside a block is (local t, local h, local w) row-major; this is the
-        blocked memory layout the CUDA library writes, restated here independently.
+        A block whose valid extents are (vt, vh, vw) (the last block along an axis may hold
+        fewer frames, rows or columns than the block shape) keeps its tokens in its first
+        vt*vh*vw slots, row-major over those extents: slot = (lt*vh + lh)*vw + lw with (lt,
+        lh, lw) the token's position inside the block; pad slots follow.  A full block is
+        plain (lt, lh, lw) row-major.  This is the blocked memory layout the CUDA library
+        writes (the pages fix no layout), restated here independently.
         """
         bt, bh, bw = self.blk
         nbt = -(-frames // bt)
         out = -np.ones((nbt * self.nbh * self.nbw, self.bs), dtype=np.int64)
         for t in range(frames):
+            vt = min(bt, frames - (t // bt) * bt)
             for h in range(self.grid_h):
+                vh = min(bh, self.grid_h - (h // bh) * bh)
                 for w in range(self.grid_w):
+                    vw = min(bw, self.grid_w - (w // bw) * bw)
                     b = ((t // bt) * self.nbh + h // bh) * self.nbw + w // bw
-                    s = ((t % bt) * bh + h % bh) * bw + w % bw
+                    s = ((t % bt) * vh + h % bh) * vw + w % bw
+                    assert s < vt * vh * vw
                     out[b, s] = (t * self.grid_h + h) * self.grid_w + w
         return out
 

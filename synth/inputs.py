@@ -90,6 +90,10 @@ WORKLOADS: Dict[str, Workload] = {
                                 cached_t=4, chunk_t=8),
     "tiny_d128": Workload("tiny_d128", 1, 2, 128, 4, 8, 8, (2, 4, 4), 3),
     "tiny_ragged": Workload("tiny_ragged", 1, 2, 64, 3, 7, 6, (2, 4, 4), 2),
+    # every class of valid count a partial 128-token block can have: 5x9x11 gives blocks of
+    # 128, 48, 32, 12, 8 and 3 tokens; 7x11x13 gives 128, 96, 80, 72, 60 and 45
+    "ragged_a": Workload("ragged_a", 1, 2, 128, 5, 9, 11, (4, 4, 8), 4),
+    "ragged_b": Workload("ragged_b", 1, 2, 128, 7, 11, 13, (4, 4, 8), 5),
 }
 
 

@@ -129,7 +129,8 @@ def test_backward_720p_sampled_blocks():
     assert check_bwd_sampled(w, pipe, x, ((0, 2), (21, 0)), seed=720) > 150
 
 
-@pytest.mark.parametrize("name", ["small", "small_b2", "small_cont", "small_cont_rope"])
+@pytest.mark.parametrize("name", ["small", "small_b2", "small_cont", "small_cont_rope", "ragged_a",
+                                  "ragged_b"])
 def test_backward_parity_small(name):
     w = WORKLOADS[name]
     pipe, x = run_fwd_bwd(w)

@@ -150,7 +150,8 @@ def check_attention(w, pipe, heads, qblocks=None):
     return float(e.max()), float(e.mean())
 
 
-SMALL = ["tiny", "tiny_ragged", "tiny_d128", "small", "small_b2", "small_cont", "small_cont_rope"]
+SMALL = ["tiny", "tiny_ragged", "tiny_d128", "small", "small_b2", "small_cont", "small_cont_rope",
+         "ragged_a", "ragged_b"]
 
 
 @pytest.mark.parametrize("name", SMALL)

@@ -58,30 +58,33 @@ def test_block_numbering_worked_by_hand():
 
     Blocks per axis: ceil(5/4) = 2, ceil(6/4) = 2, ceil(10/8) = 2, numbered
     (block-t * 2 + block-h) * 2 + block-w.  Raster index of a token = (t * 6 + h) * 10 + w.
-    Slot inside a block = (local t * 4 + local h) * 8 + local w (pad positions left empty):
+    Valid extents (vt, vh, vw) per block (the last block along an axis keeps 1 frame, 2 rows
+    or 2 columns) and valid tokens: block 0 (4,4,8) 128, 1 (4,4,2) 32, 2 (4,2,8) 64,
+    3 (4,2,2) 16, 4 (1,4,8) 32, 5 (1,4,2) 8, 6 (1,2,8) 16, 7 (1,2,2) 4.
+    Slot inside a block = (local t * vh + local h) * vw + local w (pad slots after them):
       (t, h, w) = (0, 0, 0): raster 0,   block 0, local (0, 0, 0), slot 0
       (1, 2, 3):             raster 83,  block 0, local (1, 2, 3), slot (1*4 + 2)*8 + 3 = 51
-      (2, 1, 9):             raster 139, block 1, local (2, 1, 1), slot (2*4 + 1)*8 + 1 = 73
-      (3, 4, 8):             raster 228, block 3, local (3, 0, 0), slot 96
+      (2, 1, 9):             raster 139, block 1, local (2, 1, 1), slot (2*4 + 1)*2 + 1 = 19
+      (3, 4, 8):             raster 228, block 3, local (3, 0, 0), slot (3*2 + 0)*2 + 0 = 12
       (4, 0, 2):             raster 242, block 4, local (0, 0, 2), slot 2
-      (4, 5, 9):             raster 299, block 7, local (0, 1, 1), slot 9
-    Valid tokens per block (t extent * h extent * w extent; the last block along an axis keeps
-    1 frame, 2 rows or 2 columns): block 0: 4*4*8 = 128, 1: 4*4*2 = 32, 2: 4*2*8 = 64,
-    3: 4*2*2 = 16, 4: 1*4*8 = 32, 5: 1*4*2 = 8, 6: 1*2*8 = 16, 7: 1*2*2 = 4.  The block grid
-    is a 2 x 2 x 2 cube, so only the order of the axes tells these ids apart.
+      (4, 5, 9):             raster 299, block 7, local (0, 1, 1), slot (0*2 + 1)*2 + 1 = 3
+    The block grid is a 2 x 2 x 2 cube, so only the order of the axes tells these ids apart.
     """
     g = Grid(5, 6, 10, (4, 4, 8))
     sm = g.slot_map(5)
     mem = g.block_members(5)
     for (t, h, w), (raster, blk, slot) in {(0, 0, 0): (0, 0, 0), (1, 2, 3): (83, 0, 51),
-                                           (2, 1, 9): (139, 1, 73), (3, 4, 8): (228, 3, 96),
-                                           (4, 0, 2): (242, 4, 2), (4, 5, 9): (299, 7, 9)}.items():
+                                           (2, 1, 9): (139, 1, 19), (3, 4, 8): (228, 3, 12),
+                                           (4, 0, 2): (242, 4, 2), (4, 5, 9): (299, 7, 3)}.items():
         assert (t * 6 + h) * 10 + w == raster
         assert sm[blk, slot] == raster
         assert raster in mem[blk]
     assert [len(m) for m in mem] == [128, 32, 64, 16, 32, 8, 16, 4]
     assert mem[7] == [280 + 8, 280 + 9, 290 + 8, 290 + 9]  # (4,4,8) (4,4,9) (4,5,8) (4,5,9)
-    assert sorted(np.nonzero(sm[7] >= 0)[0].tolist()) == [0, 1, 8, 9]
+    assert sm[7].tolist() == [288, 289, 298, 299] + [-1] * 124  # valid prefix, then pads
+    assert [int((row >= 0).sum()) for row in sm] == [128, 32, 64, 16, 32, 8, 16, 4]
+    assert all(np.all(row[:n] >= 0) and np.all(row[n:] < 0)
+               for row, n in zip(sm, [128, 32, 64, 16, 32, 8, 16, 4]))
 
 
 def test_workload_geometry_matches_pages():
