@@ -11,11 +11,16 @@ value    = effective TFLOP/s of the step on selected-block tile FLOPs (4*BS^2*D 
            selected (query block, key block) pair forward, 2.5x that backward) summed over
            all ranks / max-over-ranks step time.
 e2e      = the same metric through the public pipeline API with host (pinned) raster
-           inputs copied in and the output O copied back inside the timed region, every step;
-           the copies run on their own streams, overlapping the neighbouring steps' compute.
+           inputs q, k, v, dO copied in and the raster results O, dq, dk, dv copied back
+           inside the timed region, every step (O via the inverse relayout, the gradients via
+           the attention backward and the prologue backward); the copies run on their own
+           streams, overlapping the neighbouring steps' compute.
 roofline = the attention kernel with the longest launches (timed live with CUDA events on its
            stream through the library's kernel timing) against the measured sustained
-           dense bf16 tensor peak.
+           dense bf16 tensor peak (the kernels run inside a long step), with the burst-peak
+           fraction beside it.  Each kernel reports its executed GEMM-tile FLOPs and its
+           algorithmic ones: the dQ pass recomputes S and dP, which the algorithmic count
+           leaves out (a backward needs 5 GEMM tiles per pair, 2.5x the forward's 2).
 
 Multi-GPU (torchrun): every rank runs an independent replica of the workload (the path
 has no exchange step: routing and attention are independent per (batch, head)), so
@@ -150,10 +155,12 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def cpu_oracle_sample(w, budget_s: float = 12.0):
-    """Time the fp64 oracle (as it stands) on a bounded sample of the workload: routing of
-    one head plus forward attention of as many query blocks of that head as fit the budget,
-    and backward of a few; reported in TFLOP/s of the same tile-FLOP convention."""
+def cpu_oracle_sample(w, budget_s: float = 12.0, with_bwd: bool = True):
+    """Time the fp64 oracle (as it stands) on a bounded sample of the workload: prologue and
+    routing of one head, forward attention of as many query blocks of that head as fit 40 %
+    of the budget and, with the backward, the backward of as many as fit the rest.  The rate
+    is the step's: tile FLOPs of one query block's forward plus 2.5x that backward, over the
+    oracle's time per query block (routing prorated over the head's query blocks)."""
     import oracle
     grid = oracle.Grid(w.t_frames, w.grid_h, w.grid_w, w.blk, w.cached_t, w.chunk_t, w.cond_t)
     x = make_raster_inputs(w, with_grad=True)
@@ -176,25 +183,42 @@ def cpu_oracle_sample(w, budget_s: float = 12.0):
                          t_offset=w.cached_t)
     idx, cnt, _ = oracle.route(qp, kp, grid, w.top_r, k_cache=kc)
     t_route = time.perf_counter() - t0
-    n_blocks, t_attn = 0, 0.0
-    rng = np.random.default_rng(0)
-    order = rng.permutation(grid.nbq)
-    while t_attn < budget_s and n_blocks < grid.nbq:
-        i = int(order[n_blocks])
-        t1 = time.perf_counter()
-        oracle.attend(qp, kp, v, idx, grid, scale, k_cache=kc, v_cache=vc, query_blocks=[(0, 0, i)])
-        t_attn += time.perf_counter() - t1
-        n_blocks += 1
-    pairs = float(np.mean(cnt[0, 0])) * n_blocks
-    fl = tile_flops(grid.bs, w.head_dim, 1) * pairs
+    order = np.random.default_rng(0).permutation(grid.nbq)
+
+    def timed(fn, budget):
+        n, t = 0, 0.0
+        while t < budget and n < grid.nbq:
+            t1 = time.perf_counter()
+            fn(int(order[n]))
+            t += time.perf_counter() - t1
+            n += 1
+        return n, t
+
+    n_f, t_f = timed(lambda i: oracle.attend(qp, kp, v, idx, grid, scale, k_cache=kc, v_cache=vc,
+                                             query_blocks=[(0, 0, i)]),
+                     budget_s * (0.4 if with_bwd else 1.0))
+    n_b, t_b = timed(lambda i: oracle.attend_bwd(qp, kp, v, do, idx, grid, scale, k_cache=kc,
+                                                 v_cache=vc, query_blocks=[(0, 0, i)]),
+                     budget_s * 0.6) if with_bwd else (0, 0.0)
+    pairs = float(np.mean(cnt[0, 0]))  # selected key blocks per query block
+    fl_blk = tile_flops(grid.bs, w.head_dim, 1) * pairs
+    t_blk = t_f / n_f + (t_b / n_b if n_b else 0.0) + t_route / grid.nbq
+    fl = fl_blk * (3.5 if with_bwd else 1.0)
     cores = len(os.sched_getaffinity(0))
-    return {
-        "value": fl / (t_attn + t_route * n_blocks / grid.nbq) / 1e12,
+    out = {
+        "value": fl / t_blk / 1e12,
         "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+        "fwd_tflops": fl_blk / (t_f / n_f) / 1e12,
         "sample": f"fp64 oracle: prologue+route of 1/{w.heads} heads, forward attention of "
-                  f"{n_blocks} query blocks of that head ({pairs:.0f} block pairs); route time "
-                  f"prorated to the sampled blocks; {t_attn + t_route:.1f} s of CPU work",
+                  f"{n_f} query blocks of that head" +
+                  (f" and backward of {n_b}" if with_bwd else "") +
+                  f" ({pairs:.0f} key blocks each); rate = (fwd + 2.5x fwd) tile FLOPs per "
+                  f"query block over fwd + bwd + prorated route time per query block; "
+                  f"{t_f + t_b + t_route:.1f} s of CPU work",
     }
+    if with_bwd:
+        out["bwd_tflops"] = 2.5 * fl_blk / (t_b / n_b) / 1e12
+    return out
 
 
 def main():
@@ -220,7 +244,8 @@ def main():
         if rank != 0:
             return 0
         t0 = time.perf_counter()
-        vals = [cpu_oracle_sample(w, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)))
+        vals = [cpu_oracle_sample(w, budget_s=max(2.0, 60.0 / max(1, args.steps + args.warmup)),
+                                  with_bwd=not args.no_bwd)
                 for _ in range(args.warmup + args.steps)][args.warmup:]
         v = float(np.median([x["value"] for x in vals]))
         cb = dict(vals[-1])
@@ -343,41 +368,58 @@ def main():
         ms_max = float(tt.item())
 
     # ---------------- end to end through the public pipeline, host buffers in and out.
-    # Every step copies its raster q, k, v in from pinned host memory and O out; the copies
+    # Every step copies its raster q, k, v (and dO with the backward) in from pinned host
+    # memory and its results out: O turned back to the raster layout by the inverse relayout
+    # and, with the backward, the raster gradients dq, dk, dv of the step's raster inputs
+    # (attention backward, then the prologue backward through RoPE and RMSNorm).  The copies
     # run on their own streams so that step k+1's upload and step k's download overlap the
-    # compute (two device input sets; events order every reuse).
-    pin = {k_: torch.from_numpy(x[k_].view(np.int16)).pin_memory() for k_ in ("q", "k", "v")}
-    o_host = torch.empty(pipe.o.shape, dtype=torch.bfloat16).pin_memory()
+    # compute (two device sets of inputs and of outputs; events order every reuse).
+    in_keys = ("q", "k", "v") + (("do",) if with_bwd else ())
+    out_keys = ("o",) + (("dq", "dk", "dv") if with_bwd else ())
+    pin = {k_: torch.from_numpy(x[k_].view(np.int16)).pin_memory() for k_ in in_keys}
+    host_out = {k_: torch.empty(q_d.shape, dtype=torch.int16).pin_memory() for k_ in out_keys}
     e_steps = max(3, args.steps)  # as many as the timed steps; the first upload is pipeline fill
-    sets = [{k_: torch.empty_like(q_d) for k_ in ("q", "k", "v")} for _ in range(2)]
+    sets = [{k_: torch.empty_like(q_d) for k_ in in_keys} for _ in range(2)]
+    outs = [{k_: torch.empty_like(q_d) for k_ in out_keys} for _ in range(2)]
+    dgq_e = torch.empty(w.head_dim, device=dev)
+    dgk_e = torch.empty(w.head_dim, device=dev)
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
     def e2e_run(n):
         ev_in = [torch.cuda.Event() for _ in range(n)]    # inputs of step k on the device
-        ev_pro = [torch.cuda.Event() for _ in range(n)]   # prologue k done: input set free
-        ev_fwd = [torch.cuda.Event() for _ in range(n)]   # O of step k written
-        ev_out = [torch.cuda.Event() for _ in range(n)]   # O of step k copied out
+        ev_free = [torch.cuda.Event() for _ in range(n)]  # step k no longer reads its inputs
+        ev_o = [torch.cuda.Event() for _ in range(n)]     # raster O of step k written
+        ev_done = [torch.cuda.Event() for _ in range(n)]  # every output of step k written
+        ev_out = [torch.cuda.Event() for _ in range(n)]   # outputs of step k copied out
         for k_ in range(n):
-            dst = sets[k_ % 2]
+            src, dst = sets[k_ % 2], outs[k_ % 2]
             with torch.cuda.stream(up):
                 if k_ >= 2:
-                    up.wait_event(ev_pro[k_ - 2])
-                for key in ("q", "k", "v"):
-                    dst[key].view(torch.int16).copy_(pin[key], non_blocking=True)
+                    up.wait_event(ev_free[k_ - 2])
+                for key in in_keys:
+                    src[key].view(torch.int16).copy_(pin[key], non_blocking=True)
                 ev_in[k_].record(up)
             stream.wait_event(ev_in[k_])
-            pipe.prologue(dst["q"], dst["k"], dst["v"], stream)
-            ev_pro[k_].record(stream)
+            if k_ >= 2:
+                stream.wait_event(ev_out[k_ - 2])  # this output set has been copied out
+            pipe.prologue(src["q"], src["k"], src["v"], stream)
             pipe.route(stream)
-            if k_ >= 1:
-                stream.wait_event(ev_out[k_ - 1])  # O of the previous step copied out
             pipe.attn_fwd(stream)
-            ev_fwd[k_].record(stream)
+            pipe.o_to_raster(dst["o"], stream)
+            ev_o[k_].record(stream)
             if with_bwd:
+                pipe.load_grad(src["do"], stream)
                 pipe.backward(stream)
+                pipe.prologue_backward(src["q"], src["k"], dst["dq"], dst["dk"], dst["dv"],
+                                       dgq_e, dgk_e, stream)
+            ev_free[k_].record(stream)
+            ev_done[k_].record(stream)
             with torch.cuda.stream(down):
-                down.wait_event(ev_fwd[k_])
-                o_host.copy_(pipe.o, non_blocking=True)
+                down.wait_event(ev_o[k_])
+                host_out["o"].copy_(dst["o"].view(torch.int16), non_blocking=True)
+                down.wait_event(ev_done[k_])
+                for key in out_keys[1:]:
+                    host_out[key].copy_(dst[key].view(torch.int16), non_blocking=True)
                 ev_out[k_].record(down)
         return ev_out[-1]
 
@@ -392,13 +434,17 @@ def main():
     stream.wait_event(last)
     e1.record(stream)
     torch.cuda.synchronize()
+    st = bsa.bsa_device_status()
+    if st != 0:
+        raise SystemExit(f"device status {st} after the end-to-end run")
     e_ms = e0.elapsed_time(e1) / e_steps
     if world > 1:
         tt = torch.tensor([e_ms], device=dev)
         dist.all_reduce(tt, op=dist.ReduceOp.MAX)
         e_ms = float(tt.item())
     h2d = sum(pin[k_].numel() * 2 for k_ in pin)
-    d2h = o_host.numel() * 2
+    d2h = sum(host_out[k_].numel() * 2 for k_ in host_out)
+    del sets, outs
 
     # ---------------- the next row of the path, timed on its own (not part of the step):
     # the prologue backward, raster q, k, v gradients and the gains' gradients from the
@@ -516,22 +562,31 @@ def main():
 
     peaks = load_peaks()
     peak = peaks["bf16_tflops_sustained"]
-    # algorithmic tensor FLOPs per launch of each attention kernel (128x128xD GEMM tiles):
-    # forward S and PV per selected pair; dK/dV pass S^T, dP^T, dV, dK per pair with a
-    # current key block; dQ pass S, dP, dQ per selected pair
-    kflops = {"fwd": tile_flops(g.bs, g.head_dim, n_pairs),
-              "bwd_dkdv": 2 * tile_flops(g.bs, g.head_dim, n_pairs_cur),
-              "bwd_dq": 1.5 * tile_flops(g.bs, g.head_dim, n_pairs)}
+    peak_burst = peaks["bf16_tflops"]
+    # tensor FLOPs per launch of each attention kernel in 128x128xD GEMM tiles (2*BS*BS*D each).
+    # Executed: forward S and PV per selected pair; dK/dV pass S^T, dP^T, dV, dK per pair with a
+    # current key block; dQ pass S, dP, dQ per selected pair.  Algorithmic: the same, except that
+    # the dQ pass's S and dP repeat the dK/dV pass's and are not counted (dQ = dS K only), so
+    # the backward's algorithmic total is the usual 5 tiles per pair, 2.5x the forward.
+    half = 0.5 * tile_flops(g.bs, g.head_dim, 1)  # one GEMM tile
+    kflops = {"fwd": 2 * half * n_pairs, "bwd_dkdv": 4 * half * n_pairs_cur,
+              "bwd_dq": 3 * half * n_pairs}
+    kflops_alg = {"fwd": 2 * half * n_pairs, "bwd_dkdv": 4 * half * n_pairs_cur,
+                  "bwd_dq": 1 * half * n_pairs}
     kernels = {}
     for kname, (nl, tot_ms, min_ms, med_ms) in ktimes.items():
         if nl == 0:
             continue
         avg = tot_ms / nl
         kernels[kname] = {"launches": nl, "ms_per_launch": avg, "ms_median": med_ms,
-                          "ms_min": min_ms, "tflops": kflops[kname] / (avg * 1e-3) / 1e12}
+                          "ms_min": min_ms,
+                          "tflops_executed": kflops[kname] / (avg * 1e-3) / 1e12,
+                          "tflops_algorithmic": kflops_alg[kname] / (avg * 1e-3) / 1e12}
+        kernels[kname]["frac_algorithmic"] = kernels[kname]["tflops_algorithmic"] / peak
     dom = max(kernels, key=lambda k_: kernels[k_]["ms_per_launch"])
-    achieved = kernels[dom]["tflops"]
+    achieved = kernels[dom]["tflops_algorithmic"]
     value = world * fl_step / (ms_max * 1e-3) / 1e12
+    fwd_ms, bwd_ms = parts["fwd"], parts.get("bwd")
     line = {
         "metric": "BSA fwd(+bwd) effective TFLOP/s at 720p tokens",
         "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
@@ -548,17 +603,28 @@ def main():
         "kernels": kernels,
         "roofline": {"bound": "tensor", "kernel": KERNEL_NAMES[dom], "achieved": achieved,
                      "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "frac_burst": achieved / peak_burst, "peak_burst": peak_burst,
                      "peak_source": f"{peaks['source']} bf16 dense, sustained (of measured)"
                                     if peaks["source"] == "measured" else "fallback",
-                     "traffic": traffic_per_launch(dom, args.workload, n_pairs, n_pairs_cur)},
+                     "traffic": traffic_per_launch(dom, args.workload, n_pairs, n_pairs_cur),
+                     "fwd_frac": fl_fwd / (fwd_ms * 1e-3) / 1e12 / peak,
+                     "bwd_algorithmic_frac": (2.5 * fl_fwd / (bwd_ms * 1e-3) / 1e12 / peak
+                                              if with_bwd else None),
+                     "step_frac": value / world / peak, "step_frac_burst": value / world / peak_burst,
+                     "note": "achieved = algorithmic GEMM-tile FLOPs of the kernel / its mean "
+                             "launch time; fwd_frac, bwd_algorithmic_frac and step_frac use the "
+                             "step's phase times (forward 2 tiles per pair, backward 5, step 7)"},
         "e2e": {"value": world * fl_step / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "ms_per_step": e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "copied_in": list(in_keys), "copied_out": [k_ + "_raster" for k_ in out_keys],
+                "path": "prologue, route, fwd, O to raster" +
+                        (", dO relayout, bwd, prologue bwd" if with_bwd else "")},
         "next_rows": next_rows,
         "gpu_launches": args.steps * (3 + (4 if with_bwd else 0)),
         "clocks": clk.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_oracle_sample(w)
+        line["cpu_baseline"] = cpu_oracle_sample(w, with_bwd=with_bwd)
     if rank == 0:
         print(json.dumps(line))
     if world > 1:
