@@ -232,7 +232,6 @@ template <int BS, int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bsa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                         const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
-                        const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmdO16,
                         const BwdParams p) {
   using L = DkdvLayout<BS, D>;
   constexpr int NS = L::kSlots;
@@ -361,27 +360,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           const int qrow = (bh * g.NBq + i) * BS;
           if (round > 0 && !mbar_wait(&q_empty[slot], (round - 1) & 1, abort_flag)) { ok = false; break; }
           unsigned char* vec = smem + L::kVecOff + slot * L::kVecBytes;
-          const int nv = query_block_nvalid(g, i);
-          slot_nv[slot] = nv;
-          // only the rows the tensor cores read: a partial query block's valid prefix rounded
-          // up to 16, in 16-row boxes (a full block in one box per half)
-          const int nrows = nv >= BS ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
-          mbar_expect_tx(&q_full[slot], 2u * (uint32_t)nrows * 128u * (D / 64) + L::kVecBytes);
-          unsigned char* dq_ = smem + L::kQOff + slot * L::kTileBytes;
-          unsigned char* ddo = smem + L::kDOOff + slot * L::kTileBytes;
-          if (nrows == BS) {
+          slot_nv[slot] = query_block_nvalid(g, i);
+          // whole tiles even for a partial query block (16-row boxes of only its valid rows
+          // measured no faster)
+          mbar_expect_tx(&q_full[slot], 2 * L::kTileBytes + L::kVecBytes);
 #pragma unroll
-            for (int half = 0; half < D / 64; ++half) {
-              tma_load_2d(dq_ + half * BS * 128, &tmQ, half * 64, qrow, &q_full[slot]);
-              tma_load_2d(ddo + half * BS * 128, &tmdO, half * 64, qrow, &q_full[slot]);
-            }
-          } else {
-            for (int r0 = 0; r0 < nrows; r0 += 16)
-#pragma unroll
-              for (int half = 0; half < D / 64; ++half) {
-                tma_load_2d(dq_ + half * BS * 128 + r0 * 128, &tmQ16, half * 64, qrow + r0, &q_full[slot]);
-                tma_load_2d(ddo + half * BS * 128 + r0 * 128, &tmdO16, half * 64, qrow + r0, &q_full[slot]);
-              }
+          for (int half = 0; half < D / 64; ++half) {
+            tma_load_2d(smem + L::kQOff + slot * L::kTileBytes + half * BS * 128, &tmQ, half * 64,
+                        qrow, &q_full[slot]);
+            tma_load_2d(smem + L::kDOOff + slot * L::kTileBytes + half * BS * 128, &tmdO, half * 64,
+                        qrow, &q_full[slot]);
           }
           bulk_load(vec, p.nlse2 + (size_t)qrow, BS * 4, &q_full[slot]);
           bulk_load(vec + BS * 4, p.ndelta + (size_t)qrow, BS * 4, &q_full[slot]);
@@ -692,8 +680,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bsa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmdO,
                       const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                       const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
-                      const __grid_constant__ CUtensorMap tmK16, const __grid_constant__ CUtensorMap tmV16,
-                      const __grid_constant__ CUtensorMap tmKc16, const __grid_constant__ CUtensorMap tmVc16,
                       const BwdParams p) {
   using L = DqLayout<BS, D>;
   constexpr int S = L::kStages;
@@ -771,36 +757,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int bhx = item / g.NBq;
         for (int n = 0; n < cnt && ok; ++n) {
           const int j = item_idx(item, n);
-          const CUtensorMap *mk, *mv, *mk16, *mv16;
+          const CUtensorMap *mk, *mv;
           int row;
-          if (j < g.NBc) {
-            mk = &tmKc; mv = &tmVc; mk16 = &tmKc16; mv16 = &tmVc16;
-            row = (bhx * g.NBc + j) * BS;
-          } else {
-            mk = &tmK; mv = &tmV; mk16 = &tmK16; mv16 = &tmV16;
-            row = (bhx * g.NBq + (j - g.NBc)) * BS;
-          }
+          if (j < g.NBc) { mk = &tmKc; mv = &tmVc; row = (bhx * g.NBc + j) * BS; }
+          else { mk = &tmK; mv = &tmV; row = (bhx * g.NBq + (j - g.NBc)) * BS; }
           const int nv = key_block_nvalid(g, j);
-          // only the rows the tensor cores read: a partial block's valid prefix rounded up to
-          // 16, in 16-row boxes (a full block in one box per half)
-          const int nrows = nv >= BS ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
-          for (int t = 0; t < 2; ++t) {  // K_n then V_n
+          for (int t = 0; t < 2; ++t) {  // K_n then V_n (whole tiles, as in the forward)
             const int stage = seq % S, round = seq / S;
             if (round > 0 && !mbar_wait(&kv_empty[stage], (round - 1) & 1, abort_flag)) { ok = false; break; }
             unsigned char* dst = smem + L::kRingOff + stage * L::kKVBytes;
             stage_nv[stage] = nv;
-            mbar_expect_tx(&kv_full[stage], (uint32_t)nrows * 128u * (D / 64));
-            if (nrows == BS) {
+            mbar_expect_tx(&kv_full[stage], L::kKVBytes);
 #pragma unroll
-              for (int half = 0; half < D / 64; ++half)
-                tma_load_2d(dst + half * BS * 128, t == 0 ? mk : mv, half * 64, row, &kv_full[stage]);
-            } else {
-              for (int r0 = 0; r0 < nrows; r0 += 16)
-#pragma unroll
-                for (int half = 0; half < D / 64; ++half)
-                  tma_load_2d(dst + half * BS * 128 + r0 * 128, t == 0 ? mk16 : mv16, half * 64,
-                              row + r0, &kv_full[stage]);
-            }
+            for (int half = 0; half < D / 64; ++half)
+              tma_load_2d(dst + half * BS * 128, t == 0 ? mk : mv, half * 64, row, &kv_full[stage]);
             ++seq;
           }
         }
@@ -972,11 +942,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           nreg = n + lane < cnt ? key_block_nvalid(g, jcur) : BS;
           partial = __ballot_sync(0xffffffffu, nreg < BS);
         }
+        const int nvb = ((partial >> (n & 31)) & 1u) ? __shfl_sync(0xffffffffu, nreg, n & 31) : BS;
         // A group whose keys all lie past a partial block's valid prefix has nothing to do in
         // this step (the tensor cores compute only the first roundup16(valid) keys and read
         // dS of those only); it keeps the waits and arrivals, in order, so no barrier phase
-        // can be overrun.
-        const int nvb = ((partial >> (n & 31)) & 1u) ? __shfl_sync(0xffffffffu, nreg, n & 31) : BS;
+        // can be overrun.  (Spreading a small block's keys over all four groups, with dS
+        // packed behind a named barrier, measured 2 % slower.)
         if (cg * KC >= nvb) {
           bool w_ok = mbar_wait(s_full, gn & 1, abort_flag);
           w_ok = __all_sync(0xffffffffu, w_ok);
@@ -1067,8 +1038,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 }
 
 // ------------------------------------------------------------------------------ host side
-// maps: 0 Q (box 128 rows), 1 K, 2 V, 3 K cache, 4 V cache (box BS rows), 5 dO (box 128 rows);
-// 6-9 K, V, K cache, V cache and 10-11 Q, dO with 16-row boxes
+// maps: 0 Q (box 128 rows), 1 K, 2 V, 3 K cache, 4 V cache (box BS rows), 5 dO (box 128 rows)
 bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, const CUtensorMap* maps,
                      int n_sm, cudaStream_t s) {
   if (g.BS != 128) return BSA_ERR_UNSUPPORTED;  // the key-major pass needs 128-token blocks
@@ -1122,7 +1092,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
       return BSA_ERR_CUDA;                                                                        \
     cudaEvent_t e1;                                                                               \
     const int w1 = timed_begin(BSA_TIMED_BWD_DKDV, s, &e1);                                       \
-    k1<<<grid, kBwdThreads, s1, s>>>(maps[1], maps[2], maps[0], maps[5], maps[10], maps[11], a);  \
+    k1<<<grid, kBwdThreads, s1, s>>>(maps[1], maps[2], maps[0], maps[5], a);                      \
     timed_end(w1, s, e1);                                                                         \
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;                                   \
     BwdParams c = bp;                                                                             \
@@ -1134,8 +1104,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
       return BSA_ERR_CUDA;                                                                        \
     cudaEvent_t e2;                                                                               \
     const int w2 = timed_begin(BSA_TIMED_BWD_DQ, s, &e2);                                         \
-    k2<<<grid, kBwdThreads, s2, s>>>(maps[0], maps[5], maps[1], maps[2], maps[3], maps[4],      \
-                                     maps[6], maps[7], maps[8], maps[9], c);                     \
+    k2<<<grid, kBwdThreads, s2, s>>>(maps[0], maps[5], maps[1], maps[2], maps[3], maps[4], c);   \
     timed_end(w2, s, e2);                                                                         \
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;                                   \
   } while (0)

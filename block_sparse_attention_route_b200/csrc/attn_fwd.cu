@@ -46,8 +46,6 @@
 // 0 of item j (its slot's previous Q, item j-1's, is no longer read: every S of item j-1
 // completed before S(0) of item j) and free the staging buffer, and the MMA thread waits for
 // the copy before the first S of item j+1.
-#include <type_traits>
-
 #include "common.cuh"
 
 namespace bsa {
@@ -81,8 +79,7 @@ struct FwdLayout {
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kXchOff = kMiscOff + 16;               // float [2 parity][4 groups][128]
   static constexpr int kSumOff = kXchOff + 2 * 4 * 128 * 4;   // float [4 groups][128]
-  static constexpr int kStageNvOff = kSumOff + 4 * 128 * 4;  // int [stages]: valid keys of the tile
-  static constexpr int kBytes = kStageNvOff + kFwdStages * 4;
+  static constexpr int kBytes = kSumOff + 4 * 128 * 4;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
@@ -108,9 +105,7 @@ template <int BS, int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmKc,
-                   const __grid_constant__ CUtensorMap tmVc, const __grid_constant__ CUtensorMap tmK16,
-                   const __grid_constant__ CUtensorMap tmV16, const __grid_constant__ CUtensorMap tmKc16,
-                   const __grid_constant__ CUtensorMap tmVc16, const FwdParams p) {
+                   const __grid_constant__ CUtensorMap tmVc, const FwdParams p) {
   using L = FwdLayout<BS, D>;
   constexpr int S = kFwdStages;
   extern __shared__ unsigned char smem_raw[];
@@ -129,9 +124,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   uint64_t* fin_bar = o_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-  // valid keys of the K / V tile in each ring stage (written by the producer before the tile's
-  // kv_full arrival, read by the MMA thread after waiting on it)
-  volatile int* stage_nv = reinterpret_cast<volatile int*>(smem + L::kStageNvOff);
 
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const Geo& g = p.g;
@@ -183,38 +175,19 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       int seq = 0, items = 0;
       bool ok = true;
       unsigned char* ring = smem + L::kRingOff;
-      auto kv_tile = [&](int item, int n, bool is_v) -> bool {
+      // K or V tile of key block j of head row bhx into the next ring stage
+      auto kv_tile = [&](int bhx, int j, bool is_v) -> bool {
         const int stage = seq % S, round = seq / S;
         if (round > 0 && !mbar_wait(&kv_empty[stage], (round - 1) & 1, abort_flag)) return false;
-        const int j = load_idx(p, item, n);
-        const int bhx = item / g.NBq;
-        const CUtensorMap *map, *map16;
+        const CUtensorMap* map;
         int row;
-        if (j < g.NBc) {
-          map = is_v ? &tmVc : &tmKc; map16 = is_v ? &tmVc16 : &tmKc16;
-          row = (bhx * g.NBc + j) * BS;
-        } else {
-          map = is_v ? &tmV : &tmK; map16 = is_v ? &tmV16 : &tmK16;
-          row = (bhx * g.NBq + (j - g.NBc)) * BS;
-        }
+        if (j < g.NBc) { map = is_v ? &tmVc : &tmKc; row = (bhx * g.NBc + j) * BS; }
+        else { map = is_v ? &tmV : &tmK; row = (bhx * g.NBq + (j - g.NBc)) * BS; }
         unsigned char* dst = ring + stage * L::kKVBytes;
-        const int nv = key_block_nvalid(g, j);
-        stage_nv[stage] = nv;
-        // only the rows the tensor cores read: a partial 128-key block's valid prefix rounded
-        // up to 16, in 16-row boxes (full blocks and 32-key blocks in one box per half)
-        const int nrows = (BS != 128 || nv >= BS) ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
-        mbar_expect_tx(&kv_full[stage], (uint32_t)nrows * 128u * (D / 64));
-        if (nrows == BS) {
+        mbar_expect_tx(&kv_full[stage], L::kKVBytes);
 #pragma unroll
-          for (int half = 0; half < D / 64; ++half)
-            tma_load_2d(dst + half * BS * 128, map, half * 64, row, &kv_full[stage]);
-        } else {
-          for (int r0 = 0; r0 < nrows; r0 += 16)
-#pragma unroll
-            for (int half = 0; half < D / 64; ++half)
-              tma_load_2d(dst + half * BS * 128 + r0 * 128, map16, half * 64, row + r0,
-                          &kv_full[stage]);
-        }
+        for (int half = 0; half < D / 64; ++half)
+          tma_load_2d(dst + half * BS * 128, map, half * 64, row, &kv_full[stage]);
         ++seq;
         return true;
       };
@@ -238,10 +211,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int cnt = load_cnt(p, item);
         const int nxt = next_item(item + gridDim.x);
         if (nxt < p.n_items) ok = q_tile(nxt);
-        ok = ok && kv_tile(item, 0, false) && (cnt < 2 || kv_tile(item, 1, false));
+        // Key-block indices of steps n, n+1, n+2 ride in registers and the index of step n+3
+        // is loaded one step ahead, so no global-load latency sits in the chain of waits and
+        // TMA issues (each index is loaded once, for its K tile, and reused for its V tile).
+        const int bhx = item / g.NBq;
+        int j0 = load_idx(p, item, 0), j1 = cnt > 1 ? load_idx(p, item, 1) : 0;
+        int j2 = cnt > 2 ? load_idx(p, item, 2) : 0;
+        ok = ok && kv_tile(bhx, j0, false) && (cnt < 2 || kv_tile(bhx, j1, false));
         for (int n = 0; n < cnt && ok; ++n) {
-          ok = kv_tile(item, n, true);
-          if (ok && n + 2 < cnt) ok = kv_tile(item, n + 2, false);
+          const int j3 = n + 3 < cnt ? load_idx(p, item, n + 3) : 0;  // used next step
+          ok = kv_tile(bhx, j0, true);                                 // V(n)
+          if (ok && n + 2 < cnt) ok = kv_tile(bhx, j2, false);         // K(n+2)
+          j0 = j1; j1 = j2; j2 = j3;
         }
         item = nxt;
       }
@@ -258,16 +239,8 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   } else if (warp == kMmaWarp) {
     // ================================================================ MMA issuer
     if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kTileM, BS, 0, 0);
       constexpr uint32_t idPV = idesc_bf16(kTileM, D, 0, 1);
-      // Keys of a tile on the tensor cores: a 128-key block's valid prefix rounded up to 16
-      // (the MMA's N step), so a partial block's S and PV shrink with it; 32-key blocks
-      // keep their full width.  Read right after the tile's kv_full wait, ahead of the
-      // P-ready wait, so the shared-memory load stays off the MMA issue path.
-      auto tile_keys = [&](int stage) -> int {
-        if (BS != 128) return BS;
-        const int nv = stage_nv[stage];
-        return nv >= BS ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
-      };
       const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
       const uint64_t dv = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
       int seq = 0, items = 0, gs = 0, gp = 0;  // ring position, items, S issued, P consumed
@@ -280,7 +253,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       };
       // S(gs) = Q K^T into buffer gs & 1: A = Q from TMEM slot a_q (K16 slice kk at column
       // 8 kk), B = the K tile in ring stage `stage`
-      auto mma_S = [&](uint32_t a_q, int stage, uint32_t idS) {
+      auto mma_S = [&](uint32_t a_q, int stage) {
         const uint64_t kb = dk + (uint64_t)((stage * L::kKVBytes) >> 4);
         const uint32_t d_s = tmem_base + (gs & 1) * 128;
 #pragma unroll
@@ -305,14 +278,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int k1 = (k0 >= 0 && cnt >= 2) ? wait_tile() : -1;
         if (cnt >= 2) ++seq;
         if (k0 < 0 || (cnt >= 2 && k1 < 0)) { ok = false; break; }
-        const uint32_t id0 = idesc_bf16(kTileM, tile_keys(k0), 0, 0);
-        const uint32_t id1 = cnt >= 2 ? idesc_bf16(kTileM, tile_keys(k1), 0, 0) : 0u;
         tc_fence_after();
         const uint32_t dq = t_q0 + qb * (D / 2);
         const int gs0 = gs;
-        mma_S(dq, k0, id0);
+        mma_S(dq, k0);
         ++gs;
-        if (cnt >= 2) { mma_S(dq, k1, id1); ++gs; }
+        if (cnt >= 2) { mma_S(dq, k1); ++gs; }
         mma_commit(&s_full[gs0 & 1]);
         if (cnt >= 2) mma_commit(&s_full[(gs0 + 1) & 1]);
         mma_commit(&kv_empty[k0]);
@@ -324,8 +295,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const int sk = (sv >= 0 && more) ? wait_tile() : -1;
           if (more) ++seq;
           if (sv < 0 || (more && sk < 0)) { ok = false; break; }
-          const int nk = tile_keys(sv) / 16;  // K16 slices of P (keys) on the tensor cores
-          const uint32_t idk = more ? idesc_bf16(kTileM, tile_keys(sk), 0, 0) : 0u;
           // O += P(n) V(n): A = P from TMEM (buffer gp & 1), B = V (MN-major)
           if (!mbar_wait(&p_full[gp & 1], (gp >> 1) & 1, abort_flag)) { ok = false; break; }
           tc_fence_after();
@@ -333,11 +302,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
           const uint32_t a_p = tmem_base + (gp & 1) * 128;
 #pragma unroll
           for (int kk = 0; kk < BS / 16; ++kk)
-            if (kk < nk)
-              mma_ts(t_o0, a_p + kk * 8, vb + (uint64_t)((kk * 2048) >> 4), idPV,
-                     (n > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(t_o0, a_p + kk * 8, vb + (uint64_t)((kk * 2048) >> 4), idPV,
+                   (n > 0 || kk > 0) ? 1u : 0u);
           if (more) {  // S(n+2) into the buffer P(n) came from (read above, in issue order)
-            mma_S(dq, sk, idk);
+            mma_S(dq, sk);
             mma_commit(&s_full[gs & 1]);
             ++gs;
           }
@@ -397,8 +365,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       const int cnt = cnt_next;  // the next item's count is fetched one item ahead
       cnt_next = item + (int)gridDim.x < p.n_items ? load_cnt(p, item + gridDim.x) : 0;
       const int i = item % g.NBq;
-      // this row's query slot holds a token iff it lies in the block's valid prefix (rows >= BS
-      // belong to the tile's padding and are discarded)
+      // this row's query slot (rows >= BS belong to the tile's padding and are discarded)
       const bool qvalid = row < BS && row < query_block_nvalid(g, i);
       float* lse_row = p.lse + (size_t)item * BS;
       __nv_bfloat16* o_row = p.o + ((size_t)item * BS + row) * D + cg * OC;
@@ -416,7 +383,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
       float m = -INFINITY, l = 0.f;
       // Key-block indices come 32 steps at a time (lane e holds step n0 + e), the next chunk's
       // load in flight while the current one runs; per chunk a ballot marks the steps whose
-      // block is partial and each lane keeps its step's valid-key count, so no global load or
+      // block is partial and each lane keeps its step's shape code, so no global load or
       // index arithmetic sits between a step's S and its P.
       int jnext = lane < cnt ? load_idx(p, item, lane) : 0;
       int nreg = BS;
@@ -434,99 +401,79 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         if (!w_ok) { ok = false; break; }
         tc_fence_after();
         const uint32_t t_s = tmem_base + t_lane + b * 128;
-        // This step's keys held by this thread.  A full block gives each group KC keys
-        // ([cg*KC, cg*KC + KC)).  A partial 128-key block (valid keys = the first nv slots)
-        // spreads its first N = roundup16(nv) keys, all the tensor cores computed, over the
-        // four groups: CW = 8, 16 or 32 columns each, so a small block costs the softmax a
-        // fraction of a full step.  P of key k lands at column k / 2 either way (the layout
-        // the PV MMA reads).
-        const bool part = (partial >> (n & 31)) & 1u;
-        const int nvb = part ? __shfl_sync(0xffffffffu, nreg, n & 31) : BS;
-        auto softmax_step = [&](auto cw_t) -> bool {
-          constexpr int CW = decltype(cw_t)::value;
-          float s[CW];
-          {
-            uint32_t* sr = reinterpret_cast<uint32_t*>(s);
-            if constexpr (CW == 32) tmem_ld32_wait(t_s + cg * CW, sr);
-            else if constexpr (CW == 16) tmem_ld16_wait(t_s + cg * CW, sr);
-            else tmem_ld8_wait(t_s + cg * CW, sr);
-          }
-          // pad keys of a partial block (its slots >= its valid count) get -inf
-          if (part) {
-            const int nv = nvb - cg * CW;
+        float s[KC];
+        {
+          uint32_t* sr = reinterpret_cast<uint32_t*>(s);
+          if constexpr (KC == 32) tmem_ld32_wait(t_s + cg * KC, sr);
+          else tmem_ld8_wait(t_s + cg * KC, sr);
+        }
+        // pad keys of a partial block get -inf (mask from the per-shape table)
+        if ((partial >> (n & 31)) & 1u) {
+          const int nv = __shfl_sync(0xffffffffu, nreg, n & 31) - cg * KC;
 #pragma unroll
-            for (int c = 0; c < CW; ++c)
-              if (c >= nv) s[c] = -INFINITY;
-          }
-          float mx;
-          {
-            float a0 = s[0], a1 = s[1];
+          for (int c = 0; c < KC; ++c)
+            if (c >= nv) s[c] = -INFINITY;
+        }
+        float mx;
+        {
+          float a0 = s[0], a1 = s[1];
 #pragma unroll
-            for (int c = 2; c + 4 <= CW; c += 4) {
-              a0 = max3f(a0, s[c], s[c + 1]);
-              a1 = max3f(a1, s[c + 2], s[c + 3]);
-            }
-            mx = max3f(a0, a1, fmaxf(s[CW - 2], s[CW - 1]));
+          for (int c = 2; c + 4 <= KC; c += 4) {
+            a0 = max3f(a0, s[c], s[c + 1]);
+            a1 = max3f(a1, s[c + 2], s[c + 3]);
           }
-          // exchange the four partial row maxima; the slots alternate with the step parity
-          float* xs = xch + b * 512;
-          xs[cg * 128 + row] = mx;
-          named_bar_sync(1 + quarter, kSoftmaxThreads / 4);
-          mx = fmaxf(fmaxf(xs[row], xs[128 + row]), fmaxf(xs[256 + row], xs[384 + row])) * sl2;
-          // lazy rescale: raise the running max only when it grew by more than 8 (log2 units);
-          // all four threads of a row take the same decision.  tcgen05.ld/st are
-          // warp-collective, so a warp rescales together (alpha = 1 for rows that keep their
-          // max), after PV(n-1).
-          const float m_new = (n == 0 || mx > m + 8.0f) ? mx : m;
-          const bool resc = n > 0 && m_new != m;
-          if (__any_sync(0xffffffffu, resc)) {
-            bool pv_ok = mbar_wait(pv_done, (gstep - 1) & 1, abort_flag);
-            pv_ok = __all_sync(0xffffffffu, pv_ok);
-            if (!pv_ok) return false;
-            tc_fence_after();
-            const float alpha = resc ? fast_exp2(m - m_new) : 1.0f;
-            l *= alpha;
-            uint32_t r[OC];
-            if constexpr (OC == 32) tmem_ld32_wait(t_oc, r);
-            else tmem_ld16_wait(t_oc, r);
+          mx = max3f(a0, a1, fmaxf(s[KC - 2], s[KC - 1]));
+        }
+        // exchange the four partial row maxima; the slots alternate with the step parity
+        float* xs = xch + b * 512;
+        xs[cg * 128 + row] = mx;
+        named_bar_sync(1 + quarter, kSoftmaxThreads / 4);
+        mx = fmaxf(fmaxf(xs[row], xs[128 + row]), fmaxf(xs[256 + row], xs[384 + row])) * sl2;
+        // lazy rescale: raise the running max only when it grew by more than 8 (log2 units);
+        // all four threads of a row take the same decision.  tcgen05.ld/st are warp-collective,
+        // so a warp rescales together (alpha = 1 for rows that keep their max), after PV(n-1).
+        const float m_new = (n == 0 || mx > m + 8.0f) ? mx : m;
+        const bool resc = n > 0 && m_new != m;
+        if (__any_sync(0xffffffffu, resc)) {
+          bool pv_ok = mbar_wait(pv_done, (gstep - 1) & 1, abort_flag);
+          pv_ok = __all_sync(0xffffffffu, pv_ok);
+          if (!pv_ok) { ok = false; break; }
+          tc_fence_after();
+          const float alpha = resc ? fast_exp2(m - m_new) : 1.0f;
+          l *= alpha;
+          uint32_t r[OC];
+          if constexpr (OC == 32) tmem_ld32_wait(t_oc, r);
+          else tmem_ld16_wait(t_oc, r);
 #pragma unroll
-            for (int e = 0; e < OC; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-            if constexpr (OC == 32) tmem_st32(t_oc, r);
-            else tmem_st16(t_oc, r);
-            tmem_wait_st();
-          }
-          m = m_new;
-          // P = exp2(s * scale * log2e - m) as bf16 pairs into columns [cg*CW/2, ..) of this S
-          // buffer (already read by every group: the exchange barrier above)
-          const uint64_t sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(-m, -m);
-          uint64_t sum2 = f2pack(0.f, 0.f);
-          uint32_t pk[CW / 2];
-#pragma unroll
-          for (int e = 0; e < CW / 2; ++e) {
-            float x0, x1;
-            f2unpack(fma2(f2pack(s[2 * e], s[2 * e + 1]), sl2x2, nmx2), x0, x1);
-            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-            sum2 = add2(sum2, f2pack(p0, p1));
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          if constexpr (CW == 32) tmem_st16(t_s + cg * (CW / 2), pk);
-          else if constexpr (CW == 16) tmem_st8(t_s + cg * (CW / 2), pk);
-          else tmem_st4(t_s + cg * (CW / 2), pk);
-          {
-            float l0, l1;
-            f2unpack(sum2, l0, l1);
-            l += l0 + l1;
-          }
+          for (int e = 0; e < OC; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+          if constexpr (OC == 32) tmem_st32(t_oc, r);
+          else tmem_st16(t_oc, r);
           tmem_wait_st();
-          tc_fence_before();
-          mbar_arrive(&p_full[b]);
-          return true;
-        };
-        bool st_ok;
-        if (BS != 128 || nvb > 64) st_ok = softmax_step(std::integral_constant<int, KC>{});
-        else if (nvb > 32) st_ok = softmax_step(std::integral_constant<int, 16>{});
-        else st_ok = softmax_step(std::integral_constant<int, 8>{});
-        if (!st_ok) { ok = false; break; }
+        }
+        m = m_new;
+        // P = exp2(s * scale * log2e - m) as bf16 pairs into columns [cg*KC/2, ..) of this S
+        // buffer (already read by every group: the exchange barrier above)
+        const uint64_t sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(-m, -m);
+        uint64_t sum2 = f2pack(0.f, 0.f);
+        uint32_t pk[KC / 2];
+#pragma unroll
+        for (int e = 0; e < KC / 2; ++e) {
+          float x0, x1;
+          f2unpack(fma2(f2pack(s[2 * e], s[2 * e + 1]), sl2x2, nmx2), x0, x1);
+          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+          sum2 = add2(sum2, f2pack(p0, p1));
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        if constexpr (KC == 32) tmem_st16(t_s + cg * (KC / 2), pk);
+        else tmem_st4(t_s + cg * (KC / 2), pk);
+        {
+          float l0, l1;
+          f2unpack(sum2, l0, l1);
+          l += l0 + l1;
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
         // the next item's Q into the other slot (every S of the previous item, the slot's
         // last reader, completed before S(0) of this one)
         if (n == 0 && has_next && !copy_q(jq + 1)) { ok = false; break; }
@@ -574,8 +521,7 @@ cudaError_t launch_fwd(const CUtensorMap* maps, const FwdParams& p, int n_sm, cu
     const int smem = FwdLayout<BSv, Dv>::kAlloc;                                                   \
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem); \
     if (e != cudaSuccess) return e;                                                                \
-    kern<<<grid, kFwdThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],    \
-                                         maps[6], maps[7], maps[8], p);                           \
+    kern<<<grid, kFwdThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], maps[4], p);         \
     return cudaGetLastError();                                                                     \
   } while (0)
   if (bs == 128 && d == 128) BSA_LAUNCH_FWD(128, 128);

@@ -611,24 +611,16 @@ bsa_status_t bsa_attn_fwd(const bsa_geom_t* gi, int32_t top_r, const void* q_blk
   st = check_device(&n_sm);
   if (st != BSA_OK) return st;
   const long bh = (long)g.B * g.H;
-  // 0 Q, 1 K, 2 V, 3 K cache, 4 V cache (whole tiles), 5-8 the same K / V maps with 16-row
-  // boxes (a partial block's valid rows)
-  CUtensorMap maps[9];
+  CUtensorMap maps[5];
   if ((st = encode_blocked(&maps[0], q_blk, bh * g.NBq * g.BS, g.D, kTileM)) != BSA_OK) return st;
   if ((st = encode_blocked(&maps[1], k_blk, bh * g.NBq * g.BS, g.D, g.BS)) != BSA_OK) return st;
   if ((st = encode_blocked(&maps[2], v_blk, bh * g.NBq * g.BS, g.D, g.BS)) != BSA_OK) return st;
-  if ((st = encode_blocked(&maps[5], k_blk, bh * g.NBq * g.BS, g.D, 16)) != BSA_OK) return st;
-  if ((st = encode_blocked(&maps[6], v_blk, bh * g.NBq * g.BS, g.D, 16)) != BSA_OK) return st;
   if (g.NBc > 0) {
     if ((st = encode_blocked(&maps[3], k_cache_blk, bh * g.NBc * g.BS, g.D, g.BS)) != BSA_OK) return st;
     if ((st = encode_blocked(&maps[4], v_cache_blk, bh * g.NBc * g.BS, g.D, g.BS)) != BSA_OK) return st;
-    if ((st = encode_blocked(&maps[7], k_cache_blk, bh * g.NBc * g.BS, g.D, 16)) != BSA_OK) return st;
-    if ((st = encode_blocked(&maps[8], v_cache_blk, bh * g.NBc * g.BS, g.D, 16)) != BSA_OK) return st;
   } else {
     maps[3] = maps[1];
     maps[4] = maps[2];
-    maps[7] = maps[5];
-    maps[8] = maps[6];
   }
   FwdParams p;
   p.g = g;
@@ -675,28 +667,18 @@ bsa_status_t bsa_attn_bwd(const bsa_geom_t* gi, int32_t top_r, const void* q_blk
   if (g.BS != 128)
     return fail(BSA_ERR_UNSUPPORTED, "backward supports 128-token blocks (got %d)", g.BS);
   const long bh = (long)g.B * g.H;
-  // 0 Q, 1 K, 2 V, 3 K cache, 4 V cache, 5 dO (whole tiles); 6-9 K, V, K cache, V cache and
-  // 10-11 Q, dO with 16-row boxes (a partial block's valid rows)
-  CUtensorMap maps[12];
+  CUtensorMap maps[6];
   if ((st = encode_blocked(&maps[0], q_blk, bh * g.NBq * g.BS, g.D, kTileM)) != BSA_OK) return st;
   if ((st = encode_blocked(&maps[1], k_blk, bh * g.NBq * g.BS, g.D, g.BS)) != BSA_OK) return st;
   if ((st = encode_blocked(&maps[2], v_blk, bh * g.NBq * g.BS, g.D, g.BS)) != BSA_OK) return st;
-  if ((st = encode_blocked(&maps[6], k_blk, bh * g.NBq * g.BS, g.D, 16)) != BSA_OK) return st;
-  if ((st = encode_blocked(&maps[7], v_blk, bh * g.NBq * g.BS, g.D, 16)) != BSA_OK) return st;
   if (g.NBc > 0) {
     if ((st = encode_blocked(&maps[3], k_cache_blk, bh * g.NBc * g.BS, g.D, g.BS)) != BSA_OK) return st;
     if ((st = encode_blocked(&maps[4], v_cache_blk, bh * g.NBc * g.BS, g.D, g.BS)) != BSA_OK) return st;
-    if ((st = encode_blocked(&maps[8], k_cache_blk, bh * g.NBc * g.BS, g.D, 16)) != BSA_OK) return st;
-    if ((st = encode_blocked(&maps[9], v_cache_blk, bh * g.NBc * g.BS, g.D, 16)) != BSA_OK) return st;
   } else {
     maps[3] = maps[1];
     maps[4] = maps[2];
-    maps[8] = maps[6];
-    maps[9] = maps[7];
   }
   if ((st = encode_blocked(&maps[5], do_blk, bh * g.NBq * g.BS, g.D, kTileM)) != BSA_OK) return st;
-  if ((st = encode_blocked(&maps[10], q_blk, bh * g.NBq * g.BS, g.D, 16)) != BSA_OK) return st;
-  if ((st = encode_blocked(&maps[11], do_blk, bh * g.NBq * g.BS, g.D, 16)) != BSA_OK) return st;
   BwdPtrs P;
   P.q = q_blk; P.k = k_blk; P.v = v_blk; P.kc = k_cache_blk; P.vc = v_cache_blk;
   P.o = o_blk; P.lse = lse; P.dO = do_blk; P.idx = idx; P.cnt = cnt;

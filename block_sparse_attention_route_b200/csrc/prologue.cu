@@ -319,6 +319,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
   const int rid = tid / LPR, cl = tid % LPR, c0 = cl * 8;
   const int heads_here = min(kHeadsPerCta, g.H - hg * kHeadsPerCta);
   const int hpc = kSharded ? heads_here : kHeadsPerCta;  // as in the forward
+  const int rows = hpc * g.BS;
   const size_t n_raster = (size_t)f.frames * g.GH * g.GW;
   int ax[4], pi[4];
 #pragma unroll
@@ -340,37 +341,11 @@ __global__ void __launch_bounds__(kPrologueThreads)
     float gv[8], gacc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) { gv[e] = gam ? gam[c0 + e] : 1.f; gacc[e] = 0.f; }
-    // A block's valid tokens are its first slots, so the pad rows (which contribute nothing)
-    // are not visited.  This lane's 16 bytes of dz (and of x, with a gain) of the row of pass
-    // `bs`: the next pass's loads are issued before the current pass is processed, so two
-    // are in flight.
-    const int rows_v = hpc * nvalid;
-    auto fetch = [&](int bs, uint4& rz, uint4& rx) {
-      const int row = bs + rid;
-      const int hl = row % hpc, slot = row / hpc;
-      rz = rx = make_uint4(0u, 0u, 0u, 0u);
-      if (row < rows_v && hl < heads_here) {
-        const int h = hg * kHeadsPerCta + hl;
-        int lt, lh, lw, sidx;
-        slot_local(g, slot, vh, vw, full, lt, lh, lw);
-        rz = __ldg(reinterpret_cast<const uint4*>(
-            dz + ((((size_t)b * g.H + h) * (size_t)(f.nbt * per_t) + blk) * g.BS + slot) * D + c0));
-        if (gam) {
-          const size_t xo = shard_elem<kSharded, D>(f.sh, g, n_raster, b, ibt * g.bt + lt,
-                                                    ibh * g.bh + lh, ibw * g.bw + lw, h, c0, sidx);
-          rx = __ldg(reinterpret_cast<const uint4*>((kSharded ? a.x[which][sidx] : xin0) + xo));
-        }
-      }
-    };
-    uint4 nz, nx;
-    fetch(0, nz, nx);
-    for (int base = 0; base < rows_v; base += RPP) {
-      const uint4 rz = nz, rx = nx;
-      if (base + RPP < rows_v) fetch(base + RPP, nz, nx);
+    for (int base = 0; base < rows; base += RPP) {
       const int row = base + rid;
       const int hl = row % hpc, slot = row / hpc;
       const int h = hg * kHeadsPerCta + hl;
-      const bool valid = row < rows_v && hl < heads_here;
+      const bool valid = row < rows && hl < heads_here && slot < nvalid;
       int lt = 0, lh = 0, lw = 0;
       if (valid) slot_local(g, slot, vh, vw, full, lt, lh, lw);
       float v[8], xv[8];
@@ -381,6 +356,8 @@ __global__ void __launch_bounds__(kPrologueThreads)
       if (valid) {
         const int t = ibt * g.bt + lt, hh = ibh * g.bh + lh, ww = ibw * g.bw + lw;
         xoff = shard_elem<kSharded, D>(f.sh, g, n_raster, b, t, hh, ww, h, c0, sidx);
+        const uint4 rz = __ldg(reinterpret_cast<const uint4*>(
+            dz + ((((size_t)b * g.H + h) * (size_t)(f.nbt * per_t) + blk) * g.BS + slot) * D + c0));
         const __nv_bfloat162* p2 = reinterpret_cast<const __nv_bfloat162*>(&rz);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -388,6 +365,7 @@ __global__ void __launch_bounds__(kPrologueThreads)
           v[2 * e] = ff.x; v[2 * e + 1] = ff.y;
         }
         if (gam) {
+          const uint4 rx = __ldg(reinterpret_cast<const uint4*>((kSharded ? a.x[which][sidx] : xin0) + xoff));
           const __nv_bfloat162* x2 = reinterpret_cast<const __nv_bfloat162*>(&rx);
 #pragma unroll
           for (int e = 0; e < 4; ++e) {

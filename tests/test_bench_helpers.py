@@ -71,3 +71,18 @@ def test_selection_locality(bench):
 def test_traffic_scales_with_the_pairs_a_launch_reads(bench):
     assert bench.traffic_per_launch("fwd", "720p", 1000, 10) == bench.DRAM_BYTES_PER_PAIR["fwd"] * 1000
     assert bench.traffic_per_launch("bwd_dkdv", "720p", 1000, 10) == bench.DRAM_BYTES_PER_PAIR["bwd_dkdv"] * 10
+
+
+def test_cpu_baseline_times_forward_and_backward(bench):
+    """The oracle baseline reports the step's rate (forward + 2.5x forward tile FLOPs per query
+    block over the oracle's forward + backward time per block) and both parts on their own;
+    the step rate lies between the two parts' rates scaled by their FLOP shares."""
+    cb = bench.cpu_oracle_sample(WORKLOADS["small"], budget_s=0.5, with_bwd=True)
+    assert cb["kind"] == "oracle" and cb["unit"] == "TFLOP/s" and cb["cores"] >= 1
+    assert cb["value"] > 0 and cb["fwd_tflops"] > 0 and cb["bwd_tflops"] > 0
+    assert "backward of" in cb["sample"]
+    # harmonic combination of the parts (route time makes the step rate a little lower)
+    combined = 3.5 / (1.0 / cb["fwd_tflops"] + 2.5 / cb["bwd_tflops"])
+    assert cb["value"] <= combined * 1.0001
+    fwd_only = bench.cpu_oracle_sample(WORKLOADS["small"], budget_s=0.5, with_bwd=False)
+    assert "bwd_tflops" not in fwd_only and "backward of" not in fwd_only["sample"]
