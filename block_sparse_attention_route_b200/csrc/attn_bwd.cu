@@ -671,8 +671,7 @@ struct DqLayout {
   // q_full, q_empty, kv_full[5], kv_empty[5], s_full, s_loaded, dp_full, ds_full, dq_full, fin
   static constexpr int kNumBars = 2 + 2 * kStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kStageNvOff = kMiscOff + 16;  // int [stages]: valid keys of the tile
-  static constexpr int kAlloc = kStageNvOff + kStages * 4 + 1024;
+  static constexpr int kAlloc = kMiscOff + 16 + 1024;
 };
 
 template <int BS, int D>
@@ -701,9 +700,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   uint64_t* fin_bar = dq_full + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
-  // valid keys of the K / V tile in each ring stage (written by the producer before the tile's
-  // kv_full arrival, read by the MMA thread after waiting on it)
-  volatile int* stage_nv = reinterpret_cast<volatile int*>(smem + L::kStageNvOff);
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   const Geo& g = p.g;
 
@@ -761,12 +757,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           int row;
           if (j < g.NBc) { mk = &tmKc; mv = &tmVc; row = (bhx * g.NBc + j) * BS; }
           else { mk = &tmK; mv = &tmV; row = (bhx * g.NBq + (j - g.NBc)) * BS; }
-          const int nv = key_block_nvalid(g, j);
-          for (int t = 0; t < 2; ++t) {  // K_n then V_n (whole tiles, as in the forward)
+          for (int t = 0; t < 2; ++t) {  // K_n then V_n
             const int stage = seq % S, round = seq / S;
             if (round > 0 && !mbar_wait(&kv_empty[stage], (round - 1) & 1, abort_flag)) { ok = false; break; }
             unsigned char* dst = smem + L::kRingOff + stage * L::kKVBytes;
-            stage_nv[stage] = nv;
             mbar_expect_tx(&kv_full[stage], L::kKVBytes);
 #pragma unroll
             for (int half = 0; half < D / 64; ++half)
@@ -784,13 +778,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   } else if (warp == kBwdMma) {
     // ====================================================== MMA issuer
     if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kTile, BS, 0, 0);   // S, dP: B (K or V tile) K-major
       constexpr uint32_t idQ = idesc_bf16(kTile, D, 0, 1);    // dQ: B (K tile) MN-major
-      // keys of a tile on the tensor cores: the block's valid prefix rounded up to 16 (the
-      // MMA's N step), so a partial block's S, dP (N) and dQ (K) shrink with it
-      auto tile_keys = [&](int seq) -> int {
-        const int nv = stage_nv[seq % S];
-        return nv >= BS ? BS : (nv <= 16 ? 16 : (nv + 15) & ~15);
-      };
       const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
       const uint64_t dkmn = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
       int items = 0, gn = 0;  // non-empty items, global step
@@ -802,9 +791,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tc_fence_after();
         return true;
       };
-      // S(n) = Q K_n^T (A = Q from TMEM); idS carries the step's key count (read right after
-      // the K tile's wait, so the shared-memory load stays off the issue path)
-      auto mma_S = [&](int n, uint32_t idS) {
+      auto mma_S = [&](int n) {  // S(n) = Q K_n^T (A = Q from TMEM)
         const uint64_t kb = dk + (uint64_t)((((seq_base + 2 * n) % S) * L::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -813,7 +800,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_commit(s_full);
       };
-      auto mma_dP = [&](int n, uint32_t idS) {  // dP(n) = dO V_n^T (A = dO from TMEM); then V_n is done
+      auto mma_dP = [&](int n) {  // dP(n) = dO V_n^T (A = dO from TMEM); then V_n is done
         const int seq = seq_base + 2 * n + 1;
         const uint64_t vb = dk + (uint64_t)(((seq % S) * L::kKVBytes) >> 4);
 #pragma unroll
@@ -836,23 +823,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (gn > 0 && !mbar_wait(s_loaded, (gn - 1) & 1, abort_flag)) { ok = false; break; }
         tc_fence_after();
         if (!wait_tile(seq_base) || !wait_tile(seq_base + 1)) { ok = false; break; }
-        int nkeys = tile_keys(seq_base);  // keys of step n on the tensor cores (K_n, V_n alike)
-        {
-          const uint32_t id0 = idesc_bf16(kTile, nkeys, 0, 0);
-          mma_S(0, id0);
-          mma_dP(0, id0);
-        }
+        mma_S(0);
+        mma_dP(0);
         for (int n = 0; n < cnt && ok; ++n, ++gn) {
           const bool more = n + 1 < cnt;
-          int nkeys_next = BS;
-          uint32_t id_next = 0;
           if (more) {  // S(n+1) once S(n) was read out
             if (!mbar_wait(s_loaded, gn & 1, abort_flag)) { ok = false; break; }
             tc_fence_after();
             if (!wait_tile(seq_base + 2 * (n + 1))) { ok = false; break; }
-            nkeys_next = tile_keys(seq_base + 2 * (n + 1));
-            id_next = idesc_bf16(kTile, nkeys_next, 0, 0);
-            mma_S(n + 1, id_next);
+            mma_S(n + 1);
             if (!wait_tile(seq_base + 2 * (n + 1) + 1)) { ok = false; break; }  // V_{n+1}, early
           }
           // dQ += dS(n) K_n (A = dS over the dP columns), then dP(n+1) into those columns
@@ -860,15 +839,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           tc_fence_after();
           const int kseq = seq_base + 2 * n;
           const uint64_t kb = dkmn + (uint64_t)(((kseq % S) * L::kKVBytes) >> 4);
-          const int nk = nkeys / 16;
 #pragma unroll
           for (int kk = 0; kk < BS / 16; ++kk)  // dS of keys [16kk, 16kk+16): group kk/2's columns
-            if (kk < nk)
-              mma_ts(tmem_base + kTdq, tmem_base + kTdp + 32 * (kk >> 1) + 8 * (kk & 1),
-                     kb + (uint64_t)((kk * 2048) >> 4), idQ, (n > 0 || kk > 0) ? 1u : 0u);
+            mma_ts(tmem_base + kTdq, tmem_base + kTdp + 32 * (kk >> 1) + 8 * (kk & 1),
+                   kb + (uint64_t)((kk * 2048) >> 4), idQ, (n > 0 || kk > 0) ? 1u : 0u);
           mma_commit(&kv_empty[kseq % S]);  // K_n done
-          if (more) mma_dP(n + 1, id_next);
-          nkeys = nkeys_next;
+          if (more) mma_dP(n + 1);
         }
         if (!ok) break;
         mma_commit(dq_full);
@@ -931,7 +907,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       const float nd = row < BS ? p.ndelta[qrow] : 0.f;
       const uint64_t nl2x2 = f2pack(nl2, nl2), ndx2 = f2pack(nd, nd), sl2x2 = f2pack(sl2, sl2);
       // key-block indices 32 steps at a time, the next chunk's load in flight; per chunk a
-      // ballot of the partial blocks and each lane's valid-key count (as in the forward)
+      // ballot of the partial blocks and each lane's shape code (as in the forward)
       int jnext = lane < cnt ? item_idx(item, lane) : 0;
       int nreg = BS;
       uint32_t partial = 0;
@@ -942,23 +918,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           nreg = n + lane < cnt ? key_block_nvalid(g, jcur) : BS;
           partial = __ballot_sync(0xffffffffu, nreg < BS);
         }
-        const int nvb = ((partial >> (n & 31)) & 1u) ? __shfl_sync(0xffffffffu, nreg, n & 31) : BS;
-        // A group whose keys all lie past a partial block's valid prefix has nothing to do in
-        // this step (the tensor cores compute only the first roundup16(valid) keys and read
-        // dS of those only); it keeps the waits and arrivals, in order, so no barrier phase
-        // can be overrun.  (Spreading a small block's keys over all four groups, with dS
-        // packed behind a named barrier, measured 2 % slower.)
-        if (cg * KC >= nvb) {
-          bool w_ok = mbar_wait(s_full, gn & 1, abort_flag);
-          w_ok = __all_sync(0xffffffffu, w_ok);
-          if (!w_ok) { ok = false; break; }
-          mbar_arrive(s_loaded);
-          w_ok = mbar_wait(dp_full, gn & 1, abort_flag);
-          w_ok = __all_sync(0xffffffffu, w_ok);
-          if (!w_ok) { ok = false; break; }
-          mbar_arrive(ds_full);
-          continue;
-        }
         // P = exp2(S*sl2 - lse2) for this group's KC keys as soon as S(n) is in
         bool w_ok = mbar_wait(s_full, gn & 1, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
@@ -968,8 +927,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld32_wait(t_s + cg * KC, reinterpret_cast<uint32_t*>(pf));
         tc_fence_before();
         mbar_arrive(s_loaded);  // S may take S(n+1)
-        if (nvb < BS) {  // pad keys (slots >= the valid count): P = 0
-          const int nv = nvb - cg * KC;
+        if ((partial >> (n & 31)) & 1u) {  // pad keys (slots >= the valid count): P = 0
+          const int nv = __shfl_sync(0xffffffffu, nreg, n & 31) - cg * KC;
 #pragma unroll
           for (int c = 0; c < KC; ++c)
             if (c >= nv) pf[c] = -INFINITY;
