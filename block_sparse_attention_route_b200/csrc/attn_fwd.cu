@@ -10,42 +10,28 @@
 // the K/V tiles of idx[b,h,i,0:cnt].  Persistent CTAs (one per SM), items in head-major
 // order so the CTAs running at once share one head's K/V in L2.
 //
-// Warp roles (576 threads; 18 warps put 5 on two SM sub-partitions, so at most 96 registers):
-//   warps 0-15  softmax + epilogue: warp w reads TMEM lanes 32*(w%4).. (query rows) and owns
-//               the key-column group w/4 (BS/4 keys) of every S tile and the O-column group
-//               w/4 (D/4 columns) of the output
-//   warp 16     TMA producer (one thread)
-//   warp 17     MMA issuer (one thread); owns the TMEM allocation
-// TMEM columns: S0 [0,128), S1 [128,256), O [256,256+D), Q slots [256+D, 256+2D) (two of
-// D/2 columns: bf16 pairs).  Q is the A operand of S = Q K^T straight from TMEM, so the
-// tensor cores read only K from shared memory for S (a shared-memory-bandwidth saving: an SS
-// MMA pair of 128x16 bf16 tiles reads 8 KB per 64 clocks, the whole 128 B/clock).  The
-// softmax warps copy each item's Q from its staging tile into a Q slot one item ahead.
-// S is double buffered: while the
-// softmax turns S(n) into P(n) (bf16, written over the first BS/2 columns of its buffer),
-// the tensor cores already compute S(n+1).  MMA order: S(0), S(1), then per step PV(n) and
-// S(n+2) into the buffer P(n) came from (tcgen05 MMAs of one thread run in issue order, so
-// S(n+2) is written after PV(n) has read P(n)).
+// Two items per CTA in ping-pong: slot 0 takes the CTA's even-numbered items, slot 1 its
+// odd ones, and the single MMA thread alternates between them, so the tensor cores compute
+// one slot's S and P.V while the other slot's softmax runs.  Per slot: S = Q K^T into its own
+// 128 TMEM columns (P, bf16, is written back over them), O in another 128; both slots fill
+// the 512 columns.  S reads Q and K from shared memory (Q stays staged for the whole item).
 //
-// The four column groups of a row (warps q, q+4, q+8, q+12: the same TMEM lanes) exchange
-// partial row maxima through shared memory behind a named barrier of those 128 threads (one
-// per step; the exchange slots alternate with the step parity) and keep partial row sums,
-// combined once per item.  The barrier also orders every group's read of S(n) before any
-// group overwrites it with P(n).  The four row quarters run independently: P-ready is one
-// mbarrier per S buffer, so the phases of one barrier are two steps apart and a quarter can
-// never arrive for step n+2 before the MMA thread has consumed step n (S(n+2) is issued only
-// after PV(n)).  Online softmax in the exp2 domain with lazy
-// rescaling: the running max is raised only when a row's max grows by more than 8 (log2
-// units), so O is rarely touched (and then only after the previous PV has completed, which
-// the pv_done barrier tells); the final O / l and LSE are exact either way.
+// Warp roles (320 threads, so a thread may hold up to ~200 registers):
+//   warps 0-3  slot 0 softmax + epilogue, warps 4-7 slot 1: warp w owns query rows
+//              32*(w%4)..+31 (its TMEM lane quarter) and a thread owns a whole row, so the
+//              row max needs no exchange between threads
+//   warp 8     TMA producer (one thread): K / V tiles in the MMA thread's order
+//   warp 9     MMA issuer (one thread); owns the TMEM allocation
+// MMA order (per slot): S(0) | PV(0), S(1) | PV(1), S(2) | ... | PV(cnt-1), alternating
+// slots group by group.  S(n+1) is written over P(n) after PV(n) has read it (tcgen05 MMAs
+// of one thread run in issue order).  A slot's S-ready commit follows its previous PV in
+// issue order, so when the softmax sees S(n) complete, O already holds P(0..n-1) V: the lazy
+// rescale of O needs no further wait.  The softmax warps of a slot load the slot's next Q as
+// soon as the current item's last S is complete (its last reader).
 //
-// Shared memory: two Q staging buffers and a ring of K/V tiles consumed strictly in the order
-// the MMA thread uses them; the producer walks the identical schedule.  Q of the j-th
-// non-empty item of a CTA is staged in buffer j & 1 and copied to TMEM slot j & 1: the
-// producer loads Q(j+1) before the K/V tiles of item j, the softmax warps copy it during step
-// 0 of item j (its slot's previous Q, item j-1's, is no longer read: every S of item j-1
-// completed before S(0) of item j) and free the staging buffer, and the MMA thread waits for
-// the copy before the first S of item j+1.
+// Online softmax in the exp2 domain with lazy rescaling: the running max is raised only when
+// a row's max grows by more than 8 (log2 units), so O is rarely touched; the final O / l and
+// LSE are exact either way.
 #include "common.cuh"
 
 namespace bsa {
@@ -60,26 +46,23 @@ struct FwdParams {
   float* lse;
 };
 
-constexpr int kFwdThreads = 576;
-constexpr int kSoftmaxThreads = 512;
-constexpr int kProducerWarp = 16, kMmaWarp = 17;
+constexpr int kFwdThreads = 320;
+constexpr int kSlotThreads = 128;  // softmax threads of one slot
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr int kFwdStages = 5;
-constexpr int kQBufs = 1;  // Q staging buffers (Q leaves for TMEM at step 0 of the item before)
 constexpr int kTileM = 128;
 
 template <int BS, int D>
 struct FwdLayout {
   static constexpr int kQBytes = kTileM * D * 2;
   static constexpr int kKVBytes = BS * D * 2;
-  static constexpr int kQOff = 0;
-  static constexpr int kRingOff = kQBufs * kQBytes;
+  static constexpr int kQOff = 0;                       // Q of slot s at kQOff + s * kQBytes
+  static constexpr int kRingOff = 2 * kQBytes;
   static constexpr int kBarOff = kRingOff + kFwdStages * kKVBytes;
-  // q_full[2] q_empty[2] qt_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] pv_done o_full fin
-  static constexpr int kNumBars = 6 + 2 * kFwdStages + 2 + 2 + 3;
+  // q_full[2] kv_full[S] kv_empty[S] s_full[2] p_full[2] o_full[2] fin
+  static constexpr int kNumBars = 2 + 2 * kFwdStages + 2 + 2 + 2 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kXchOff = kMiscOff + 16;               // float [2 parity][4 groups][128]
-  static constexpr int kSumOff = kXchOff + 2 * 4 * 128 * 4;   // float [4 groups][128]
-  static constexpr int kBytes = kSumOff + 4 * 128 * 4;
+  static constexpr int kBytes = kMiscOff + 16;
   static constexpr int kAlloc = kBytes + 1024;  // slack to align the base to 1024
 };
 
@@ -101,6 +84,11 @@ __device__ __forceinline__ int load_idx(const FwdParams& p, int item, int n) {
   return j;
 }
 
+// The k-th item of slot s of this CTA: items blockIdx.x + (2k + s) * gridDim.x.
+__device__ __forceinline__ int slot_item(int s, int k) {
+  return (int)blockIdx.x + (2 * k + s) * (int)gridDim.x;
+}
+
 template <int BS, int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
     bsa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -108,20 +96,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                    const __grid_constant__ CUtensorMap tmVc, const FwdParams p) {
   using L = FwdLayout<BS, D>;
   constexpr int S = kFwdStages;
+  static_assert(BS <= 128 && D <= 128, "one slot's S and O fit 128 TMEM columns each");
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBarOff);
-  uint64_t* q_full = bars;            // [2] Q staged (TMA)
-  uint64_t* q_empty = bars + 2;       // [2] staging buffer copied out (kSoftmaxThreads arrivals)
-  uint64_t* qt_full = bars + 4;       // [2] Q in its TMEM slot (kSoftmaxThreads arrivals)
-  uint64_t* kv_full = bars + 6;       // [S]
+  uint64_t* q_full = bars;            // [2] Q of the slot's next item staged (TMA)
+  uint64_t* kv_full = bars + 2;       // [S]
   uint64_t* kv_empty = kv_full + S;   // [S]
-  uint64_t* s_full = kv_empty + S;    // [2] S(n) in buffer n & 1
-  uint64_t* p_full = s_full + 2;      // [2] P(n) written into buffer n & 1 (kSoftmaxThreads arrivals)
-  uint64_t* pv_done = p_full + 2;     // PV(n) complete
-  uint64_t* o_full = pv_done + 1;     // O of the item complete
-  uint64_t* fin_bar = o_full + 1;
+  uint64_t* s_full = kv_empty + S;    // [2] S(n) of the slot in TMEM
+  uint64_t* p_full = s_full + 2;      // [2] P(n) of the slot in TMEM (kSlotThreads arrivals)
+  uint64_t* o_full = p_full + 2;      // [2] O of the slot's item complete
+  uint64_t* fin_bar = o_full + 2;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -129,19 +115,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   const Geo& g = p.g;
 
   if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&q_full[i], 1);
-      mbar_init(&q_empty[i], kSoftmaxThreads);
-      mbar_init(&qt_full[i], kSoftmaxThreads);
-      mbar_init(&s_full[i], 1);
-      mbar_init(&p_full[i], kSoftmaxThreads);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&q_full[s], 1);
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], kSlotThreads);
+      mbar_init(&o_full[s], 1);
     }
     for (int s = 0; s < S; ++s) {
       mbar_init(&kv_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(pv_done, 1);
-    mbar_init(o_full, 1);
     mbar_init(fin_bar, 1);
     *abort_flag = 0;
     mbar_fence_init();
@@ -159,23 +142,29 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const uint32_t t_o0 = tmem_base + 256;
-  const uint32_t t_q0 = tmem_base + 256 + D;  // Q slot b at t_q0 + b * D / 2
-  // next item with a non-empty selection at or after `it` in this CTA's sequence
-  auto next_item = [&](int it) {
-    while (it < p.n_items && load_cnt(p, it) == 0) it += gridDim.x;
-    return it;
+  // TMEM columns of slot s: S at 256 s, O at 256 s + 128
+  auto t_s_col = [&](int s) -> uint32_t { return tmem_base + 256u * s; };
+  auto t_o_col = [&](int s) -> uint32_t { return tmem_base + 256u * s + 128u; };
+  // next item of slot s with a non-empty selection, from its k-th item on (k advanced)
+  auto next_slot_item = [&](int s, int& k, int& cnt) -> int {
+    for (;;) {
+      const int it = slot_item(s, k);
+      if (it >= p.n_items) return -1;
+      cnt = load_cnt(p, it);
+      if (cnt > 0) return it;
+      ++k;
+    }
   };
 
   if (warp == kProducerWarp) {
     // ================================================================ TMA producer
-    // Load order = MMA consumption order: per item K(0), K(1), then per step n: V(n),
-    // K(n+2); Q of the next non-empty item is staged before the current item's tiles.
+    // Walks the MMA thread's turn sequence (slot 0, slot 1, slot 0, ... skipping a finished
+    // slot): a slot's first turn of an item loads K(0); its turn n loads V(n) and, unless n is
+    // the item's last step, K(n+1).  Key-block indices are loaded a step ahead.
     if (lane == 0) {
-      int seq = 0, items = 0;
+      int seq = 0;
       bool ok = true;
       unsigned char* ring = smem + L::kRingOff;
-      // K or V tile of key block j of head row bhx into the next ring stage
       auto kv_tile = [&](int bhx, int j, bool is_v) -> bool {
         const int stage = seq % S, round = seq / S;
         if (round > 0 && !mbar_wait(&kv_empty[stage], (round - 1) & 1, abort_flag)) return false;
@@ -191,49 +180,41 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         ++seq;
         return true;
       };
-      // Q of the `items`-th non-empty item into staging buffer items % kQBufs (free once the
-      // softmax warps copied out the Q kQBufs items back)
-      auto q_tile = [&](int item) -> bool {
-        const int qb = items % kQBufs;
-        if (items >= kQBufs &&
-            !mbar_wait(&q_empty[qb], ((items / kQBufs) - 1) & 1, abort_flag)) return false;
-        mbar_expect_tx(&q_full[qb], L::kQBytes);
-#pragma unroll
-        for (int half = 0; half < D / 64; ++half)
-          tma_load_2d(smem + L::kQOff + qb * L::kQBytes + half * kTileM * 128, &tmQ, half * 64,
-                      item * BS, &q_full[qb]);
-        ++items;
-        return true;
-      };
-      int item = next_item(blockIdx.x);
-      if (item < p.n_items) ok = q_tile(item);
-      while (item < p.n_items && ok) {
-        const int cnt = load_cnt(p, item);
-        const int nxt = next_item(item + gridDim.x);
-        if (nxt < p.n_items) ok = q_tile(nxt);
-        // Key-block indices of steps n, n+1, n+2 ride in registers and the index of step n+3
-        // is loaded one step ahead, so no global-load latency sits in the chain of waits and
-        // TMA issues (each index is loaded once, for its K tile, and reused for its V tile).
-        const int bhx = item / g.NBq;
-        int j0 = load_idx(p, item, 0), j1 = cnt > 1 ? load_idx(p, item, 1) : 0;
-        int j2 = cnt > 2 ? load_idx(p, item, 2) : 0;
-        ok = ok && kv_tile(bhx, j0, false) && (cnt < 2 || kv_tile(bhx, j1, false));
-        for (int n = 0; n < cnt && ok; ++n) {
-          const int j3 = n + 3 < cnt ? load_idx(p, item, n + 3) : 0;  // used next step
-          ok = kv_tile(bhx, j0, true);                                 // V(n)
-          if (ok && n + 2 < cnt) ok = kv_tile(bhx, j2, false);         // K(n+2)
-          j0 = j1; j1 = j2; j2 = j3;
+      // the two slots' states in registers: `a` takes this turn, then the two swap when the
+      // other slot still has work (the turn order the MMA thread follows too)
+      struct Slot { int s, k, item, cnt, n, jcur, jnext; };  // jcur / jnext: blocks of V(n), K(n+1)
+      Slot a{0, 0, -1, 0, -1, 0, 0}, b{1, 0, -1, 0, -1, 0, 0};
+      a.item = next_slot_item(0, a.k, a.cnt);
+      b.item = next_slot_item(1, b.k, b.cnt);
+      while (ok && (a.item >= 0 || b.item >= 0)) {
+        if (a.item < 0) { const Slot t = a; a = b; b = t; }
+        const int it = a.item, bhx = it / g.NBq;
+        if (a.n < 0) {  // first turn of the item: K(0)
+          a.jcur = load_idx(p, it, 0);
+          a.jnext = a.cnt > 1 ? load_idx(p, it, 1) : 0;
+          ok = kv_tile(bhx, a.jcur, false);
+          a.n = 0;
+        } else {  // turn n: V(n), then K(n+1)
+          const int nn = a.n;
+          const int jn2 = nn + 2 < a.cnt ? load_idx(p, it, nn + 2) : 0;  // a step ahead
+          ok = kv_tile(bhx, a.jcur, true);
+          if (ok && nn + 1 < a.cnt) ok = kv_tile(bhx, a.jnext, false);
+          a.jcur = a.jnext;
+          a.jnext = jn2;
+          if (nn + 1 < a.cnt) {
+            a.n = nn + 1;
+          } else {  // item done: the slot's next item
+            ++a.k;
+            a.item = next_slot_item(a.s, a.k, a.cnt);
+            a.n = -1;
+          }
         }
-        item = nxt;
+        if (b.item >= 0) { const Slot t = a; a = b; b = t; }
       }
       // drain: every issued TMA load must land before the CTA may exit
       for (int st = 0; st < S; ++st) {
         const int loads = seq / S + (st < seq % S ? 1 : 0);
         if (loads > 0) mbar_wait_drain(&kv_full[st], (loads - 1) & 1);
-      }
-      for (int b = 0; b < kQBufs; ++b) {
-        const int loads = items / kQBufs + (b < items % kQBufs ? 1 : 0);
-        if (loads > 0) mbar_wait_drain(&q_full[b], (loads - 1) & 1);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -241,80 +222,74 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kTileM, BS, 0, 0);
       constexpr uint32_t idPV = idesc_bf16(kTileM, D, 0, 1);
-      const uint64_t dk = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
-      const uint64_t dv = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
-      int seq = 0, items = 0, gs = 0, gp = 0;  // ring position, items, S issued, P consumed
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(smem + L::kQOff), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(smem + L::kRingOff), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(smem + L::kRingOff), BS * 128, 1024);
+      int seq = 0;
       bool ok = true;
       auto wait_tile = [&]() -> int {
         const int stage = seq % S;
         if (!mbar_wait(&kv_full[stage], (seq / S) & 1, abort_flag)) return -1;
-        tc_fence_after();
+        ++seq;
         return stage;
       };
-      // S(gs) = Q K^T into buffer gs & 1: A = Q from TMEM slot a_q (K16 slice kk at column
-      // 8 kk), B = the K tile in ring stage `stage`
-      auto mma_S = [&](uint32_t a_q, int stage) {
-        const uint64_t kb = dk + (uint64_t)((stage * L::kKVBytes) >> 4);
-        const uint32_t d_s = tmem_base + (gs & 1) * 128;
+      // S of slot s = Q_s K^T: A = Q (128 rows, K-major), B = the K tile in `stage`
+      auto mma_S = [&](int s, int stage) {
+        const uint64_t qd = dq0 + (uint64_t)((s * L::kQBytes) >> 4);
+        const uint64_t kd = dk0 + (uint64_t)((stage * L::kKVBytes) >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t offq = ((kk / 4) * (kTileM * 128) + (kk % 4) * 32) >> 4;
           const uint32_t offk = ((kk / 4) * (BS * 128) + (kk % 4) * 32) >> 4;
-          mma_ts(d_s, a_q + kk * 8, kb + offk, idS, kk > 0 ? 1u : 0u);
+          mma_ss(t_s_col(s), qd + offq, kd + offk, idS, kk > 0 ? 1u : 0u);
         }
       };
-      // Every wait comes before the MMAs it guards, so each step issues one uninterrupted
-      // group (PV(n) then S(n+2): 2 * D/16 or BS/16 + D/16 MMAs) followed by its commits;
-      // a wait or commit between MMAs would let the tensor pipe drain.
-      int cnt_next = (int)blockIdx.x < p.n_items ? load_cnt(p, blockIdx.x) : 0;
-      for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-        const int cnt = cnt_next;
-        cnt_next = item + (int)gridDim.x < p.n_items ? load_cnt(p, item + gridDim.x) : 0;
-        if (cnt == 0) continue;
-        const int qb = items & 1;
-        if (!mbar_wait(&qt_full[qb], (items >> 1) & 1, abort_flag)) { ok = false; break; }
-        ++items;
-        const int k0 = wait_tile();
-        ++seq;
-        const int k1 = (k0 >= 0 && cnt >= 2) ? wait_tile() : -1;
-        if (cnt >= 2) ++seq;
-        if (k0 < 0 || (cnt >= 2 && k1 < 0)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t dq = t_q0 + qb * (D / 2);
-        const int gs0 = gs;
-        mma_S(dq, k0);
-        ++gs;
-        if (cnt >= 2) { mma_S(dq, k1); ++gs; }
-        mma_commit(&s_full[gs0 & 1]);
-        if (cnt >= 2) mma_commit(&s_full[(gs0 + 1) & 1]);
-        mma_commit(&kv_empty[k0]);
-        if (cnt >= 2) mma_commit(&kv_empty[k1]);
-        for (int n = 0; n < cnt && ok; ++n) {
-          const int sv = wait_tile();
-          ++seq;
-          const bool more = n + 2 < cnt;
-          const int sk = (sv >= 0 && more) ? wait_tile() : -1;
-          if (more) ++seq;
-          if (sv < 0 || (more && sk < 0)) { ok = false; break; }
-          // O += P(n) V(n): A = P from TMEM (buffer gp & 1), B = V (MN-major)
-          if (!mbar_wait(&p_full[gp & 1], (gp >> 1) & 1, abort_flag)) { ok = false; break; }
+      // the two slots' states in registers, swapped after each turn as in the producer
+      struct Slot { int s, k, item, cnt, n, qc, pc; };  // qc / pc: Q loads, P(n) consumed
+      Slot a{0, 0, -1, 0, -1, 0, 0}, b{1, 0, -1, 0, -1, 0, 0};
+      a.item = next_slot_item(0, a.k, a.cnt);
+      b.item = next_slot_item(1, b.k, b.cnt);
+      while (ok && (a.item >= 0 || b.item >= 0)) {
+        if (a.item < 0) { const Slot t = a; a = b; b = t; }
+        const int s = a.s;
+        if (a.n < 0) {  // S(0) once the slot's Q has landed
+          const int sk = wait_tile();
+          if (sk < 0 || !mbar_wait(&q_full[s], a.qc & 1, abort_flag)) { ok = false; break; }
+          ++a.qc;
           tc_fence_after();
-          const uint64_t vb = dv + (uint64_t)((sv * L::kKVBytes) >> 4);
-          const uint32_t a_p = tmem_base + (gp & 1) * 128;
+          mma_S(s, sk);
+          mma_commit(&s_full[s]);
+          mma_commit(&kv_empty[sk]);
+          a.n = 0;
+        } else {
+          // turn n: O += P(n) V(n) (A = P from TMEM), then S(n+1) over P(n)
+          const int nn = a.n;
+          const bool more = nn + 1 < a.cnt;
+          const int sv = wait_tile();
+          const int sk = (sv >= 0 && more) ? wait_tile() : -1;
+          if (sv < 0 || (more && sk < 0)) { ok = false; break; }
+          if (!mbar_wait(&p_full[s], a.pc & 1, abort_flag)) { ok = false; break; }
+          ++a.pc;
+          tc_fence_after();
+          const uint64_t vd = dv0 + (uint64_t)((sv * L::kKVBytes) >> 4);
 #pragma unroll
           for (int kk = 0; kk < BS / 16; ++kk)
-            mma_ts(t_o0, a_p + kk * 8, vb + (uint64_t)((kk * 2048) >> 4), idPV,
-                   (n > 0 || kk > 0) ? 1u : 0u);
-          if (more) {  // S(n+2) into the buffer P(n) came from (read above, in issue order)
-            mma_S(dq, sk);
-            mma_commit(&s_full[gs & 1]);
-            ++gs;
+            mma_ts(t_o_col(s), t_s_col(s) + kk * 8, vd + (uint64_t)((kk * 2048) >> 4), idPV,
+                   (nn > 0 || kk > 0) ? 1u : 0u);
+          if (more) {
+            mma_S(s, sk);
+            mma_commit(&s_full[s]);
+            mma_commit(&kv_empty[sk]);
+            a.n = nn + 1;
+          } else {
+            mma_commit(&o_full[s]);
+            ++a.k;
+            a.item = next_slot_item(s, a.k, a.cnt);
+            a.n = -1;
           }
-          mma_commit(pv_done);
-          if (n == cnt - 1) mma_commit(o_full);
           mma_commit(&kv_empty[sv]);
-          if (more) mma_commit(&kv_empty[sk]);
-          ++gp;
         }
+        if (b.item >= 0) { const Slot t = a; a = b; b = t; }
       }
       // all MMAs issued by this thread must finish before TMEM is released
       mma_commit(fin_bar);
@@ -322,150 +297,127 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     }
   } else {
     // ================================================================ softmax + epilogue
-    constexpr int KC = BS / 4;  // keys (S columns) per thread
-    constexpr int OC = D / 4;   // O columns per thread
-    const int cg = warp / 4, quarter = warp & 3;
+    const int s = warp / 4, quarter = warp & 3;
     const int row = 32 * quarter + lane;
     const uint32_t t_lane = (uint32_t)(32 * quarter) << 16;
-    const uint32_t t_oc = t_o0 + t_lane + cg * OC;
-    float* xch = reinterpret_cast<float*>(smem + L::kXchOff);
-    float* xsum = reinterpret_cast<float*>(smem + L::kSumOff);
+    const uint32_t t_s = t_s_col(s) + t_lane, t_o = t_o_col(s) + t_lane;
     const float sl2 = g.scale * 1.4426950408889634f;
-    int gstep = 0, ocons = 0;  // global step (= S buffer use / P / PV index)
+    const bool leader = quarter == 0 && lane == 0;  // issues the slot's Q loads
+    unsigned char* qbuf = smem + L::kQOff + s * L::kQBytes;
+    int qloads = 0, gs = 0, oc = 0;  // Q loads issued, S steps consumed, items finished
     bool ok = true;
-    // This thread's part of Q (row `row`, dims [cg*D/4, (cg+1)*D/4)) of the jj-th non-empty
-    // item: from the 128-byte-swizzled staging tile into TMEM slot jj & 1 as bf16 pairs.
-    auto copy_q = [&](int jj) -> bool {
-      const int qb = jj % kQBufs, slot = jj & 1;
-      bool w_ok = mbar_wait(&q_full[qb], (jj / kQBufs) & 1, abort_flag);
-      w_ok = __all_sync(0xffffffffu, w_ok);
-      if (!w_ok) return false;
-      constexpr int DC = D / 4;
-      const int d0 = cg * DC, half = d0 / 64, c0 = (d0 % 64) / 8;
-      const unsigned char* tile = smem + L::kQOff + qb * L::kQBytes + half * (kTileM * 128) + row * 128;
-      uint32_t w[DC / 2];
+    auto load_q = [&](int item) {
+      mbar_expect_tx(&q_full[s], L::kQBytes);
 #pragma unroll
-      for (int c = 0; c < DC / 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(tile + (((c0 + c) ^ (row & 7)) << 4));
-        w[4 * c] = v.x; w[4 * c + 1] = v.y; w[4 * c + 2] = v.z; w[4 * c + 3] = v.w;
-      }
-      const uint32_t dst = t_q0 + t_lane + slot * (D / 2) + cg * (DC / 2);
-      if constexpr (DC == 32) tmem_st16(dst, w);
-      else tmem_st8(dst, w);
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&qt_full[slot]);
-      mbar_arrive(&q_empty[qb]);
-      return true;
+      for (int half = 0; half < D / 64; ++half)
+        tma_load_2d(qbuf + half * kTileM * 128, &tmQ, half * 64, item * BS, &q_full[s]);
     };
-    int jq = -1;  // non-empty items started
-    if (next_item(blockIdx.x) < p.n_items) ok = copy_q(0);
-    int cnt_next = (int)blockIdx.x < p.n_items ? load_cnt(p, blockIdx.x) : 0;
-    for (int item = blockIdx.x; item < p.n_items && ok; item += gridDim.x) {
-      const int cnt = cnt_next;  // the next item's count is fetched one item ahead
-      cnt_next = item + (int)gridDim.x < p.n_items ? load_cnt(p, item + gridDim.x) : 0;
-      const int i = item % g.NBq;
-      // this row's query slot (rows >= BS belong to the tile's padding and are discarded)
+    {
+      int k0 = 0, c0 = 0;
+      const int first = next_slot_item(s, k0, c0);
+      if (leader && first >= 0) { load_q(first); ++qloads; }
+    }
+    // items of this slot, empty ones included (their O rows are zeros, LSE -inf)
+    for (int kk = 0; ok; ++kk) {
+      const int it = slot_item(s, kk);
+      if (it >= p.n_items) break;
+      const int c = load_cnt(p, it);
+      const int i = it % g.NBq;
       const bool qvalid = row < BS && row < query_block_nvalid(g, i);
-      float* lse_row = p.lse + (size_t)item * BS;
-      __nv_bfloat16* o_row = p.o + ((size_t)item * BS + row) * D + cg * OC;
-      if (cnt == 0) {
+      float* lse_row = p.lse + (size_t)it * BS;
+      __nv_bfloat16* o_row = p.o + ((size_t)it * BS + row) * D;
+      if (c == 0) {
         if (row < BS) {
           const uint4 z = make_uint4(0, 0, 0, 0);
 #pragma unroll
-          for (int c = 0; c < OC / 8; ++c) reinterpret_cast<uint4*>(o_row)[c] = z;
-          if (cg == 0) lse_row[row] = -INFINITY;
+          for (int e = 0; e < D / 8; ++e) reinterpret_cast<uint4*>(o_row)[e] = z;
+          lse_row[row] = -INFINITY;
         }
         continue;
       }
-      ++jq;
-      const bool has_next = next_item(item + gridDim.x) < p.n_items;
+      // the slot's next non-empty item (its Q is loaded once this item's last S is done)
+      int kn = kk + 1, cn = 0;
+      const int nxt = next_slot_item(s, kn, cn);
       float m = -INFINITY, l = 0.f;
-      // Key-block indices come 32 steps at a time (lane e holds step n0 + e), the next chunk's
-      // load in flight while the current one runs; per chunk a ballot marks the steps whose
-      // block is partial and each lane keeps its step's shape code, so no global load or
-      // index arithmetic sits between a step's S and its P.
-      int jnext = lane < cnt ? load_idx(p, item, lane) : 0;
+      // key-block valid counts 32 steps at a time (lane e holds step n0 + e), the next chunk's
+      // index load in flight
+      int jnext = lane < c ? load_idx(p, it, lane) : 0;
       int nreg = BS;
       uint32_t partial = 0;
-      for (int n = 0; n < cnt; ++n, ++gstep) {
-        const int b = gstep & 1;
+      for (int n = 0; n < c; ++n, ++gs) {
         if ((n & 31) == 0) {
           const int jcur = jnext;
-          jnext = n + 32 + lane < cnt ? load_idx(p, item, n + 32 + lane) : 0;
-          nreg = n + lane < cnt ? key_block_nvalid(g, jcur) : BS;
+          jnext = n + 32 + lane < c ? load_idx(p, it, n + 32 + lane) : 0;
+          nreg = n + lane < c ? key_block_nvalid(g, jcur) : BS;
           partial = __ballot_sync(0xffffffffu, nreg < BS);
         }
-        bool w_ok = mbar_wait(&s_full[b], (gstep >> 1) & 1, abort_flag);
+        bool w_ok = mbar_wait(&s_full[s], gs & 1, abort_flag);
         w_ok = __all_sync(0xffffffffu, w_ok);
         if (!w_ok) { ok = false; break; }
         tc_fence_after();
-        const uint32_t t_s = tmem_base + t_lane + b * 128;
-        float s[KC];
+        // S(c-1) complete: Q of this item has no reader left; stage the next item's Q
+        if (n == c - 1 && leader && nxt >= 0) { load_q(nxt); ++qloads; }
+        // the row of S (BS fp32 values) in registers; pad keys of a partial block (its slots
+        // >= its valid count) count as -inf
+        float sv[BS];
         {
-          uint32_t* sr = reinterpret_cast<uint32_t*>(s);
-          if constexpr (KC == 32) tmem_ld32_wait(t_s + cg * KC, sr);
-          else tmem_ld8_wait(t_s + cg * KC, sr);
+          uint32_t* sr = reinterpret_cast<uint32_t*>(sv);
+          if constexpr (BS == 128) tmem_ld128_wait(t_s, sr);
+          else tmem_ld32_wait(t_s, sr);
         }
-        // pad keys of a partial block get -inf (mask from the per-shape table)
         if ((partial >> (n & 31)) & 1u) {
-          const int nv = __shfl_sync(0xffffffffu, nreg, n & 31) - cg * KC;
+          const int nv = __shfl_sync(0xffffffffu, nreg, n & 31);
 #pragma unroll
-          for (int c = 0; c < KC; ++c)
-            if (c >= nv) s[c] = -INFINITY;
+          for (int e = 0; e < BS; ++e)
+            if (e >= nv) sv[e] = -INFINITY;
         }
         float mx;
-        {
-          float a0 = s[0], a1 = s[1];
+        {  // four independent max3 chains over the row (BS is a multiple of 8)
+          float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-          for (int c = 2; c + 4 <= KC; c += 4) {
-            a0 = max3f(a0, s[c], s[c + 1]);
-            a1 = max3f(a1, s[c + 2], s[c + 3]);
+          for (int e = 0; e < BS; e += 8) {
+            a0 = max3f(a0, sv[e], sv[e + 1]);
+            a1 = max3f(a1, sv[e + 2], sv[e + 3]);
+            a2 = max3f(a2, sv[e + 4], sv[e + 5]);
+            a3 = max3f(a3, sv[e + 6], sv[e + 7]);
           }
-          mx = max3f(a0, a1, fmaxf(s[KC - 2], s[KC - 1]));
+          mx = fmaxf(fmaxf(a0, a1), fmaxf(a2, a3)) * sl2;
         }
-        // exchange the four partial row maxima; the slots alternate with the step parity
-        float* xs = xch + b * 512;
-        xs[cg * 128 + row] = mx;
-        named_bar_sync(1 + quarter, kSoftmaxThreads / 4);
-        mx = fmaxf(fmaxf(xs[row], xs[128 + row]), fmaxf(xs[256 + row], xs[384 + row])) * sl2;
-        // lazy rescale: raise the running max only when it grew by more than 8 (log2 units);
-        // all four threads of a row take the same decision.  tcgen05.ld/st are warp-collective,
-        // so a warp rescales together (alpha = 1 for rows that keep their max), after PV(n-1).
+        // lazy rescale: raise the running max only when it grew by more than 8 (log2 units).
+        // O holds P(0..n-1) V already (S(n)'s commit followed PV(n-1)); tcgen05.ld/st are
+        // warp-collective, so a warp rescales together (alpha = 1 for rows that keep their max)
         const float m_new = (n == 0 || mx > m + 8.0f) ? mx : m;
         const bool resc = n > 0 && m_new != m;
         if (__any_sync(0xffffffffu, resc)) {
-          bool pv_ok = mbar_wait(pv_done, (gstep - 1) & 1, abort_flag);
-          pv_ok = __all_sync(0xffffffffu, pv_ok);
-          if (!pv_ok) { ok = false; break; }
-          tc_fence_after();
           const float alpha = resc ? fast_exp2(m - m_new) : 1.0f;
           l *= alpha;
-          uint32_t r[OC];
-          if constexpr (OC == 32) tmem_ld32_wait(t_oc, r);
-          else tmem_ld16_wait(t_oc, r);
 #pragma unroll
-          for (int e = 0; e < OC; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          if constexpr (OC == 32) tmem_st32(t_oc, r);
-          else tmem_st16(t_oc, r);
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32_wait(t_o + c0, r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+            tmem_st32(t_o + c0, r);
+          }
           tmem_wait_st();
         }
         m = m_new;
-        // P = exp2(s * scale * log2e - m) as bf16 pairs into columns [cg*KC/2, ..) of this S
-        // buffer (already read by every group: the exchange barrier above)
+        // P = exp2(s * scale * log2e - m) as bf16 pairs over the first BS/2 columns of S
         const uint64_t sl2x2 = f2pack(sl2, sl2), nmx2 = f2pack(-m, -m);
         uint64_t sum2 = f2pack(0.f, 0.f);
-        uint32_t pk[KC / 2];
 #pragma unroll
-        for (int e = 0; e < KC / 2; ++e) {
-          float x0, x1;
-          f2unpack(fma2(f2pack(s[2 * e], s[2 * e + 1]), sl2x2, nmx2), x0, x1);
-          const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
-          sum2 = add2(sum2, f2pack(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
+        for (int c0 = 0; c0 < BS; c0 += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float x0, x1;
+            f2unpack(fma2(f2pack(sv[c0 + 2 * e], sv[c0 + 2 * e + 1]), sl2x2, nmx2), x0, x1);
+            const float p0 = fast_exp2(x0), p1 = fast_exp2(x1);
+            sum2 = add2(sum2, f2pack(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tmem_st16(t_s + c0 / 2, pk);
         }
-        if constexpr (KC == 32) tmem_st16(t_s + cg * (KC / 2), pk);
-        else tmem_st4(t_s + cg * (KC / 2), pk);
         {
           float l0, l1;
           f2unpack(sum2, l0, l1);
@@ -473,36 +425,35 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(&p_full[b]);
-        // the next item's Q into the other slot (every S of the previous item, the slot's
-        // last reader, completed before S(0) of this one)
-        if (n == 0 && has_next && !copy_q(jq + 1)) { ok = false; break; }
+        mbar_arrive(&p_full[s]);
       }
       if (!ok) break;
-      // combine the four partial row sums
-      xsum[cg * 128 + row] = l;
-      named_bar_sync(1 + quarter, kSoftmaxThreads / 4);
-      l = (xsum[row] + xsum[128 + row]) + (xsum[256 + row] + xsum[384 + row]);
-      bool w_ok = mbar_wait(o_full, ocons & 1, abort_flag);
+      // epilogue: O / l and LSE of this row, once the item's last PV has completed
+      bool w_ok = mbar_wait(&o_full[s], oc & 1, abort_flag);
       w_ok = __all_sync(0xffffffffu, w_ok);
       if (!w_ok) { ok = false; break; }
-      ++ocons;
+      ++oc;
       tc_fence_after();
       const float inv_l = qvalid ? 1.0f / l : 0.f;
-      uint32_t r[OC];
-      if constexpr (OC == 32) tmem_ld32_wait(t_oc, r);
-      else tmem_ld16_wait(t_oc, r);
-      if (row < BS) {
-        uint4 v[OC / 8];
-        uint32_t* v32 = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
-        for (int e = 0; e < OC / 2; ++e)
-          v32[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32_wait(t_o + c0, r);
+        if (row < BS) {
+          uint4 v[4];
+          uint32_t* v32 = reinterpret_cast<uint32_t*>(v);
 #pragma unroll
-        for (int e = 0; e < OC / 8; ++e) reinterpret_cast<uint4*>(o_row)[e] = v[e];
-        if (cg == 0) lse_row[row] = qvalid ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+          for (int e = 0; e < 16; ++e)
+            v32[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv_l, __uint_as_float(r[2 * e + 1]) * inv_l);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) reinterpret_cast<uint4*>(o_row + c0)[e] = v[e];
+        }
       }
+      if (row < BS) lse_row[row] = qvalid ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+      tc_fence_before();
     }
+    // every Q load this slot issued must land before the CTA may exit
+    if (leader && qloads > 0) mbar_wait_drain(&q_full[s], (qloads - 1) & 1);
   }
 
   tc_fence_before();
@@ -513,7 +464,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
 cudaError_t launch_fwd(const CUtensorMap* maps, const FwdParams& p, int n_sm, cudaStream_t s) {
   const int bs = p.g.BS, d = p.g.D;
-  int grid = min(n_sm, p.n_items);
+  int grid = min(n_sm, (p.n_items + 1) / 2);
   if (grid < 1) grid = 1;
 #define BSA_LAUNCH_FWD(BSv, Dv)                                                                    \
   do {                                                                                             \
