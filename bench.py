@@ -56,7 +56,7 @@ KERNEL_NAMES = {"fwd": "bsa_fwd_kernel", "bwd_dkdv": "bsa_bwd_dkdv_kernel",
 # selected block pair (fwd, dq) or a pair with a current key block (dkdv).  Traffic grows with
 # the pairs a launch processes, so a full launch is scaled from it.  None = not captured for
 # the kernel as it now stands.
-DRAM_BYTES_PER_PAIR = {"fwd": 3840, "bwd_dkdv": 5762, "bwd_dq": 4842}
+DRAM_BYTES_PER_PAIR = {"fwd": 3998, "bwd_dkdv": 5762, "bwd_dq": 4842}
 
 
 def block_token_counts(g, frames: int) -> np.ndarray:
