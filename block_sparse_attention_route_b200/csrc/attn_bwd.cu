@@ -24,7 +24,7 @@
 namespace bsa {
 
 struct BwdWs {
-  size_t ndelta, nlse2, rev_off, rev_list, ctr, total;
+  size_t ndelta, nlse2, rev_off, rev_list, order, ctr, total;
 };
 inline size_t bwd_align(size_t x) { return (x + 255) & ~size_t(255); }
 BwdWs bwd_ws_layout(const Geo& g, int r) {
@@ -34,7 +34,8 @@ BwdWs bwd_ws_layout(const Geo& g, int r) {
   w.nlse2 = bwd_align(rows * 4);
   w.rev_off = w.nlse2 + bwd_align(rows * 4);
   w.rev_list = w.rev_off + bwd_align((size_t)g.B * g.H * (g.NBk + 1) * 4);
-  w.ctr = w.rev_list + bwd_align((size_t)g.B * g.H * g.NBq * r * 4);
+  w.order = w.rev_list + bwd_align((size_t)g.B * g.H * g.NBq * r * 4);
+  w.ctr = w.order + bwd_align((size_t)g.B * g.H * g.NBq * 4);
   w.total = w.ctr + 256;  // dK/dV work counter (one int, zeroed by the prep pass)
   return w;
 }
@@ -54,6 +55,7 @@ struct BwdParams {
   const int* cnt;
   const int* rev_off;     // [B*H][NBk+1]
   const int* rev_list;    // [B*H][NBq*r]
+  const int* order;       // [B*H][NBq]: each head's current key blocks, longest list first
   const float* ndelta;    // [B*H*NBq*BS] -Delta
   const float* nlse2;     // [B*H*NBq*BS] -LSE * log2(e), -inf for pad rows
   int* ctr;               // dkdv: next item to hand out (minus gridDim.x), zeroed by prep
@@ -105,11 +107,12 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(const __nv_bfloat16* __re
 // chunk's first position in each list; (3) each warp fills its chunk's entries in increasing
 // query-block order.  Lists come out ordered by i, deterministically and without atomics:
 // the entries of one row are distinct blocks, so the lanes handling a row touch distinct
-// counters.
+// counters.  (4) the head's current key blocks are ranked by decreasing list length into
+// `order`, the key-major pass's hand-out order.
 constexpr int kRevChunks = 8;
 constexpr int kRevThreads = 32 * kRevChunks;
 __global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams p, int* rev_off,
-                                                                int* rev_list) {
+                                                                int* rev_list, int* order) {
   // counts / cursors [kRevChunks][NBk], totals [NBk], scan scratch [kRevThreads]
   extern __shared__ int rsm[];
   const Geo& g = p.g;
@@ -177,6 +180,23 @@ __global__ void __launch_bounds__(kRevThreads) bwd_revidx_kernel(const BwdParams
     }
     __syncwarp();
   }
+  // (4) the head's current key blocks by decreasing list length (a counting sort; blocks of
+  // equal length in any order): the key-major pass hands its items out in this order within
+  // each head, so the longest lists start first and the pass does not end on a long one
+  __syncthreads();
+  int* hist = rsm;  // [NBq + 1] over the chunk counters, which are no longer needed
+  for (int e = tid; e <= g.NBq; e += kRevThreads) hist[e] = 0;
+  __syncthreads();
+  for (int jc = tid; jc < g.NBq; jc += kRevThreads) atomicAdd(&hist[min(tot[g.NBc + jc], g.NBq)], 1);
+  __syncthreads();
+  if (tid == 0) {
+    int pos = 0;
+    for (int len = g.NBq; len >= 0; --len) { const int v = hist[len]; hist[len] = pos; pos += v; }
+  }
+  __syncthreads();
+  int* ord = order + (size_t)bh * g.NBq;
+  for (int jc = tid; jc < g.NBq; jc += kRevThreads)
+    ord[atomicAdd(&hist[min(tot[g.NBc + jc], g.NBq)], 1)] = jc;
 }
 
 // ------------------------------------------------------------------------------ common
@@ -298,10 +318,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     end = off[1];
     if (beg < 0 || end < beg || end > g.NBq * p.r) { set_status(DEV_BAD_INDEX); beg = end = 0; }
   };
-  // Work distribution: items (key blocks) are handed out dynamically in their natural
-  // head-major order -- the first one per CTA is blockIdx.x, the rest come from a global
-  // counter -- so the CTAs finish together although items differ in steps (a key block is
-  // selected by anything from a few to a few hundred query blocks).  The producer fetches,
+  // Work distribution: items (key blocks) are handed out dynamically, head by head and within
+  // a head longest list first (the order the reverse index wrote) -- the first one per CTA
+  // is queue position blockIdx.x, the rest come from a global counter -- so the CTAs finish
+  // together although items differ in steps (a key block is selected by anything from a few
+  // to a few hundred query blocks), and the CTAs running at once share one head's Q / dO.  The producer fetches,
   // zero-fills empty items itself, and passes the non-empty ones (then -1) to the MMA thread
   // and the elementwise warps through a small queue in shared memory.
   auto read_item = [&](int k, bool elem) -> int {  // k-th queue entry; -1 = no more
@@ -321,8 +342,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       int q_loads = 0;               // slot loads issued (for the drain)
       bool ok = true;
       for (int k = 0; ok; ++k) {
-        // next non-empty item; empty ones get their zero dK / dV rows here
-        int item = k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.ctr, 1);
+        // next non-empty item; empty ones get their zero dK / dV rows here.  Queue position
+        // q is item (q / NBq) * NBq + order[q]: heads in turn, each head's longest lists first
+        auto queue_item = [&](int q) -> int {
+          if (q >= p.n_items) return p.n_items;
+          int jc = p.order[q];
+          if (jc < 0 || jc >= g.NBq) { set_status(DEV_BAD_INDEX); jc = 0; }
+          return (q / g.NBq) * g.NBq + jc;
+        };
+        int item = queue_item(k == 0 ? (int)blockIdx.x : (int)gridDim.x + atomicAdd(p.ctr, 1));
         int beg = 0, end = 0;
         while (item < p.n_items) {
           item_range(item, beg, end);
@@ -331,7 +359,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
           uint4* dk4 = reinterpret_cast<uint4*>(p.out0 + (size_t)item * BS * D);
           uint4* dv4 = reinterpret_cast<uint4*>(p.out1 + (size_t)item * BS * D);
           for (int c = 0; c < BS * D / 8; ++c) { dk4[c] = z; dv4[c] = z; }
-          item = (int)gridDim.x + atomicAdd(p.ctr, 1);
+          item = queue_item((int)gridDim.x + atomicAdd(p.ctr, 1));
         }
         const int slot = k % L::kQueue;
         if (k >= L::kQueue && !mbar_wait(&iq_empty[slot], ((k / L::kQueue) - 1) & 1, abort_flag)) {
@@ -1005,6 +1033,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
   float* nlse2 = reinterpret_cast<float*>(P.ws + w.nlse2);
   int* rev_off = reinterpret_cast<int*>(P.ws + w.rev_off);
   int* rev_list = reinterpret_cast<int*>(P.ws + w.rev_list);
+  int* order = reinterpret_cast<int*>(P.ws + w.order);
   int* ctr = reinterpret_cast<int*>(P.ws + w.ctr);
   const size_t rows = (size_t)g.B * g.H * g.NBq * g.BS;
   {
@@ -1028,6 +1057,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
   bp.cnt = P.cnt;
   bp.rev_off = rev_off;
   bp.rev_list = rev_list;
+  bp.order = order;
   bp.ndelta = ndelta;
   bp.nlse2 = nlse2;
   bp.ctr = ctr;
@@ -1036,7 +1066,7 @@ bsa_status_t run_bwd(const Geo& g, int r, const BwdPtrs& P, const BwdWs& w, cons
     if (cudaFuncSetAttribute(bwd_revidx_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
       return BSA_ERR_CUDA;
-    bwd_revidx_kernel<<<g.B * g.H, kRevThreads, smem, s>>>(bp, rev_off, rev_list);
+    bwd_revidx_kernel<<<g.B * g.H, kRevThreads, smem, s>>>(bp, rev_off, rev_list, order);
     if (cudaGetLastError() != cudaSuccess) return BSA_ERR_CUDA;
   }
   const int grid = max(1, min(n_sm, bp.n_items));

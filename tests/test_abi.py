@@ -47,8 +47,10 @@ def test_workspace_sizes_720p():
     bwd = bsa.bsa_workspace_size(g, 72, bsa.WS_BWD)
     up = lambda x: -(-x // 256) * 256  # noqa: E731
     rows = 32 * nbq * 128
-    # -Delta and -log2 LSE per query row, reverse-index offsets and lists, work counter
-    assert bwd == 2 * up(rows * 4) + up(32 * (nbq + 1) * 4) + up(32 * nbq * 72 * 4) + 256
+    # -Delta and -log2 LSE per query row, reverse-index offsets and lists, the key-major
+    # pass's hand-out order (one int per current key block), work counter
+    assert bwd == (2 * up(rows * 4) + up(32 * (nbq + 1) * 4) + up(32 * nbq * 72 * 4)
+                   + up(32 * nbq * 4) + 256)
 
 
 @pytest.mark.parametrize("bad", [dict(head_dim=96), dict(blk=(4, 4, 4)), dict(cached_t=3),
