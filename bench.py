@@ -51,12 +51,12 @@ def tile_flops(bs: int, d: int, n_pairs: int) -> float:
 KERNEL_NAMES = {"fwd": "bsa_fwd_kernel", "bwd_dkdv": "bsa_bwd_dkdv_kernel",
                 "bwd_dq": "bsa_bwd_dq_kernel"}
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) per unit of work, from one ncu
-# --set full capture of the kernel as it now stands on the 480p workload (365,568 pairs; the
-# attention-kernel summary under profiles/ holds the figures and the command); a unit is a
+# capture of the kernel as it now stands on the 480p workload (365,568 pairs; the
+# attention-kernel summary under profiles/ holds the figures and the commands); a unit is a
 # selected block pair (fwd, dq) or a pair with a current key block (dkdv).  Traffic grows with
 # the pairs a launch processes, so a full launch is scaled from it.  None = not captured for
 # the kernel as it now stands.
-DRAM_BYTES_PER_PAIR = {"fwd": 3998, "bwd_dkdv": 5762, "bwd_dq": 4842}
+DRAM_BYTES_PER_PAIR = {"fwd": 3998, "bwd_dkdv": 5752, "bwd_dq": 4842}
 
 
 def block_token_counts(g, frames: int) -> np.ndarray:
