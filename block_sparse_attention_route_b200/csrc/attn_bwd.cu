@@ -222,8 +222,8 @@ constexpr int kTile = 128;
 // queries (so the K16 slice kk of P^T sits at column 16kk, of dS^T at 16kk + 8) -- and
 // R[(g & 1) ^ 1] is free once dP^T(g) has been loaded: S^T(g+1) goes there while P^T(g),
 // dS^T(g) are being formed.
-// MMA order: S^T(g) | dK(g-1), dV(g-1), dP^T(g) | S^T(g+1) | ...; dP^T(g) reuses the region
-// that dK(g-1) and dV(g-1) read, after them in issue order.
+// MMA order: ... | dV(g-1) | S^T(g) | dK(g-1) | dP^T(g) | dV(g) | S^T(g+1) | ...; dP^T(g)
+// reuses the region that dV(g-1) and dK(g-1) read, after them in issue order.
 // Q_i and dO_i (with -lse2_i, -delta_i) share a 2-slot ring; a slot is released after dK(g),
 // its last reader.
 template <int BS, int D>
